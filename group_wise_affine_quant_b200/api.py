@@ -1,0 +1,146 @@
+"""Thin Python binding over the C ABI (include/aq.h), one function per entry
+point with the same name.  It only marshals arguments: torch tensors supply
+device memory and the current CUDA stream; every step of the computation runs
+in libaq.so's kernels.
+
+Tensors: x / w / y are fp16 or bf16 CUDA tensors; w_q is uint8 [N, K*bits/8];
+affine scales / biases are T [N, K/group_size]; FP4 scales are uint8.
+"""
+import torch
+
+from . import _lib
+from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, AQ_OP_QMM,
+                   AQ_OP_QMV, AqError, check, lib)
+
+__all__ = ["aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmm", "aq_qconv2d_nhwc",
+           "aq_workspace_size", "aq_last_error", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4",
+           "Workspace"]
+
+_DT = {torch.float16: AQ_F16, torch.bfloat16: AQ_BF16}
+_TORCH_DT = {AQ_F16: torch.float16, AQ_BF16: torch.bfloat16}
+
+
+def _dt(t):
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError("expected an fp16 or bf16 tensor, got %s" % t.dtype) from None
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device):
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _mode(scales):
+    return AQ_MODE_FP4 if scales.dtype == torch.uint8 else AQ_MODE_AFFINE
+
+
+class Workspace:
+    """Per-device zero-initialised scratch buffer, grown on demand.
+
+    The kernels leave their counters at zero after every call, so one buffer
+    serves all calls issued on one stream; calls on different streams need
+    different Workspace objects."""
+
+    def __init__(self):
+        self._bufs = {}
+
+    def get(self, device, nbytes):
+        if nbytes == 0:
+            return None
+        buf = self._bufs.get(device)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+            self._bufs[device] = buf
+        return buf
+
+
+_default_ws = Workspace()
+
+
+def aq_last_error():
+    return lib().aq_last_error().decode()
+
+
+def aq_workspace_size(op, M, N, K, bits, group_size, mode=AQ_MODE_AFFINE, groups=1):
+    return lib().aq_workspace_size(op, M, N, K, bits, group_size, mode, groups)
+
+
+def aq_quantize(w, bits=4, group_size=64, out=None):
+    """w [N, K] T -> (w_q uint8 [N, K*bits/8], scales T [N, G], biases T [N, G])."""
+    N, K = w.shape
+    if out is None:
+        G = K // group_size if group_size > 0 else 0
+        out = (torch.empty((N, K * bits // 8), dtype=torch.uint8, device=w.device),
+               torch.empty((N, G), dtype=w.dtype, device=w.device),
+               torch.empty((N, G), dtype=w.dtype, device=w.device))
+    w_q, s, b = out
+    check(lib().aq_quantize(_ptr(w), _ptr(w_q), _ptr(s), _ptr(b), N, K, bits, group_size, _dt(w),
+                            _stream(w.device)), "aq_quantize")
+    return w_q, s, b
+
+
+def aq_dequantize(w_q, scales, biases, K, bits=4, group_size=64, dtype=None, out=None):
+    """-> w_out T [N, K].  dtype defaults to the affine scales' dtype (bf16 for FP4)."""
+    mode = _mode(scales)
+    N = w_q.shape[0]
+    if dtype is None:
+        dtype = scales.dtype if mode == AQ_MODE_AFFINE else torch.bfloat16
+    if out is None:
+        out = torch.empty((N, K), dtype=dtype, device=w_q.device)
+    check(lib().aq_dequantize(_ptr(w_q), _ptr(scales), _ptr(biases), _ptr(out), N, K, bits,
+                              group_size, mode, _DT[dtype], _stream(w_q.device)), "aq_dequantize")
+    return out
+
+
+def _mm(fn_name, op, x, w_q, scales, biases, bits, group_size, out, workspace):
+    M, K = x.shape
+    N = w_q.shape[0]
+    mode = _mode(scales)
+    if out is None:
+        out = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    ws_bytes = aq_workspace_size(op, M, N, K, bits, group_size, mode)
+    ws = (workspace or _default_ws).get(x.device, ws_bytes)
+    fn = getattr(lib(), fn_name)
+    check(fn(_ptr(x), _ptr(w_q), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, bits,
+             group_size, mode, _dt(x), _ptr(ws), 0 if ws is None else ws.numel(),
+             _stream(x.device)), fn_name)
+    return out
+
+
+def aq_qmv(x, w_q, scales, biases, bits=4, group_size=64, out=None, workspace=None):
+    """y = x . dequant(w)^T for 1 <= M <= 16 rows of x."""
+    return _mm("aq_qmv", AQ_OP_QMV, x, w_q, scales, biases, bits, group_size, out, workspace)
+
+
+def aq_qmm(x, w_q, scales, biases, bits=4, group_size=64, out=None, workspace=None):
+    """y = x . dequant(w)^T for any M."""
+    return _mm("aq_qmm", AQ_OP_QMM, x, w_q, scales, biases, bits, group_size, out, workspace)
+
+
+def conv_out_hw(H, W, kh, kw, stride, pad):
+    return (H + 2 * pad[0] - kh) // stride[0] + 1, (W + 2 * pad[1] - kw) // stride[1] + 1
+
+
+def aq_qconv2d_nhwc(x, w_q, scales, biases, Cout, kh, kw, stride=(1, 1), pad=(0, 0), groups=1,
+                    bits=4, group_size=64, out=None, workspace=None):
+    """x [B, H, W, Cin] T -> y [B, Ho, Wo, Cout] T (weights as aq_qconv2d_nhwc documents)."""
+    B, H, W, Cin = x.shape
+    Ho, Wo = conv_out_hw(H, W, kh, kw, stride, pad)
+    if out is None:
+        out = torch.empty((B, Ho, Wo, Cout), dtype=x.dtype, device=x.device)
+    Cg = Cin // groups if groups > 0 else 0
+    Kp = -(-kh * kw * Cg // group_size) * group_size if group_size > 0 else 0
+    ws_bytes = aq_workspace_size(AQ_OP_QCONV2D, B * Ho * Wo, Cout // max(groups, 1), Kp, bits,
+                                 group_size, AQ_MODE_AFFINE, groups)
+    ws = (workspace or _default_ws).get(x.device, ws_bytes)
+    check(lib().aq_qconv2d_nhwc(_ptr(x), _ptr(w_q), _ptr(scales), _ptr(biases), _ptr(out), B, H,
+                                W, Cin, Cout, kh, kw, stride[0], stride[1], pad[0], pad[1],
+                                groups, bits, group_size, _dt(x), _ptr(ws),
+                                0 if ws is None else ws.numel(), _stream(x.device)),
+          "aq_qconv2d_nhwc")
+    return out

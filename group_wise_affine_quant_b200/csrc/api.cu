@@ -1,0 +1,181 @@
+// api.cu — the exported C ABI: argument validation, planning and dispatch.
+// Every entry point validates on the host before it enqueues anything and
+// reports failures through its return value and a thread-local message.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "common.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+aq_status fail(aq_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+aq_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return AQ_OK;
+  return fail(AQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+const int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+// Format checks shared by every entry point.
+aq_status check_format(int bits, int gs, aq_mode mode, aq_dtype dt) {
+  if (dt != AQ_F16 && dt != AQ_BF16) return fail(AQ_ERR_UNSUPPORTED, "dtype %d is not fp16 (0) or bf16 (1)", (int)dt);
+  if (mode == AQ_MODE_AFFINE) {
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 5 || bits == 6 || bits == 8))
+      return fail(AQ_ERR_UNSUPPORTED, "bits %d: affine mode supports 2, 3, 4, 5, 6 or 8", bits);
+    if (!(gs == 32 || gs == 64 || gs == 128))
+      return fail(AQ_ERR_UNSUPPORTED, "group_size %d: affine mode supports 32, 64 or 128", gs);
+  } else if (mode == AQ_MODE_FP4) {
+    if (bits != 4) return fail(AQ_ERR_UNSUPPORTED, "bits %d: FP4 mode has 4-bit codes", bits);
+    if (gs != 16 && gs != 32)
+      return fail(AQ_ERR_UNSUPPORTED, "group_size %d: FP4 mode supports 32 (E8M0) or 16 (E4M3)", gs);
+  } else {
+    return fail(AQ_ERR_UNSUPPORTED, "mode %d is not affine (0) or fp4 (1)", (int)mode);
+  }
+  return AQ_OK;
+}
+
+aq_status check_weight(const void* w_q, const void* scales, const void* biases, int64_t N,
+                       int64_t K, int bits, int gs, aq_mode mode, aq_dtype dt) {
+  aq_status st = check_format(bits, gs, mode, dt);
+  if (st != AQ_OK) return st;
+  if (N < 0 || K < 0 || N > kMaxDim || K > kMaxDim)
+    return fail(AQ_ERR_INVALID_ARG, "N=%lld K=%lld out of range", (long long)N, (long long)K);
+  if (K % gs) return fail(AQ_ERR_INVALID_ARG, "K=%lld is not a multiple of group_size %d", (long long)K, gs);
+  if (N > 0 && K > 0) {
+    if (!w_q || !scales) return fail(AQ_ERR_INVALID_ARG, "w_q and scales must not be NULL");
+    if (!aligned(w_q, 16)) return fail(AQ_ERR_MISALIGNED, "w_q must be 16-byte aligned");
+    if (mode == AQ_MODE_AFFINE) {
+      if (!biases) return fail(AQ_ERR_INVALID_ARG, "affine mode needs biases");
+      if (!aligned(scales, 2) || !aligned(biases, 2))
+        return fail(AQ_ERR_MISALIGNED, "scales and biases must be 2-byte aligned");
+    } else if (biases) {
+      return fail(AQ_ERR_INVALID_ARG, "FP4 mode takes no biases (pass NULL)");
+    }
+  }
+  return AQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* aq_last_error(void) { return g_err; }
+
+int aq_version(void) { return 100; }
+
+aq_status aq_quantize(const void* w, void* w_q, void* scales, void* biases, int64_t N,
+                      int64_t K, int bits, int group_size, aq_dtype dtype, aq_stream_t stream) {
+  g_err[0] = 0;
+  aq_status st = check_weight(w_q, scales, biases, N, K, bits, group_size, AQ_MODE_AFFINE, dtype);
+  if (st != AQ_OK) return st;
+  if (N == 0 || K == 0) return AQ_OK;
+  if (!w) return fail(AQ_ERR_INVALID_ARG, "w must not be NULL");
+  if (!aligned(w, 16)) return fail(AQ_ERR_MISALIGNED, "w must be 16-byte aligned");
+  return cuda_status(aq::launch_quantize(w, w_q, scales, biases, N, K, bits, group_size, dtype,
+                                         (cudaStream_t)stream),
+                     "aq_quantize launch");
+}
+
+aq_status aq_dequantize(const void* w_q, const void* scales, const void* biases, void* w_out,
+                        int64_t N, int64_t K, int bits, int group_size, aq_mode mode,
+                        aq_dtype dtype, aq_stream_t stream) {
+  g_err[0] = 0;
+  aq_status st = check_weight(w_q, scales, biases, N, K, bits, group_size, mode, dtype);
+  if (st != AQ_OK) return st;
+  if (N == 0 || K == 0) return AQ_OK;
+  if (!w_out) return fail(AQ_ERR_INVALID_ARG, "w_out must not be NULL");
+  if (!aligned(w_out, 16)) return fail(AQ_ERR_MISALIGNED, "w_out must be 16-byte aligned");
+  return cuda_status(aq::launch_dequantize(w_q, scales, biases, w_out, N, K, bits, group_size,
+                                           mode, dtype, (cudaStream_t)stream),
+                     "aq_dequantize launch");
+}
+
+static aq_status check_mm(const void* x, const void* y, int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || M > kMaxDim) return fail(AQ_ERR_INVALID_ARG, "M=%lld out of range", (long long)M);
+  if (M > 0 && N > 0) {
+    if (!y) return fail(AQ_ERR_INVALID_ARG, "y must not be NULL");
+    if (!aligned(y, 16)) return fail(AQ_ERR_MISALIGNED, "y must be 16-byte aligned");
+    if (K > 0) {
+      if (!x) return fail(AQ_ERR_INVALID_ARG, "x must not be NULL");
+      if (!aligned(x, 16)) return fail(AQ_ERR_MISALIGNED, "x must be 16-byte aligned");
+    }
+  }
+  return AQ_OK;
+}
+
+static aq_status zero_output(void* y, int64_t M, int64_t N, aq_stream_t stream) {
+  // K == 0: the empty sum is +0 in every output.
+  return cuda_status(cudaMemsetAsync(y, 0, (size_t)(M * N) * 2, (cudaStream_t)stream),
+                     "zero-fill of y");
+}
+
+aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void* biases,
+                 void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                 aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
+                 aq_stream_t stream) {
+  g_err[0] = 0;
+  aq_status st = check_weight(w_q, scales, biases, N, K, bits, group_size, mode, dtype);
+  if (st != AQ_OK) return st;
+  if (M < 1 || M > 16) return fail(AQ_ERR_INVALID_ARG, "aq_qmv takes 1 <= M <= 16 (got %lld)", (long long)M);
+  if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
+  if (N == 0) return AQ_OK;
+  if (K == 0) return zero_output(y, M, N, stream);
+  const aq::QmvPlan p = aq::plan_qmv(M, N, K, bits, group_size, mode);
+  if (p.ws_bytes) {
+    if (!workspace || workspace_bytes < p.ws_bytes)
+      return fail(AQ_ERR_WORKSPACE, "aq_qmv needs %zu workspace bytes (got %zu%s)", p.ws_bytes,
+                  workspace_bytes, workspace ? "" : ", NULL");
+    if (!aligned(workspace, 256)) return fail(AQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  }
+  return cuda_status(aq::launch_qmv(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
+                                    mode, dtype, workspace, (cudaStream_t)stream),
+                     "aq_qmv launch");
+}
+
+aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void* biases,
+                 void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                 aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
+                 aq_stream_t stream) {
+  g_err[0] = 0;
+  (void)x; (void)w_q; (void)scales; (void)biases; (void)y; (void)M; (void)N; (void)K;
+  (void)bits; (void)group_size; (void)mode; (void)dtype; (void)workspace;
+  (void)workspace_bytes; (void)stream;
+  return fail(AQ_ERR_UNSUPPORTED, "aq_qmm is not built yet");
+}
+
+aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* scales,
+                          const void* biases, void* y, int B, int H, int W, int Cin,
+                          int Cout, int kh, int kw, int stride_h, int stride_w, int pad_h,
+                          int pad_w, int groups, int bits, int group_size, aq_dtype dtype,
+                          void* workspace, size_t workspace_bytes, aq_stream_t stream) {
+  g_err[0] = 0;
+  (void)x; (void)w_q; (void)scales; (void)biases; (void)y; (void)B; (void)H; (void)W;
+  (void)Cin; (void)Cout; (void)kh; (void)kw; (void)stride_h; (void)stride_w; (void)pad_h;
+  (void)pad_w; (void)groups; (void)bits; (void)group_size; (void)dtype; (void)workspace;
+  (void)workspace_bytes; (void)stream;
+  return fail(AQ_ERR_UNSUPPORTED, "aq_qconv2d_nhwc is not built yet");
+}
+
+size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                         aq_mode mode, int groups) {
+  (void)groups;
+  if (M <= 0 || N <= 0 || K <= 0 || group_size <= 0 || K % group_size) return 0;
+  if (op == AQ_OP_QMV) {
+    if (M > 16) return 0;
+    return aq::plan_qmv(M, N, K, bits, group_size, mode).ws_bytes;
+  }
+  return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,175 @@
+/*
+ * aq.h — C ABI of the group-wise affine quantized matmul library for NVIDIA
+ * B200 (sm_100a).  libaq.so exports exactly the functions declared here.
+ *
+ * The operation (sources cited by page title and section):
+ *   y = x . dequant(w_q, scales, biases)^T
+ * "Add the 3bit packed qmm_t" (quantized_matmul with transpose=true): x is
+ * [M, K], the weight has N rows of K elements, y is [M, N].
+ *
+ * Weight format ("mlx 1.0.0, mlx/backend/cpu/quantized.cpp": quantize,
+ * get_pack_factor, get_bytes_per_pack, extract_bits, FP4_LUT,
+ * dequantize_scale):
+ *   - Affine mode: each row is cut into K/group_size groups of group_size
+ *     (32, 64, 128) consecutive elements; group g of row n has one scale
+ *     s[n, g] and one bias b[n, g] (dtype T) and codes q in [0, 2^bits - 1];
+ *     w_hat = s * q + b.  bits is 2, 3, 4, 5, 6 or 8.
+ *   - Packing: row n of w_q is K*bits/8 bytes.  Code k of the row occupies
+ *     bits [k*bits, (k+1)*bits) of the row read as a little-endian bit
+ *     stream.  For 2/4/8 bits this is 32/bits codes per uint32 word, low bits
+ *     first; 3- and 5-bit put 8 codes in 3 and 5 bytes, 6-bit puts 4 codes
+ *     in 3 bytes.
+ *   - FP4 mode: 4-bit E2M1 codes (2 per byte, low nibble first, value table
+ *     +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}) with one uint8 scale per group and no
+ *     bias: group_size 32 -> E8M0 scale (bf16 bit pattern s == 0 ? 0x40 :
+ *     s << 7, so 255 decodes to +inf), group_size 16 -> FP8 E4M3 scale (OCP
+ *     E4M3FN).  The scale is converted to T before use; w_hat = LUT[q] * s_T.
+ *   - scales / biases are [N, K/group_size] row-major.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer except aq_last_error's result is a DEVICE pointer owned
+ *     by the caller.  The library allocates nothing on the device, frees
+ *     nothing and retains no pointer after it returns.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream):
+ *     it validates its arguments on the host, enqueues kernels and returns
+ *     without synchronising.  Outputs are overwritten, never accumulated.
+ *   - Row-major dense layouts; leading dimensions equal the row lengths.
+ *   - Errors: a non-AQ_OK status is returned before anything is enqueued
+ *     (argument errors) or right after a launch fails (AQ_ERR_CUDA).  A
+ *     thread-local message is available from aq_last_error().  No call
+ *     throws, aborts or writes to stdout/stderr.
+ *   - Alignment: x, y and w (T data) 16 bytes; w_q 16 bytes; scales and
+ *     biases 2 bytes (1 byte in FP4 mode); workspace 256 bytes.
+ */
+#ifndef AQ_H_
+#define AQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AQ_API __attribute__((visibility("default")))
+#else
+#define AQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL is the default stream. */
+typedef struct CUstream_st* aq_stream_t;
+
+typedef enum {
+  AQ_OK = 0,
+  AQ_ERR_INVALID_ARG = 1,   /* shape, NULL pointer, or inconsistent sizes */
+  AQ_ERR_UNSUPPORTED = 2,   /* bits / group_size / dtype / mode outside the set */
+  AQ_ERR_MISALIGNED = 3,    /* a pointer below its required alignment */
+  AQ_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed */
+  AQ_ERR_WORKSPACE = 5      /* workspace NULL or smaller than aq_workspace_size */
+} aq_status;
+
+typedef enum { AQ_F16 = 0, AQ_BF16 = 1 } aq_dtype;
+
+typedef enum {
+  AQ_MODE_AFFINE = 0,       /* bits in {2,3,4,5,6,8}, group_size in {32,64,128} */
+  AQ_MODE_FP4 = 1           /* bits = 4; group_size 32 (E8M0) or 16 (E4M3); biases NULL */
+} aq_mode;
+
+typedef enum { AQ_OP_QMV = 0, AQ_OP_QMM = 1, AQ_OP_QCONV2D = 2 } aq_op;
+
+/*
+ * aq_quantize — affine group quantizer ("mlx 1.0.0, .../quantized.cpp",
+ * quantize; "Improvements in the quantizer and dequantization kernel",
+ * item 1).  Per group, in fp32 with IEEE division and ties-to-even rint:
+ *   lo, hi = min, max;  at_min = |lo| > |hi|
+ *   s = max((hi - lo) / (2^bits - 1), 1e-7), negated unless at_min
+ *   edge = at_min ? lo : hi;  q0 = rint(edge / s)
+ *   if q0 != 0: s = edge / q0, b = edge   (so 0 is exactly code -q0)
+ *   else:       b = 0
+ *   q = clamp(rint((w - b) / s), 0, 2^bits - 1);  store T(s), T(b)
+ * The scale is negative when the bias sits at the maximum.
+ *   w      [N, K] T (input)
+ *   w_q    [N, K*bits/8] bytes (output)
+ *   scales [N, K/group_size] T (output); biases likewise.
+ * Requires K % group_size == 0.  Affine mode only.
+ */
+AQ_API aq_status aq_quantize(const void* w, void* w_q, void* scales, void* biases, int64_t N,
+                      int64_t K, int bits, int group_size, aq_dtype dtype,
+                      aq_stream_t stream);
+
+/*
+ * aq_dequantize — writes w_out [N, K] T with every element rounded once
+ * (to nearest, ties to even) from the exact value s*q + b (affine) or
+ * LUT[q] * s_T (FP4).  Same weight arguments as aq_qmm.
+ */
+AQ_API aq_status aq_dequantize(const void* w_q, const void* scales, const void* biases, void* w_out,
+                        int64_t N, int64_t K, int bits, int group_size, aq_mode mode,
+                        aq_dtype dtype, aq_stream_t stream);
+
+/*
+ * aq_qmv — y = x . w_hat^T for small M (1 <= M <= 16): the weight-streaming
+ * path ("Add the 3bit packed qmm_t", affine_packed_qmv_fast, routed for few
+ * rows of x).  x [M, K] T, y [M, N] T, fp32 accumulation.  Split-K partial
+ * sums go to `workspace` (aq_workspace_size(AQ_OP_QMV, ...) bytes, which may
+ * be 0, in which case workspace may be NULL).  The workspace must be
+ * zero-filled once before its first use; every call leaves it ready for the
+ * next one.  Calls that share a workspace must not run concurrently.
+ * Returns AQ_ERR_INVALID_ARG for M outside 1..16.
+ */
+AQ_API aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void* biases,
+                 void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                 aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
+                 aq_stream_t stream);
+
+/*
+ * aq_qmm — y = x . w_hat^T for any M >= 1 ("Add the 3bit packed qmm_t",
+ * affine_packed_qmm_t): weight tiles are dequantized into shared memory in T
+ * and multiplied on the tensor cores with fp32 accumulation.  Arguments and
+ * workspace rules as aq_qmv.
+ */
+AQ_API aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void* biases,
+                 void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                 aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
+                 aq_stream_t stream);
+
+/*
+ * aq_qconv2d_nhwc — quantized 2-D convolution as an implicit GEMM
+ * ("[Feature] Quantized Convolution 2D - Possible PR?": quantize_weights and
+ * img2col followed by quantized_matmul), without materialising im2col.
+ *   x [B, H, W, Cin] T;  y [B, Ho, Wo, Cout] T with Ho = (H + 2 pad_h - kh) /
+ *   stride_h + 1 (likewise Wo).
+ *   Conv group g reads input channels [g Cg, (g+1) Cg), Cg = Cin / groups,
+ *   and writes output channels [g Ng, (g+1) Ng), Ng = Cout / groups.
+ *   Weight row co (of Cout) is the filter flattened in (kh, kw, Cg) order and
+ *   zero-padded to Kp = ceil(kh kw Cg / group_size) * group_size before it is
+ *   quantized with aq_quantize(N = Cout, K = Kp): w_q is [Cout, Kp*bits/8]
+ *   bytes, scales/biases [Cout, Kp/group_size].
+ *   Image borders and the K..Kp-1 pad read zero activations.  No conv bias.
+ * Affine mode only.  Workspace rules as aq_qmv (AQ_OP_QCONV2D sizing).
+ */
+AQ_API aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* scales,
+                          const void* biases, void* y, int B, int H, int W, int Cin,
+                          int Cout, int kh, int kw, int stride_h, int stride_w, int pad_h,
+                          int pad_w, int groups, int bits, int group_size, aq_dtype dtype,
+                          void* workspace, size_t workspace_bytes, aq_stream_t stream);
+
+/*
+ * aq_workspace_size — bytes of workspace the given call needs (0 if none).
+ * For AQ_OP_QCONV2D pass M = B*Ho*Wo, N = Cout / groups, K = Kp and the
+ * number of conv groups in `groups`; for the others pass groups = 1.
+ */
+AQ_API size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                         aq_mode mode, int groups);
+
+/* Message for the last non-AQ_OK status on the calling thread ("" if none). */
+AQ_API const char* aq_last_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+AQ_API int aq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQ_H_ */

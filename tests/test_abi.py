@@ -1,0 +1,106 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every symbol the header declares, and rejects bad arguments before it touches
+the device.  Pointers here are fake addresses that validation must refuse
+without dereferencing."""
+import ctypes
+
+import pytest
+
+from group_wise_affine_quant_b200 import _lib
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, CUDA, WORKSPACE = range(6)
+A = 0x10000  # a 16- and 256-byte aligned fake device address
+
+
+def L():
+    return _lib.lib()
+
+
+def test_exports_every_declared_symbol():
+    names = _lib.declared_symbols()
+    assert set(names) == set(_lib.SIGNATURES), names
+    for n in names:
+        assert hasattr(L(), n), n
+    assert L().aq_version() >= 100
+
+
+def _qmv(**kw):
+    a = dict(x=A, w_q=A, s=A, b=A, y=A, M=1, N=64, K=128, bits=4, gs=64, mode=0, dt=0,
+             ws=A, wsb=1 << 30)
+    a.update(kw)
+    return L().aq_qmv(a["x"], a["w_q"], a["s"], a["b"], a["y"], a["M"], a["N"], a["K"], a["bits"],
+                      a["gs"], a["mode"], a["dt"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("bits", [0, 1, 7, 9, 16])
+def test_unsupported_bits(bits):
+    assert _qmv(bits=bits) == UNSUPPORTED
+    assert b"bits" in L().aq_last_error()
+
+
+@pytest.mark.parametrize("gs", [0, 8, 16, 48, 256])
+def test_unsupported_group_affine(gs):
+    assert _qmv(gs=gs) == UNSUPPORTED
+
+
+def test_fp4_rules():
+    assert _qmv(mode=1, gs=64, b=None) == UNSUPPORTED
+    assert _qmv(mode=1, bits=8, gs=32, b=None) == UNSUPPORTED
+    assert _qmv(mode=1, gs=32, b=A) == INVALID        # FP4 takes no biases
+    assert _qmv(mode=2) == UNSUPPORTED
+
+
+def test_dtype_and_shape_errors():
+    assert _qmv(dt=2) == UNSUPPORTED
+    assert _qmv(K=96) == INVALID                       # not a multiple of 64
+    assert _qmv(M=0) == INVALID and _qmv(M=17) == INVALID
+    assert _qmv(N=-1) == INVALID
+    assert _qmv(b=None) == INVALID                     # affine needs biases
+    assert _qmv(x=None) == INVALID and _qmv(y=None) == INVALID
+
+
+def test_alignment_errors():
+    assert _qmv(x=A + 2) == MISALIGNED
+    assert _qmv(y=A + 8) == MISALIGNED
+    assert _qmv(w_q=A + 4) == MISALIGNED
+    assert _qmv(s=A + 1) == MISALIGNED
+
+
+def test_workspace_errors():
+    need = L().aq_workspace_size(0, 1, 64, 16384, 4, 64, 0, 1)
+    assert need > 0
+    assert _qmv(K=16384, ws=None, wsb=0) == WORKSPACE
+    assert _qmv(K=16384, wsb=need - 1) == WORKSPACE
+    assert _qmv(K=16384, ws=A + 16) == MISALIGNED
+    assert L().aq_workspace_size(0, 1, 64, 0, 4, 64, 0, 1) == 0
+    assert L().aq_workspace_size(0, 17, 64, 128, 4, 64, 0, 1) == 0
+
+
+def test_quantize_validation():
+    q = L().aq_quantize
+    assert q(A, A, A, A, 4, 64, 7, 64, 0, None) == UNSUPPORTED
+    assert q(A, A, A, A, 4, 96, 4, 64, 0, None) == INVALID
+    assert q(A + 2, A, A, A, 4, 64, 4, 64, 0, None) == MISALIGNED
+    assert q(None, A, A, A, 4, 64, 4, 64, 0, None) == INVALID
+    assert q(A, A, A, A, 0, 64, 4, 64, 0, None) == OK          # empty: nothing to do
+
+
+def test_dequantize_validation():
+    d = L().aq_dequantize
+    assert d(A, A, A, A + 8, 4, 64, 4, 64, 0, 0, None) == MISALIGNED
+    assert d(A, A, None, A, 4, 64, 4, 64, 0, 0, None) == INVALID
+    assert d(A, A, A, A, 4, 64, 4, 16, 0, 0, None) == UNSUPPORTED
+
+
+def test_error_message_is_thread_local_and_cleared():
+    assert _qmv(bits=7) == UNSUPPORTED
+    assert L().aq_last_error() != b""
+    assert L().aq_quantize(A, A, A, A, 0, 64, 4, 64, 0, None) == OK
+    assert L().aq_last_error() == b""
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        _lib.lib()

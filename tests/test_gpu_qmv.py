@@ -1,0 +1,130 @@
+"""GPU parity for aq_qmv against the oracle, within
+|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_affine_quant_b200 import api, inputs
+from tests.gpu_util import DEV, TDT, dev_u16, dev_u8, to_dev
+from tests.util import check_matmul
+
+pytestmark = pytest.mark.gpu
+
+BITS = (2, 3, 4, 5, 6, 8)
+
+
+def _case(M, N, K, bits, gs, dt, seed, wstd=0.05):
+    g = inputs.gen(seed)
+    w = inputs.normal((N, K), wstd, dt, g)
+    x = inputs.normal((M, K), 1.0, dt, g)
+    wq, s, b = api.aq_quantize(to_dev(w), bits, gs)
+    return to_dev(x), wq, s, b
+
+
+def _check(x, wq, s, b, y, bits, gs, dt, mode=0):
+    N = wq.shape[0]
+    sc = dev_u8(s) if mode == 1 else dev_u16(s)
+    bi = None if b is None else dev_u16(b)
+    yr, den = oracle.qmm(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt)
+    return check_matmul(dev_u16(y), yr, den, dt)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 13, 16])
+@pytest.mark.parametrize("bits", BITS)
+def test_qmv_affine_small(M, bits):
+    dt = 1 if M % 2 else 0
+    gs = {1: 32, 2: 64, 3: 128}[M % 3 + 1]
+    x, wq, s, b = _case(M, 100, 5 * 128, bits, gs, dt, seed=M * 10 + bits)
+    y = api.aq_qmv(x, wq, s, b, bits, gs)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, bits, gs, dt)
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("K", [32 * 3, 64 * 7, 4096 + 128, 16384])
+def test_qmv_ragged_and_split_k(bits, K):
+    """K slices that end mid-warp, and long K that splits across CTAs."""
+    gs = 32
+    M, N = 4, 72
+    x, wq, s, b = _case(M, N, K, bits, gs, 1, seed=K + bits)
+    y = api.aq_qmv(x, wq, s, b, bits, gs)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, bits, gs, 1)
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_qmv_workspace_reused_twice(M):
+    """Two calls in a row through the same workspace (tickets reset)."""
+    bits, gs, dt = 4, 64, 1
+    x, wq, s, b = _case(M, 512, 8192, bits, gs, dt, seed=5)
+    assert api.aq_workspace_size(api.AQ_OP_QMV if hasattr(api, "AQ_OP_QMV") else 0,
+                                 M, 512, 8192, bits, gs) > 0
+    ws = api.Workspace()
+    y1 = api.aq_qmv(x, wq, s, b, bits, gs, workspace=ws)
+    y2 = api.aq_qmv(x, wq, s, b, bits, gs, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    _check(x, wq, s, b, y2, bits, gs, dt)
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_qmv_tiny_config_fp16(M):
+    """Tiny correctness workload: 512 x 512, 4-bit g64, fp16, seed 0."""
+    x, w = inputs.tiny(M)
+    wq, s, b = api.aq_quantize(to_dev(w), 4, 64)
+    torch.cuda.synchronize()
+    rq, rs, rb = oracle.quantize(inputs.as_u16(w), 4, 64, 0)
+    assert np.array_equal(dev_u8(wq), rq)
+    y = api.aq_qmv(to_dev(x), wq, s, b, 4, 64)
+    torch.cuda.synchronize()
+    _check(to_dev(x), wq, s, b, y, 4, 64, 0)
+
+
+@pytest.mark.parametrize("name,N,K", inputs.LLAMA_1B_PROJ)
+@pytest.mark.parametrize("M", [1, 16])
+def test_qmv_decode_projection_full(name, N, K, M):
+    """Decode-sweep projections at full size, bf16 4-bit g64."""
+    x, wq, s, b = _case(M, N, K, 4, 64, 1, seed=N + K + M, wstd=0.02)
+    y = api.aq_qmv(x, wq, s, b, 4, 64)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, 4, 64, 1)
+
+
+@pytest.mark.parametrize("gs", [16, 32])
+@pytest.mark.parametrize("M", [1, 16])
+@pytest.mark.parametrize("dt", [0, 1])
+def test_qmv_fp4(gs, M, dt):
+    N, K = 96, 1024
+    codes, scales = inputs.fp4(N, K, gs, seed=gs + M)
+    x = inputs.normal((M, K), 1.0, dt, inputs.gen(M))
+    xd, wq, sc = to_dev(x), codes.to(DEV), scales.to(DEV)
+    y = api.aq_qmv(xd, wq, sc, None, 4, gs)
+    torch.cuda.synchronize()
+    _check(xd, wq, sc, None, y, 4, gs, dt, mode=1)
+
+
+def test_qmv_fp4_literal_scales_nonfinite():
+    """E8M0 scales over 0..254: rows with huge scales overflow to inf in the
+    same places as the oracle's exact result rounded to bf16."""
+    N, K, gs, M = 64, 1024, 32, 1
+    codes, scales = inputs.fp4(N, K, gs, scale_range="literal", seed=3)
+    x = inputs.fp4_x(M, K)
+    xd, wq, sc = to_dev(x), codes.to(DEV), scales.to(DEV)
+    y = api.aq_qmv(xd, wq, sc, None, 4, gs)
+    torch.cuda.synchronize()
+    _check(xd, wq, sc, None, y, 4, gs, 1, mode=1)
+
+
+def test_qmv_k_zero_and_n_zero():
+    x = torch.zeros((3, 0), dtype=torch.float16, device=DEV)
+    wq = torch.zeros((5, 0), dtype=torch.uint8, device=DEV)
+    s = torch.zeros((5, 0), dtype=torch.float16, device=DEV)
+    y = torch.full((3, 5), 9.0, dtype=torch.float16, device=DEV)
+    api.aq_qmv(x, wq, s, s, 4, 64, out=y)
+    torch.cuda.synchronize()
+    assert torch.all(y == 0)
+    x = torch.zeros((3, 64), dtype=torch.float16, device=DEV)
+    wq = torch.zeros((0, 32), dtype=torch.uint8, device=DEV)
+    s = torch.zeros((0, 1), dtype=torch.float16, device=DEV)
+    api.aq_qmv(x, wq, s, s, 4, 64)
