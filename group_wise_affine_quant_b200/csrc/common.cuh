@@ -95,8 +95,10 @@ struct QmvPlan {
   int lpr;         // lanes per weight row
   int rows_cta;    // weight rows per CTA
   int64_t row_blocks;
+  int ri;          // row groups per CTA
+  int chunk_units; // 32-code units of x staged at a time
   size_t smem;     // dynamic shared memory
-  size_t ws_bytes; // workspace (partials + counters), 0 if splits == 1
+  size_t ws_bytes; // workspace bytes (0: the cluster reduction needs none)
 };
 QmvPlan plan_qmv(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode);
 cudaError_t launch_qmv(const QmvPlan& p, const void* x, const void* w_q, const void* scales,

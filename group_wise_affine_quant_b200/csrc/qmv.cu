@@ -18,13 +18,19 @@
 //     row of x.  A 32-code unit never straddles an affine group (group_size
 //     >= 32); FP4 at group 16 applies one scale per 16-code half.
 //   * Lanes of a row combine by warp shuffles.  With more than one K-slice
-//     (split-K), each CTA writes fp32 partial sums to the workspace and the
-//     last CTA of a row block to finish (an atomic ticket) adds the slices in
-//     slice order and writes y; it then resets its ticket, so the workspace is
-//     ready for the next call.  No CTA waits for another.
+//     (split-K, up to 8 slices), the slices of a row block form one thread
+//     block cluster; each CTA keeps its fp32 row sums in shared memory and,
+//     after a cluster barrier, adds the slices' sums in slice order through
+//     distributed shared memory.  No workspace and no global atomics.
+//   * A CTA stages x once and then walks RI groups of rows, and each lane
+//     issues the load of its first weight unit before staging x.
+#include <cooperative_groups.h>
+
 #include <utility>
 
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace aq {
 namespace {
@@ -69,31 +75,49 @@ template <typename T, int BITS, int MT, bool FP4>
 __global__ void __launch_bounds__(kThreads)
 qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
            const void* __restrict__ scales_v, const T* __restrict__ biases, T* __restrict__ y,
-           float* __restrict__ partials, unsigned* __restrict__ counters, int M, int64_t N,
-           int64_t K, int gs, int64_t Ks, int S, int lpr_log2) {
+           int M, int64_t N, int64_t K, int gs, int64_t Ks, int S, int lpr_log2, int RI,
+           int chunk_units) {
   extern __shared__ float4 smem4[];
   float* smem = reinterpret_cast<float*>(smem4);
-  const int split = blockIdx.y;
-  const int64_t k0 = (int64_t)split * Ks;
-  const int64_t klen = (K - k0 < Ks) ? (K - k0) : Ks;        // multiple of 32
+  const int rank = blockIdx.y;                              // cluster spans all of y
+  const int64_t k0 = (int64_t)rank * Ks;
+  const int64_t klen = (K - k0 < Ks) ? (K - k0) : Ks;       // multiple of 32, > 0
   const int nunits = (int)(klen / kUnit);
-  const int units_max = (int)(Ks / kUnit);
-  const int xs_stride = units_max * kUnitStride;
-  float* xs = smem;                                         // [MT][xs_stride]
-  float* bs = smem + MT * xs_stride;                        // [MT][units_max]
   const int lpr = 1 << lpr_log2;
   const int rpw = 32 >> lpr_log2;
   const int rows_cta = (kThreads / 32) * rpw;
-  const int64_t row0 = (int64_t)blockIdx.x * rows_cta;
+  const int rows_blk = rows_cta * RI;
+  const int64_t row_base = (int64_t)blockIdx.x * rows_blk;
+  const int xs_stride = chunk_units * kUnitStride;
+  float* xs = smem;                                         // [MT][xs_stride]
+  float* bs = xs + MT * xs_stride;                          // [MT][chunk_units]
+  float* red = bs + MT * chunk_units;                       // [MT][rows_blk]
 
-  // Stage x[:, k0:k0+klen) as fp32 (rows m >= M read as zero).
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = lane >> lpr_log2, ul = lane & (lpr - 1);
+  const int64_t G = K / gs;
+  const int64_t row_bytes = K * BITS / 8;
+
+  // Prefetch this lane's first weight unit before staging x, so the HBM
+  // latency overlaps the staging.
+  uint32_t wd[BITS];
   {
-    const int per_row = (int)(klen / 8);
+    const int64_t row = row_base + warp * rpw + seg;
+    if (row < N && ul < nunits && ul < chunk_units)
+      load_unit<BITS>(wq + row * row_bytes + k0 * BITS / 8 + (int64_t)ul * (4 * BITS), wd);
+  }
+
+  for (int c0 = 0; c0 < nunits; c0 += chunk_units) {
+    const int cu = (nunits - c0 < chunk_units) ? (nunits - c0) : chunk_units;
+    if (c0) __syncthreads();                                // previous chunk fully consumed
+    // Stage x[:, k0 + 32 c0 : + 32 cu) as fp32 (rows m >= M are zero).
+    const int per_row = cu * (kUnit / 8);
     for (int i = threadIdx.x; i < MT * per_row; i += kThreads) {
       const int m = i / per_row, c8 = i - m * per_row;
       float f[8];
       if (m < M) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(x + (int64_t)m * K + k0 + c8 * 8);
+        const uint4 raw =
+            *reinterpret_cast<const uint4*>(x + (int64_t)m * K + k0 + (int64_t)c0 * kUnit + c8 * 8);
         const T* t = reinterpret_cast<const T*>(&raw);
 #pragma unroll
         for (int j = 0; j < 8; ++j) f[j] = TT<T>::to_f(t[j]);
@@ -108,106 +132,98 @@ qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
     }
     __syncthreads();
     if (!FP4) {
-      for (int i = threadIdx.x; i < MT * nunits; i += kThreads) {
-        const int m = i / nunits, u = i - m * nunits;
+      for (int i = threadIdx.x; i < MT * cu; i += kThreads) {
+        const int m = i / cu, u = i - m * cu;
         const float* src = xs + m * xs_stride + u * kUnitStride;
-        float s = 0.0f;
+        float sum = 0.0f;
 #pragma unroll
-        for (int j = 0; j < kUnit; ++j) s += src[j];
-        bs[m * units_max + u] = s;
+        for (int j = 0; j < kUnit; ++j) sum += src[j];
+        bs[m * chunk_units + u] = sum;
       }
+      __syncthreads();
     }
-    __syncthreads();
-  }
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int seg = lane >> lpr_log2, ul = lane & (lpr - 1);
-  const int64_t row = row0 + warp * rpw + seg;
-  const int64_t G = K / gs;
-  float acc[MT];
+    for (int ri = 0; ri < RI; ++ri) {
+      const int rloc = ri * rows_cta + warp * rpw + seg;
+      const int64_t row = row_base + rloc;
+      float acc[MT];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
-
-  if (row < N) {
-    const uint8_t* wrow = wq + row * (K * BITS / 8) + k0 * BITS / 8;
-    uint32_t wd[BITS];
-    if (ul < nunits) load_unit<BITS>(wrow + (int64_t)ul * (4 * BITS), wd);
-    for (int u = ul; u < nunits; u += lpr) {
-      uint32_t cur[BITS];
-#pragma unroll
-      for (int i = 0; i < BITS; ++i) cur[i] = wd[i];
-      if (u + lpr < nunits) load_unit<BITS>(wrow + (int64_t)(u + lpr) * (4 * BITS), wd);
-      const int64_t g = (k0 + (int64_t)u * kUnit) / gs;
-      // FP4 at group 16 has two scales per 32-code unit (halves lo / hi).
-      float s_lo, s_hi, b = 0.0f;
-      if constexpr (FP4) {
-        const uint8_t* sp = reinterpret_cast<const uint8_t*>(scales_v) + row * G;
-        s_lo = fp4_scale_t<T>(__ldg(sp + g), gs);
-        s_hi = gs == 16 ? fp4_scale_t<T>(__ldg(sp + g + 1), gs) : s_lo;
-      } else {
-        s_lo = s_hi = TT<T>::to_f(reinterpret_cast<const T*>(scales_v)[row * G + g]);
-        b = TT<T>::to_f(biases[row * G + g]);
-      }
-      float q[kUnit];
-      if constexpr (FP4) unpack_fp4(cur, q, std::make_integer_sequence<int, kUnit>{});
-      else unpack_affine<BITS>(cur, q, std::make_integer_sequence<int, kUnit>{});
-      const float* xu = xs + u * kUnitStride;
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const float4* xv = reinterpret_cast<const float4*>(xu + m * xs_stride);
-        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // [half][parity]
-#pragma unroll
-        for (int j = 0; j < kUnit / 4; ++j) {
-          const float4 a = xv[j];
-          const int h = (j >= kUnit / 8) ? 2 : 0;
-          d[h] = fmaf(a.x, q[4 * j + 0], d[h]);
-          d[h + 1] = fmaf(a.y, q[4 * j + 1], d[h + 1]);
-          d[h] = fmaf(a.z, q[4 * j + 2], d[h]);
-          d[h + 1] = fmaf(a.w, q[4 * j + 3], d[h + 1]);
+      for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+      if (row < N) {
+        const uint8_t* wrow = wq + row * row_bytes + (k0 + (int64_t)c0 * kUnit) * BITS / 8;
+        // the first unit of this row was prefetched (ri == 0, c0 == 0) or is loaded now
+        if (ri > 0 || c0 > 0) {
+          if (ul < cu) load_unit<BITS>(wrow + (int64_t)ul * (4 * BITS), wd);
         }
-        if constexpr (FP4) {
-          acc[m] = fmaf(s_lo, d[0] + d[1], acc[m]);
-          acc[m] = fmaf(s_hi, d[2] + d[3], acc[m]);
-        } else {
-          acc[m] = fmaf(s_lo, (d[0] + d[1]) + (d[2] + d[3]), acc[m]);
-          acc[m] = fmaf(b, bs[m * units_max + u], acc[m]);
+        for (int u = ul; u < cu; u += lpr) {
+          uint32_t cur[BITS];
+#pragma unroll
+          for (int i = 0; i < BITS; ++i) cur[i] = wd[i];
+          if (u + lpr < cu) load_unit<BITS>(wrow + (int64_t)(u + lpr) * (4 * BITS), wd);
+          const int64_t g = (k0 + (int64_t)(c0 + u) * kUnit) / gs;
+          // FP4 at group 16 has two scales per 32-code unit (halves lo / hi).
+          float s_lo, s_hi, b = 0.0f;
+          if constexpr (FP4) {
+            const uint8_t* sp = reinterpret_cast<const uint8_t*>(scales_v) + row * G;
+            s_lo = fp4_scale_t<T>(__ldg(sp + g), gs);
+            s_hi = gs == 16 ? fp4_scale_t<T>(__ldg(sp + g + 1), gs) : s_lo;
+          } else {
+            s_lo = s_hi = TT<T>::to_f(reinterpret_cast<const T*>(scales_v)[row * G + g]);
+            b = TT<T>::to_f(biases[row * G + g]);
+          }
+          float q[kUnit];
+          if constexpr (FP4) unpack_fp4(cur, q, std::make_integer_sequence<int, kUnit>{});
+          else unpack_affine<BITS>(cur, q, std::make_integer_sequence<int, kUnit>{});
+          const float* xu = xs + u * kUnitStride;
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const float4* xv = reinterpret_cast<const float4*>(xu + m * xs_stride);
+            float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // [half][parity]
+#pragma unroll
+            for (int j = 0; j < kUnit / 4; ++j) {
+              const float4 a = xv[j];
+              const int h = (j >= kUnit / 8) ? 2 : 0;
+              d[h] = fmaf(a.x, q[4 * j + 0], d[h]);
+              d[h + 1] = fmaf(a.y, q[4 * j + 1], d[h + 1]);
+              d[h] = fmaf(a.z, q[4 * j + 2], d[h]);
+              d[h + 1] = fmaf(a.w, q[4 * j + 3], d[h + 1]);
+            }
+            if constexpr (FP4) {
+              acc[m] = fmaf(s_lo, d[0] + d[1], acc[m]);
+              acc[m] = fmaf(s_hi, d[2] + d[3], acc[m]);
+            } else {
+              acc[m] = fmaf(s_lo, (d[0] + d[1]) + (d[2] + d[3]), acc[m]);
+              acc[m] = fmaf(b, bs[m * chunk_units + u], acc[m]);
+            }
+          }
         }
       }
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < MT; ++m)
-    for (int o = lpr >> 1; o; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
-
-  if (S == 1) {
-    if (ul == 0 && row < N) {
 #pragma unroll
       for (int m = 0; m < MT; ++m)
-        if (m < M) y[(int64_t)m * N + row] = TT<T>::from_f(acc[m]);
-    }
-    return;
-  }
-  if (ul == 0 && row < N) {
+        for (int o = lpr >> 1; o; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
+      if (ul == 0) {
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
-      if (m < M) partials[((int64_t)split * M + m) * N + row] = acc[m];
+        for (int m = 0; m < MT; ++m) red[m * rows_blk + rloc] = (c0 ? red[m * rows_blk + rloc] : 0.0f) + acc[m];
+      }
+    }
   }
-  __threadfence();
-  __syncthreads();
-  __shared__ unsigned ticket;
-  if (threadIdx.x == 0) ticket = atomicAdd(counters + blockIdx.x, 1u);
-  __syncthreads();
-  if (ticket != (unsigned)(S - 1)) return;
-  __threadfence();
-  for (int i = threadIdx.x; i < rows_cta * M; i += kThreads) {
-    const int m = i / rows_cta;
-    const int64_t r = row0 + (i - m * rows_cta);
-    if (r >= N) continue;
+
+  // Combine the K-slices: slice `rank` of the cluster finishes rows i with
+  // i % S == rank, adding the slices' sums in slice order through
+  // distributed shared memory.  Two cluster barriers: one before the reads,
+  // one so that no CTA exits while another still reads its shared memory.
+  cg::cluster_group cluster = cg::this_cluster();
+  if (S > 1) cluster.sync(); else __syncthreads();
+  for (int i = threadIdx.x; i < MT * rows_blk; i += kThreads) {
+    if (i % S != rank) continue;
+    const int m = i / rows_blk, rloc = i - m * rows_blk;
+    const int64_t row = row_base + rloc;
+    if (m >= M || row >= N) continue;
     float sum = 0.0f;
-    for (int s = 0; s < S; ++s) sum += __ldcg(partials + ((int64_t)s * M + m) * N + r);
-    y[(int64_t)m * N + r] = TT<T>::from_f(sum);
+    for (int q = 0; q < S; ++q) sum += (S > 1 ? cluster.map_shared_rank(red, q) : red)[i];
+    y[(int64_t)m * N + row] = TT<T>::from_f(sum);
   }
-  if (threadIdx.x == 0) counters[blockIdx.x] = 0u;
+  if (S > 1) cluster.sync();
 }
 
 int ilog2_floor(int64_t v) {
@@ -219,7 +235,7 @@ int ilog2_floor(int64_t v) {
 template <typename T, int BITS, int MT, bool FP4>
 cudaError_t launch_one(const QmvPlan& p, const void* x, const void* w_q, const void* scales,
                        const void* biases, void* y, int64_t M, int64_t N, int64_t K, int gs,
-                       void* ws, cudaStream_t st) {
+                       cudaStream_t st) {
   auto kern = qmv_kernel<T, BITS, MT, FP4>;
   if (p.smem > 48 * 1024) {
     static bool attr_done[64] = {};   // per instantiation and device
@@ -232,45 +248,48 @@ cudaError_t launch_one(const QmvPlan& p, const void* x, const void* w_q, const v
       if (dev < 64) attr_done[dev] = true;
     }
   }
-  float* partials = nullptr;
-  unsigned* counters = nullptr;
-  if (p.splits > 1) {
-    partials = reinterpret_cast<float*>(ws);
-    size_t off = ((size_t)p.splits * M * N * sizeof(float) + 255) & ~size_t(255);
-    counters = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(ws) + off);
-  }
-  dim3 grid((unsigned)p.row_blocks, (unsigned)p.splits);
-  kern<<<grid, kThreads, p.smem, st>>>((const T*)x, (const uint8_t*)w_q, scales,
-                                       (const T*)biases, (T*)y, partials, counters, (int)M, N, K,
-                                       gs, p.ks, p.splits, ilog2_floor(p.lpr));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.row_blocks, (unsigned)p.splits, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)p.splits;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, (const T*)x, (const uint8_t*)w_q, scales,
+                            (const T*)biases, (T*)y, (int)M, N, K, gs, p.ks, p.splits,
+                            ilog2_floor(p.lpr), p.ri, p.chunk_units);
 }
 
 template <typename T, int BITS, bool FP4>
 cudaError_t by_mt(const QmvPlan& p, const void* x, const void* w_q, const void* scales,
-                  const void* biases, void* y, int64_t M, int64_t N, int64_t K, int gs, void* ws,
+                  const void* biases, void* y, int64_t M, int64_t N, int64_t K, int gs,
                   cudaStream_t st) {
   switch (p.mt) {
-    case 1: return launch_one<T, BITS, 1, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    case 2: return launch_one<T, BITS, 2, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    case 4: return launch_one<T, BITS, 4, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    case 8: return launch_one<T, BITS, 8, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    default: return launch_one<T, BITS, 16, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
+    case 1: return launch_one<T, BITS, 1, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 2: return launch_one<T, BITS, 2, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 4: return launch_one<T, BITS, 4, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 8: return launch_one<T, BITS, 8, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    default: return launch_one<T, BITS, 16, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
   }
 }
 
 template <typename T>
 cudaError_t by_bits(const QmvPlan& p, const void* x, const void* w_q, const void* scales,
                     const void* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
-                    int gs, int mode, void* ws, cudaStream_t st) {
-  if (mode == AQ_MODE_FP4) return by_mt<T, 4, true>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
+                    int gs, int mode, cudaStream_t st) {
+  if (mode == AQ_MODE_FP4) return by_mt<T, 4, true>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
   switch (bits) {
-    case 2: return by_mt<T, 2, false>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    case 3: return by_mt<T, 3, false>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    case 4: return by_mt<T, 4, false>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    case 5: return by_mt<T, 5, false>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    case 6: return by_mt<T, 6, false>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
-    case 8: return by_mt<T, 8, false>(p, x, w_q, scales, biases, y, M, N, K, gs, ws, st);
+    case 2: return by_mt<T, 2, false>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 3: return by_mt<T, 3, false>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 4: return by_mt<T, 4, false>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 5: return by_mt<T, 5, false>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 6: return by_mt<T, 6, false>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 8: return by_mt<T, 8, false>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -282,40 +301,51 @@ QmvPlan plan_qmv(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
   QmvPlan p{};
   p.mt = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
   const int64_t units = K / kUnit;
-  const int64_t max_units = (16384 / p.mt) / kUnit;        // shared-memory bound on Ks
+  // Shared memory per staged unit and row of x: 36 floats + 1 sum.
+  const int64_t smem_cap = 160 * 1024;
+  const int64_t cap_units = smem_cap / ((int64_t)p.mt * (kUnitStride + 1) * 4);
   const int64_t target_ctas = 2 * 148;
-  int64_t S = (units + max_units - 1) / max_units;
-  if (S < 1) S = 1;
+  // Split K over up to 8 CTAs of a cluster until there are enough CTAs.
+  int64_t S = 1, us = units;
   for (;;) {
-    const int64_t us = (units + S - 1) / S;                // units per slice
-    p.ks = us * kUnit;
-    p.splits = (int)((units + us - 1) / us);
+    us = (units + S - 1) / S;
     int64_t l = 1;
     while (l * 2 <= us && l * 2 <= 32) l *= 2;
-    p.lpr = (int)l;
-    p.rows_cta = (kThreads / 32) * (32 / p.lpr);
-    p.row_blocks = (N + p.rows_cta - 1) / p.rows_cta;
-    if (p.row_blocks * p.splits >= target_ctas || us <= 8) break;
+    const int64_t rows_cta = (kThreads / 32) * (32 / l);
+    const int64_t rb = (N + rows_cta - 1) / rows_cta;
+    const bool fits = us <= cap_units;
+    if ((rb * S >= target_ctas && fits) || S == 8 || us <= 8) break;
     ++S;
   }
-  if (p.row_blocks < 1) p.row_blocks = 1;
-  const int64_t umax = p.ks / kUnit;
-  p.smem = (size_t)p.mt * (umax * kUnitStride + umax) * sizeof(float);
-  p.ws_bytes = 0;
-  if (p.splits > 1) {
-    size_t part = ((size_t)p.splits * M * N * sizeof(float) + 255) & ~size_t(255);
-    p.ws_bytes = part + (((size_t)p.row_blocks * sizeof(unsigned) + 255) & ~size_t(255));
+  p.ks = us * kUnit;
+  p.splits = (int)((units + us - 1) / us);
+  int64_t l = 1;
+  while (l * 2 <= us && l * 2 <= 32) l *= 2;
+  p.lpr = (int)l;
+  p.rows_cta = (kThreads / 32) * (32 / p.lpr);
+  p.chunk_units = (int)(us < cap_units ? us : cap_units);
+  // Several row groups per CTA (x staged once) when the slice fits in one
+  // chunk and there are CTAs to spare.
+  const int64_t rb1 = (N + p.rows_cta - 1) / p.rows_cta;
+  p.ri = 1;
+  if (p.chunk_units >= us) {
+    while (p.ri < 8 && (rb1 + 2 * p.ri - 1) / (2 * p.ri) * p.splits >= target_ctas) p.ri *= 2;
   }
+  p.row_blocks = (N + (int64_t)p.rows_cta * p.ri - 1) / ((int64_t)p.rows_cta * p.ri);
+  if (p.row_blocks < 1) p.row_blocks = 1;
+  p.smem = (size_t)p.mt * ((size_t)p.chunk_units * kUnitStride + p.chunk_units +
+                           (size_t)p.rows_cta * p.ri) * sizeof(float);
+  p.ws_bytes = 0;
   return p;
 }
 
 cudaError_t launch_qmv(const QmvPlan& p, const void* x, const void* w_q, const void* scales,
                        const void* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                        int gs, int mode, int dtype, void* ws, cudaStream_t st) {
+  (void)ws;
   return dtype == AQ_F16
-             ? by_bits<__half>(p, x, w_q, scales, biases, y, M, N, K, bits, gs, mode, ws, st)
-             : by_bits<__nv_bfloat16>(p, x, w_q, scales, biases, y, M, N, K, bits, gs, mode, ws,
-                                      st);
+             ? by_bits<__half>(p, x, w_q, scales, biases, y, M, N, K, bits, gs, mode, st)
+             : by_bits<__nv_bfloat16>(p, x, w_q, scales, biases, y, M, N, K, bits, gs, mode, st);
 }
 
 }  // namespace aq

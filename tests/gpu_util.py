@@ -26,9 +26,21 @@ def u16_to_dev(a, dt):
     return torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(TDT[dt]).to(DEV)
 
 
-def assert_equal_bits(got, want, what):
+def canon_nan(a, dt):
+    """Map every NaN pattern of T to one value (a NaN has no unique encoding)."""
+    a = np.array(a, dtype=np.uint16, copy=True)
+    exp = 0x7C00 if dt == 0 else 0x7F80
+    frac = 0x03FF if dt == 0 else 0x007F
+    nan = ((a & exp) == exp) & ((a & frac) != 0)
+    a[nan] = 0x7FFF
+    return a
+
+
+def assert_equal_bits(got, want, what, nan_dt=None):
     got = np.asarray(got)
     want = np.asarray(want)
+    if nan_dt is not None:
+        got, want = canon_nan(got, nan_dt), canon_nan(want, nan_dt)
     assert got.shape == want.shape, (what, got.shape, want.shape)
     if not np.array_equal(got, want):
         bad = np.argwhere(got != want)

@@ -66,14 +66,12 @@ def test_alignment_errors():
     assert _qmv(s=A + 1) == MISALIGNED
 
 
-def test_workspace_errors():
-    need = L().aq_workspace_size(0, 1, 64, 16384, 4, 64, 0, 1)
-    assert need > 0
-    assert _qmv(K=16384, ws=None, wsb=0) == WORKSPACE
-    assert _qmv(K=16384, wsb=need - 1) == WORKSPACE
-    assert _qmv(K=16384, ws=A + 16) == MISALIGNED
+def test_qmv_needs_no_workspace():
+    """qmv reduces its K-slices inside a thread block cluster: no workspace."""
+    for M in (1, 7, 16):
+        for K in (64, 16384, 1 << 20):
+            assert L().aq_workspace_size(0, M, 4096, K, 4, 64, 0, 1) == 0
     assert L().aq_workspace_size(0, 1, 64, 0, 4, 64, 0, 1) == 0
-    assert L().aq_workspace_size(0, 17, 64, 128, 4, 64, 0, 1) == 0
 
 
 def test_quantize_validation():

@@ -54,18 +54,25 @@ def test_qmv_ragged_and_split_k(bits, K):
 
 
 @pytest.mark.parametrize("M", [1, 16])
-def test_qmv_workspace_reused_twice(M):
-    """Two calls in a row through the same workspace (tickets reset)."""
+def test_qmv_split_k_twice_in_a_row(M):
+    """Long K splits over a cluster of CTAs; two calls give identical results."""
     bits, gs, dt = 4, 64, 1
     x, wq, s, b = _case(M, 512, 8192, bits, gs, dt, seed=5)
-    assert api.aq_workspace_size(api.AQ_OP_QMV if hasattr(api, "AQ_OP_QMV") else 0,
-                                 M, 512, 8192, bits, gs) > 0
-    ws = api.Workspace()
-    y1 = api.aq_qmv(x, wq, s, b, bits, gs, workspace=ws)
-    y2 = api.aq_qmv(x, wq, s, b, bits, gs, workspace=ws)
+    y1 = api.aq_qmv(x, wq, s, b, bits, gs)
+    y2 = api.aq_qmv(x, wq, s, b, bits, gs)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
     _check(x, wq, s, b, y2, bits, gs, dt)
+
+
+@pytest.mark.parametrize("M", [1, 3, 16])
+def test_qmv_very_long_k_chunked(M):
+    """K beyond one shared-memory chunk per slice (x staged in chunks)."""
+    bits, gs, dt = 4, 128, 0
+    x, wq, s, b = _case(M, 40, 65536 + 128, bits, gs, dt, seed=9, wstd=0.01)
+    y = api.aq_qmv(x, wq, s, b, bits, gs)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, bits, gs, dt)
 
 
 @pytest.mark.parametrize("M", [1, 8])
