@@ -31,6 +31,7 @@ SIGNATURES = {
     "aq_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I, _I, _I, _I]),
     "aq_last_error": (ctypes.c_char_p, []),
     "aq_version": (_I, []),
+    "aq_device_errors": (ctypes.c_uint, []),
 }
 
 _lib = None

@@ -148,10 +148,22 @@ aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void*
                  aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
                  aq_stream_t stream) {
   g_err[0] = 0;
-  (void)x; (void)w_q; (void)scales; (void)biases; (void)y; (void)M; (void)N; (void)K;
-  (void)bits; (void)group_size; (void)mode; (void)dtype; (void)workspace;
-  (void)workspace_bytes; (void)stream;
-  return fail(AQ_ERR_UNSUPPORTED, "aq_qmm is not built yet");
+  (void)workspace; (void)workspace_bytes;
+  aq_status st = check_weight(w_q, scales, biases, N, K, bits, group_size, mode, dtype);
+  if (st != AQ_OK) return st;
+  if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
+  if (M == 0 || N == 0) return AQ_OK;
+  if (K == 0) return zero_output(y, M, N, stream);
+  const aq::QmmPlan p = aq::plan_qmm(M, N, K, bits, group_size, mode);
+  return cuda_status(aq::launch_qmm(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
+                                    mode, dtype, (cudaStream_t)stream),
+                     "aq_qmm launch");
+}
+
+unsigned aq_device_errors(void) {
+  unsigned v = 0;
+  if (aq::read_device_error(&v) != cudaSuccess) return 0xFFFFFFFFu;
+  return v;
 }
 
 aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* scales,

@@ -104,4 +104,18 @@ QmvPlan plan_qmv(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode);
 cudaError_t launch_qmv(const QmvPlan& p, const void* x, const void* w_q, const void* scales,
                        const void* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                        int gs, int mode, int dtype, void* ws, cudaStream_t st);
+
+struct QmmPlan {
+  int bt;          // x rows per tile (MMA N)
+  int64_t n_tiles; // weight row tiles of 128
+  int64_t m_tiles; // x row tiles of bt
+  int k_tiles;     // K / 64 rounded up
+  int k_tiles_split;
+  int splits;      // K-slices, one cluster per output tile
+};
+QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode);
+cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const void* scales,
+                       const void* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+                       int gs, int mode, int dtype, cudaStream_t st);
+cudaError_t read_device_error(unsigned* out);
 }  // namespace aq

@@ -1,0 +1,643 @@
+// qmm.cu — tensor-core quantized matmul y = x . dequant(W)^T (tcgen05 + TMEM).
+//
+// Prior art: affine_packed_qmm_t in "Add the 3bit packed qmm_t" (a block
+// loader dequantizes a weight tile into threadgroup memory, then a simdgroup
+// MMA).  The B200 design, per CTA and output tile of 128 weight rows x BT
+// rows of x:
+//   * The weight is the MMA's A operand (M = 128 rows of N) and x is the B
+//     operand (N = BT in 16..256 rows of M), so a decode-sized M still fills a
+//     full 128-row MMA: one wave of tiles covers M = 1..64 at the weight
+//     stream's cost.
+//   * Warp 0 (one thread) loads x tiles with TMA into 128-byte-swizzled shared
+//     memory; warp 1 allocates TMEM and one of its threads issues
+//     tcgen05.mma (kind::f16, fp32 accumulate in TMEM); warps 2-5 are the
+//     dequantizers (one weight row per thread): they stream packed codes and
+//     the group's scale and bias from global memory several stages ahead in
+//     registers, form w_hat = s*q + b in T with packed half2/bfloat162 FMAs
+//     (single rounding, the same value aq_dequantize writes), and store it in
+//     the same swizzled K-major layout.  Stages hand over through mbarriers;
+//     the MMA's commit frees a stage for both producers.
+//   * K-step 64 (one 128-byte swizzle atom of 16-bit values); a K tail of 32
+//     reads zero x through TMA's out-of-bounds fill and writes zero w_hat.
+//   * The epilogue (warps 2-5) reads TMEM with tcgen05.ld.  With split-K the
+//     K-slices of a tile form a thread block cluster: each CTA parks its fp32
+//     tile in shared memory and the slices are added in slice order through
+//     distributed shared memory.  No workspace, no global atomics.
+//   * Every mbarrier wait is bounded (2 s); a timeout sets a device error
+//     flag, every role stops issuing work and the CTA frees its TMEM.
+#include <cooperative_groups.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace aq {
+
+__device__ unsigned int g_aq_device_error = 0u;   // bit 0: a wait timed out
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBK = 64;                  // K elements per stage (128 bytes of T)
+constexpr int kRowsW = 128;              // weight rows per tile (MMA M)
+constexpr int kThreads = 192;            // 6 warps
+constexpr int kProducerWarp0 = 2;        // warps 2..5 dequantize and run the epilogue
+constexpr int kPrefetch = 4;             // stages of packed codes in flight per thread
+
+template <int BT>
+struct QmmShape {
+  static constexpr int kStages = BT >= 256 ? 3 : BT >= 128 ? 4 : 6;
+  static constexpr int kABytes = kRowsW * kBK * 2;          // 16 KB
+  static constexpr int kBBytes = BT * kBK * 2;              // BT * 128
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kRedBytes = BT * kRowsW * 4;          // split-K parking
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kDataBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
+  static constexpr int kTmemCols = BT < 32 ? 32 : BT;
+  // 1024 for alignment slack + data + barriers
+  static constexpr int kSmem = 1024 + kDataBytes + 256;
+};
+
+struct QmmArgs {
+  const uint8_t* wq;
+  const void* scales;
+  const void* biases;
+  void* y;
+  int M, N, K;
+  int gs_log2;
+  int k_tiles;          // ceil(K / 64)
+  int k_tiles_split;    // k-tiles per split
+  int splits;
+  int narrow;           // 1: 4-byte weight loads (row stride not 16-byte aligned)
+  int64_t row_bytes;
+};
+
+// ------------------------------------------------------------- dequantizer
+// Per thread and stage: the 64 codes of one weight row as 2*BITS words.
+template <int BITS>
+struct Packed {
+  static constexpr int kWords = 2 * BITS;
+  uint32_t w[kWords];
+};
+
+template <int BITS>
+__device__ __forceinline__ void load_packed(Packed<BITS>& p, const uint8_t* src, bool full,
+                                            bool narrow) {
+  // src: 8*BITS bytes (full stage) or 4*BITS bytes (K tail of 32 codes).
+  // Vector loads need the row stride K*bits/8 to be a multiple of 16 bytes
+  // (8 for 3/5-bit); otherwise (`narrow`) 4-byte loads, which every row and
+  // stage offset satisfies since K % 32 == 0.
+  if (full && narrow) {
+#pragma unroll
+    for (int i = 0; i < 2 * BITS; ++i) p.w[i] = __ldg(reinterpret_cast<const uint32_t*>(src) + i);
+  } else if (full) {
+    if constexpr (BITS == 2 || BITS == 4 || BITS == 6 || BITS == 8) {
+#pragma unroll
+      for (int i = 0; i < BITS / 2; ++i) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+        p.w[4 * i] = v.x; p.w[4 * i + 1] = v.y; p.w[4 * i + 2] = v.z; p.w[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < BITS; ++i) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + i);
+        p.w[2 * i] = v.x; p.w[2 * i + 1] = v.y;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) p.w[i] = __ldg(reinterpret_cast<const uint32_t*>(src) + i);
+#pragma unroll
+    for (int i = BITS; i < 2 * BITS; ++i) p.w[i] = 0u;
+  }
+}
+
+template <typename T> struct Pair;
+template <> struct Pair<__half> {
+  static constexpr uint32_t kMagic = 0x64006400u;            // 1024.0 in each half
+  static __device__ __forceinline__ uint32_t sub_magic(uint32_t v) {
+    __half2 h = *reinterpret_cast<__half2*>(&v);
+    h = __hsub2(h, __half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ uint32_t fma(uint32_t q, uint32_t s, uint32_t b) {
+    __half2 r = __hfma2(*reinterpret_cast<__half2*>(&q), *reinterpret_cast<__half2*>(&s),
+                        *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+  static __device__ __forceinline__ uint32_t mul(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+  static __device__ __forceinline__ uint32_t from_f2(float lo, float hi) {
+    __half2 r = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+  static constexpr int kMagicMaxCode = 1023;
+};
+template <> struct Pair<__nv_bfloat16> {
+  static constexpr uint32_t kMagic = 0x43004300u;            // 128.0 in each half
+  static __device__ __forceinline__ uint32_t sub_magic(uint32_t v) {
+    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
+    h = __hsub2(h, __nv_bfloat162(__ushort_as_bfloat16(0x4300), __ushort_as_bfloat16(0x4300)));
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ uint32_t fma(uint32_t q, uint32_t s, uint32_t b) {
+    __nv_bfloat162 r = __hfma2(*reinterpret_cast<__nv_bfloat162*>(&q),
+                               *reinterpret_cast<__nv_bfloat162*>(&s),
+                               *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+  static __device__ __forceinline__ uint32_t mul(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+  static __device__ __forceinline__ uint32_t from_f2(float lo, float hi) {
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+  }
+  static constexpr int kMagicMaxCode = 127;
+};
+
+// Exact codes of elements (2j, 2j+1) of chunk c as a T pair.
+template <typename T, int BITS, int C, int J>
+__device__ __forceinline__ uint32_t code_pair(const Packed<BITS>& p) {
+  constexpr int k0 = 8 * C + 2 * J;
+  if constexpr (BITS == 4) {
+    // byte J of word C holds codes 2J (low nibble) and 2J+1 (high nibble):
+    // put byte J of w at byte 0 and byte J of w >> 4 at byte 2, keep the low
+    // nibbles, OR in the magic exponent and subtract it.
+    const uint32_t w = p.w[C];
+    constexpr uint32_t sel = (uint32_t)J | ((uint32_t)J << 4) | ((uint32_t)(J + 4) << 8) |
+                             ((uint32_t)(J + 4) << 12);
+    const uint32_t t = __byte_perm(w, w >> 4, sel);
+    return Pair<T>::sub_magic((t & 0x000F000Fu) | Pair<T>::kMagic);
+  } else if constexpr (BITS == 8 && std::is_same<T, __nv_bfloat16>::value) {
+    const float lo = u_to_f_exact(code_at<8, k0>(p.w));
+    const float hi = u_to_f_exact(code_at<8, k0 + 1>(p.w));
+    return Pair<T>::from_f2(lo, hi);
+  } else {
+    const uint32_t lo = code_at<BITS, k0>(p.w);
+    const uint32_t hi = code_at<BITS, k0 + 1>(p.w);
+    return Pair<T>::sub_magic(lo | (hi << 16) | Pair<T>::kMagic);
+  }
+}
+
+template <typename T, int C, int J>
+__device__ __forceinline__ uint32_t fp4_pair(const Packed<4>& p) {
+  constexpr int k0 = 8 * C + 2 * J;
+  return Pair<T>::from_f2(e2m1_to_float(code_at<4, k0>(p.w)), e2m1_to_float(code_at<4, k0 + 1>(p.w)));
+}
+
+// Dequantize chunk C (8 elements) into 16 bytes.
+template <typename T, int BITS, bool FP4, int C>
+__device__ __forceinline__ uint4 dequant_chunk(const Packed<BITS>& p, uint32_t s2, uint32_t b2) {
+  uint4 o;
+  if constexpr (FP4) {
+    o.x = Pair<T>::mul(fp4_pair<T, C, 0>(p), s2);
+    o.y = Pair<T>::mul(fp4_pair<T, C, 1>(p), s2);
+    o.z = Pair<T>::mul(fp4_pair<T, C, 2>(p), s2);
+    o.w = Pair<T>::mul(fp4_pair<T, C, 3>(p), s2);
+  } else {
+    o.x = Pair<T>::fma(code_pair<T, BITS, C, 0>(p), s2, b2);
+    o.y = Pair<T>::fma(code_pair<T, BITS, C, 1>(p), s2, b2);
+    o.z = Pair<T>::fma(code_pair<T, BITS, C, 2>(p), s2, b2);
+    o.w = Pair<T>::fma(code_pair<T, BITS, C, 3>(p), s2, b2);
+  }
+  return o;
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t splat(T v) {
+  const uint16_t u = *reinterpret_cast<const uint16_t*>(&v);
+  return (uint32_t)u | ((uint32_t)u << 16);
+}
+
+// Scale/bias pairs (splatted T) for the two 32-element halves of a stage.
+struct StageSB {
+  uint32_t s[2], b[2];
+};
+
+template <typename T, bool FP4>
+__device__ __forceinline__ StageSB load_sb(const QmmArgs& a, int64_t row, int kt, int G, bool tail) {
+  StageSB r;
+  const int k = kt * kBK;
+  const int g0 = k >> a.gs_log2;
+  // the upper half of a K-tail stage has no group (and must not be read)
+  const int g1 = tail ? g0 : (k + 32) >> a.gs_log2;
+  if constexpr (FP4) {
+    const uint8_t* sp = reinterpret_cast<const uint8_t*>(a.scales) + row * G;
+    const int gs = 1 << a.gs_log2;
+    // group 16: four groups per stage; each 16-element quarter gets its own
+    // scale, handled by the caller through s[] = quarters (0,1) and b[] = (2,3)
+    if (gs == 16) {
+      const int g2 = tail ? g0 : g0 + 2, g3 = tail ? g0 : g0 + 3;
+      r.s[0] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g0), 16)));
+      r.s[1] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g0 + 1), 16)));
+      r.b[0] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g2), 16)));
+      r.b[1] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g3), 16)));
+    } else {
+      r.s[0] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g0), 32)));
+      r.s[1] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g1), 32)));
+      r.b[0] = r.b[1] = 0u;
+    }
+  } else {
+    const T* sp = reinterpret_cast<const T*>(a.scales) + row * G;
+    const T* bp = reinterpret_cast<const T*>(a.biases) + row * G;
+    r.s[0] = splat(sp[g0]);
+    r.b[0] = splat(bp[g0]);
+    r.s[1] = splat(sp[g1]);
+    r.b[1] = splat(bp[g1]);
+  }
+  return r;
+}
+
+template <typename T, int BITS, bool FP4>
+__device__ __forceinline__ void dequant_stage(const Packed<BITS>& p, const StageSB& sb, bool fp4_g16,
+                                              uint8_t* a_row, int r, bool tail) {
+  // chunk c of 8 elements lands at 16-byte slot c ^ (r & 7) of the row
+  const int sw = r & 7;
+  auto put = [&](int c, uint4 v) {
+    *reinterpret_cast<uint4*>(a_row + ((c ^ sw) << 4)) = v;
+  };
+  if constexpr (FP4) {
+    // quarters of 16 elements: scales s0 s1 (g16: b0 b1 hold quarters 2, 3)
+    const uint32_t q0 = sb.s[0];
+    const uint32_t q1 = fp4_g16 ? sb.s[1] : sb.s[0];
+    const uint32_t q2 = fp4_g16 ? sb.b[0] : sb.s[1];
+    const uint32_t q3 = fp4_g16 ? sb.b[1] : sb.s[1];
+    put(0, dequant_chunk<T, BITS, FP4, 0>(p, q0, 0u));
+    put(1, dequant_chunk<T, BITS, FP4, 1>(p, q0, 0u));
+    put(2, dequant_chunk<T, BITS, FP4, 2>(p, q1, 0u));
+    put(3, dequant_chunk<T, BITS, FP4, 3>(p, q1, 0u));
+    if (!tail) {
+      put(4, dequant_chunk<T, BITS, FP4, 4>(p, q2, 0u));
+      put(5, dequant_chunk<T, BITS, FP4, 5>(p, q2, 0u));
+      put(6, dequant_chunk<T, BITS, FP4, 6>(p, q3, 0u));
+      put(7, dequant_chunk<T, BITS, FP4, 7>(p, q3, 0u));
+    }
+  } else {
+    put(0, dequant_chunk<T, BITS, FP4, 0>(p, sb.s[0], sb.b[0]));
+    put(1, dequant_chunk<T, BITS, FP4, 1>(p, sb.s[0], sb.b[0]));
+    put(2, dequant_chunk<T, BITS, FP4, 2>(p, sb.s[0], sb.b[0]));
+    put(3, dequant_chunk<T, BITS, FP4, 3>(p, sb.s[0], sb.b[0]));
+    if (!tail) {
+      put(4, dequant_chunk<T, BITS, FP4, 4>(p, sb.s[1], sb.b[1]));
+      put(5, dequant_chunk<T, BITS, FP4, 5>(p, sb.s[1], sb.b[1]));
+      put(6, dequant_chunk<T, BITS, FP4, 6>(p, sb.s[1], sb.b[1]));
+      put(7, dequant_chunk<T, BITS, FP4, 7>(p, sb.s[1], sb.b[1]));
+    }
+  }
+  if (tail) {
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    put(4, z); put(5, z); put(6, z); put(7, z);
+  }
+}
+
+// -------------------------------------------------------------------- kernel
+template <typename T, int BITS, bool FP4, int BT>
+__global__ void __launch_bounds__(kThreads, 1)
+qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
+  using S = QmmShape<BT>;
+  constexpr int ST = S::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* ring = smem;                                   // [ST] x (A 16 KB | B BT*128)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kDataBytes);
+  // bars: full_a[ST], full_b[ST], empty[ST], acc_full
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * ST + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kRowsW;
+  const int m0 = blockIdx.y * BT;
+  const int split = blockIdx.z;
+  const int kt0 = split * a.k_tiles_split;
+  const int kt1 = min(a.k_tiles, kt0 + a.k_tiles_split);
+  const int nkt = kt1 - kt0;                              // >= 1
+
+  auto full_a = [&](int s) { return smem_u32(bars + s); };
+  auto full_b = [&](int s) { return smem_u32(bars + ST + s); };
+  auto empty = [&](int s) { return smem_u32(bars + 2 * ST + s); };
+  const uint32_t acc_full = smem_u32(bars + 3 * ST);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(full_a(s), 4);          // one arrive per dequantizer warp
+      mbar_init(full_b(s), 1);          // TMA producer's arrive + tx bytes
+      mbar_init(empty(s), 1);           // MMA commit
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer (x)
+    if (lane == 0) {
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i % ST;
+        const uint32_t par = ((i / ST) & 1) ^ 1;
+        if (!mbar_wait(empty(s), par, abort_flag)) break;
+        mbar_arrive_expect_tx(full_b(s), S::kBBytes);
+        tma_load_2d(smem_u32(ring + s * S::kStageBytes + S::kABytes), &tmap_x, full_b(s),
+                    (kt0 + i) * kBK, m0);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(std::is_same<T, __nv_bfloat16>::value, kRowsW, BT);
+      bool ok = true;
+      for (int i = 0; i < nkt && ok; ++i) {
+        const int s = i % ST;
+        const uint32_t par = (i / ST) & 1;
+        ok = mbar_wait(full_a(s), par, abort_flag) && mbar_wait(full_b(s), par, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(ring + s * S::kStageBytes);
+        const uint32_t b_addr = a_addr + S::kABytes;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          mma_f16(tmem, sdesc_sw128(a_addr + k * 32), sdesc_sw128(b_addr + k * 32), idesc,
+                  (i > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(empty(s));
+      }
+      // Signals the epilogue once every issued MMA has completed (also on
+      // abort, so nothing is in flight when TMEM is freed).
+      mma_commit(acc_full);
+    }
+  } else {
+    // ------------------------------------------- dequantizers (warps 2..5)
+    const int r = threadIdx.x - kProducerWarp0 * 32;       // weight row in the tile
+    const int64_t row = n0 + r;
+    const bool row_ok = row < a.N;
+    const int G = a.K >> a.gs_log2;
+    const bool fp4_g16 = FP4 && a.gs_log2 == 4;
+    const uint8_t* wrow = a.wq + (row_ok ? row : 0) * a.row_bytes;
+    Packed<BITS> pk[kPrefetch];
+    StageSB sb[kPrefetch];
+    auto issue = [&](int i, Packed<BITS>& p, StageSB& q) {
+      const int kt = kt0 + i;
+      if (i < nkt && row_ok) {
+        const bool tail = (kt + 1) * kBK > a.K;
+        load_packed<BITS>(p, wrow + (int64_t)kt * (8 * BITS), !tail, a.narrow);
+        q = load_sb<T, FP4>(a, row, kt, G, tail);
+      }
+    };
+#pragma unroll
+    for (int j = 0; j < kPrefetch; ++j) issue(j, pk[j], sb[j]);
+    bool ok = true;
+    for (int i0 = 0; i0 < nkt && ok; i0 += kPrefetch) {
+#pragma unroll
+      for (int j = 0; j < kPrefetch; ++j) {
+        const int i = i0 + j;
+        if (i >= nkt || !ok) break;
+        const int s = i % ST;
+        const uint32_t par = ((i / ST) & 1) ^ 1;
+        ok = mbar_wait(empty(s), par, abort_flag);
+        if (!ok) break;
+        uint8_t* a_row = ring + s * S::kStageBytes + r * 128;
+        const int kt = kt0 + i;
+        if (row_ok) {
+          dequant_stage<T, BITS, FP4>(pk[j], sb[j], fp4_g16, a_row, r, (kt + 1) * kBK > a.K);
+        } else {
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a_row + (c << 4)) = z;
+        }
+        issue(i + kPrefetch, pk[j], sb[j]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full_a(s));
+      }
+    }
+
+    // ------------------------------------------------------- epilogue
+    const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, 4000000000ull);
+    tc_fence_after();
+    const int q = warp & 3;                                 // TMEM lane quarter
+    const int rr = q * 32 + lane;                           // tile row of this thread
+    const int64_t orow = n0 + rr;
+    float* red = reinterpret_cast<float*>(ring);            // [BT][128] when split
+    if (acc_ok && !*abort_flag) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < BT; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld_16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+        if (a.splits == 1) {
+          if (orow < a.N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int m = m0 + c0 + j;
+              if (m < a.M)
+                reinterpret_cast<T*>(a.y)[(int64_t)m * a.N + orow] = TT<T>::from_f(__uint_as_float(v[j]));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) red[(c0 + j) * kRowsW + rr] = __uint_as_float(v[j]);
+        }
+      }
+    }
+  }
+
+  // --------------------------------------------------------- split-K reduce
+  if (a.splits > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    if (!*abort_flag) {
+      const float* red = reinterpret_cast<const float*>(ring);
+      for (int i = threadIdx.x; i < BT * kRowsW; i += kThreads) {
+        if (i % a.splits != split) continue;
+        const int j = i / kRowsW, rr = i - j * kRowsW;
+        const int m = m0 + j;
+        const int64_t orow = n0 + rr;
+        if (m >= a.M || orow >= a.N) continue;
+        float sum = 0.0f;
+        for (int q = 0; q < a.splits; ++q) sum += cluster.map_shared_rank(red, q)[i];
+        reinterpret_cast<T*>(a.y)[(int64_t)m * a.N + orow] = TT<T>::from_f(sum);
+      }
+    }
+    cluster.sync();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) atomicOr(&g_aq_device_error, 1u);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, S::kTmemCols);
+  }
+}
+
+// -------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// x [rows, K] T, box {64, box_rows}, 128-byte swizzle, zero fill out of bounds.
+cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K, int dtype,
+                       int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dtype == AQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   2, const_cast<void*>(x), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <typename T, int BITS, bool FP4, int BT>
+cudaError_t launch_tc(const QmmPlan& p, const CUtensorMap& map, const QmmArgs& a, cudaStream_t st) {
+  using S = QmmShape<BT>;
+  auto kern = qmm_tc_kernel<T, BITS, FP4, BT>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !attr_done[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.n_tiles, (unsigned)p.m_tiles, (unsigned)p.splits);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = S::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = (unsigned)p.splits;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map, a);
+}
+
+template <typename T, int BITS, bool FP4>
+cudaError_t by_bt(const QmmPlan& p, const CUtensorMap& map, const QmmArgs& a, cudaStream_t st) {
+  switch (p.bt) {
+    case 16: return launch_tc<T, BITS, FP4, 16>(p, map, a, st);
+    case 32: return launch_tc<T, BITS, FP4, 32>(p, map, a, st);
+    case 64: return launch_tc<T, BITS, FP4, 64>(p, map, a, st);
+    case 128: return launch_tc<T, BITS, FP4, 128>(p, map, a, st);
+    default: return launch_tc<T, BITS, FP4, 256>(p, map, a, st);
+  }
+}
+
+template <typename T>
+cudaError_t by_bits_tc(const QmmPlan& p, const CUtensorMap& map, const QmmArgs& a, int bits,
+                       int mode, cudaStream_t st) {
+  if (mode == AQ_MODE_FP4) return by_bt<T, 4, true>(p, map, a, st);
+  switch (bits) {
+    case 2: return by_bt<T, 2, false>(p, map, a, st);
+    case 3: return by_bt<T, 3, false>(p, map, a, st);
+    case 4: return by_bt<T, 4, false>(p, map, a, st);
+    case 5: return by_bt<T, 5, false>(p, map, a, st);
+    case 6: return by_bt<T, 6, false>(p, map, a, st);
+    case 8: return by_bt<T, 8, false>(p, map, a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int ilog2i(int v) {
+  int r = 0;
+  while ((1 << (r + 1)) <= v) ++r;
+  return r;
+}
+
+}  // namespace
+
+QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
+  (void)bits; (void)gs; (void)mode;
+  QmmPlan p{};
+  const int64_t n_tiles = (N + kRowsW - 1) / kRowsW;
+  const int64_t k_tiles = (K + kBK - 1) / kBK;
+  const int sms = 148;
+  // Token tile: the smallest that covers M up to 64 (one wave of weight
+  // tiles), else the largest whose tile count fills the GPU.
+  int bt;
+  if (M <= 16) bt = 16;
+  else if (M <= 32) bt = 32;
+  else if (M <= 64) bt = 64;
+  else {
+    bt = 256;
+    while (bt > 64 && n_tiles * ((M + bt - 1) / bt) < sms) bt /= 2;
+  }
+  p.bt = bt;
+  p.n_tiles = n_tiles;
+  p.m_tiles = (M + bt - 1) / bt;
+  // Split K over up to 8 CTAs of a cluster while the tiles underfill the GPU.
+  int splits = 1;
+  const int64_t tiles = p.n_tiles * p.m_tiles;
+  while (splits < 8 && tiles * splits * 2 <= sms && k_tiles / (splits * 2) >= 2) splits *= 2;
+  p.k_tiles_split = (int)((k_tiles + splits - 1) / splits);
+  p.splits = (int)((k_tiles + p.k_tiles_split - 1) / p.k_tiles_split);
+  p.k_tiles = (int)k_tiles;
+  return p;
+}
+
+cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const void* scales,
+                       const void* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+                       int gs, int mode, int dtype, cudaStream_t st) {
+  CUtensorMap map;
+  cudaError_t e = make_x_map(&map, x, M, K, dtype, p.bt);
+  if (e != cudaSuccess) return e;
+  QmmArgs a;
+  a.wq = (const uint8_t*)w_q;
+  a.scales = scales;
+  a.biases = biases;
+  a.y = y;
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.gs_log2 = ilog2i(gs);
+  a.k_tiles = p.k_tiles;
+  a.k_tiles_split = p.k_tiles_split;
+  a.splits = p.splits;
+  a.row_bytes = K * bits / 8;
+  const int vec = (bits == 3 || bits == 5) ? 8 : 16;
+  a.narrow = (a.row_bytes % vec) != 0;
+  return dtype == AQ_F16 ? by_bits_tc<__half>(p, map, a, bits, mode, st)
+                         : by_bits_tc<__nv_bfloat16>(p, map, a, bits, mode, st);
+}
+
+cudaError_t read_device_error(unsigned* out) {
+  return cudaMemcpyFromSymbol(out, g_aq_device_error, sizeof(unsigned));
+}
+
+}  // namespace aq

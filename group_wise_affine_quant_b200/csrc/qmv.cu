@@ -75,8 +75,9 @@ template <typename T, int BITS, int MT, bool FP4>
 __global__ void __launch_bounds__(kThreads)
 qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
            const void* __restrict__ scales_v, const T* __restrict__ biases, T* __restrict__ y,
-           int M, int64_t N, int64_t K, int gs, int64_t Ks, int S, int lpr_log2, int RI,
+           int M, int64_t N, int64_t K, int gs_log2, int64_t Ks, int S, int lpr_log2, int RI,
            int chunk_units) {
+  const int gs = 1 << gs_log2;
   extern __shared__ float4 smem4[];
   float* smem = reinterpret_cast<float*>(smem4);
   const int rank = blockIdx.y;                              // cluster spans all of y
@@ -95,7 +96,7 @@ qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = lane >> lpr_log2, ul = lane & (lpr - 1);
-  const int64_t G = K / gs;
+  const int64_t G = K >> gs_log2;
   const int64_t row_bytes = K * BITS / 8;
 
   // Prefetch this lane's first weight unit before staging x, so the HBM
@@ -160,7 +161,7 @@ qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
 #pragma unroll
           for (int i = 0; i < BITS; ++i) cur[i] = wd[i];
           if (u + lpr < cu) load_unit<BITS>(wrow + (int64_t)(u + lpr) * (4 * BITS), wd);
-          const int64_t g = (k0 + (int64_t)(c0 + u) * kUnit) / gs;
+          const int g = (int)(((int)k0 + (c0 + u) * kUnit) >> gs_log2);
           // FP4 at group 16 has two scales per 32-code unit (halves lo / hi).
           float s_lo, s_hi, b = 0.0f;
           if constexpr (FP4) {
@@ -261,7 +262,7 @@ cudaError_t launch_one(const QmvPlan& p, const void* x, const void* w_q, const v
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, (const T*)x, (const uint8_t*)w_q, scales,
-                            (const T*)biases, (T*)y, (int)M, N, K, gs, p.ks, p.splits,
+                            (const T*)biases, (T*)y, (int)M, N, K, ilog2_floor(gs), p.ks, p.splits,
                             ilog2_floor(p.lpr), p.ri, p.chunk_units);
 }
 

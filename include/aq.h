@@ -110,11 +110,9 @@ AQ_API aq_status aq_dequantize(const void* w_q, const void* scales, const void* 
 /*
  * aq_qmv — y = x . w_hat^T for small M (1 <= M <= 16): the weight-streaming
  * path ("Add the 3bit packed qmm_t", affine_packed_qmv_fast, routed for few
- * rows of x).  x [M, K] T, y [M, N] T, fp32 accumulation.  Split-K partial
- * sums go to `workspace` (aq_workspace_size(AQ_OP_QMV, ...) bytes, which may
- * be 0, in which case workspace may be NULL).  The workspace must be
- * zero-filled once before its first use; every call leaves it ready for the
- * next one.  Calls that share a workspace must not run concurrently.
+ * rows of x).  x [M, K] T, y [M, N] T, fp32 accumulation.  K-slices are
+ * reduced inside a thread block cluster, so no workspace is needed
+ * (aq_workspace_size returns 0; workspace may be NULL and is not touched).
  * Returns AQ_ERR_INVALID_ARG for M outside 1..16.
  */
 AQ_API aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void* biases,
@@ -125,8 +123,9 @@ AQ_API aq_status aq_qmv(const void* x, const void* w_q, const void* scales, cons
 /*
  * aq_qmm — y = x . w_hat^T for any M >= 1 ("Add the 3bit packed qmm_t",
  * affine_packed_qmm_t): weight tiles are dequantized into shared memory in T
- * and multiplied on the tensor cores with fp32 accumulation.  Arguments and
- * workspace rules as aq_qmv.
+ * (the values aq_dequantize writes) and multiplied on the tensor cores
+ * (tcgen05, fp32 accumulation in tensor memory).  Arguments as aq_qmv; M may
+ * be any size.  Needs no workspace (workspace may be NULL).
  */
 AQ_API aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void* biases,
                  void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
@@ -161,6 +160,15 @@ AQ_API aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* sca
  */
 AQ_API size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size,
                          aq_mode mode, int groups);
+
+/*
+ * Device-side error bits accumulated since the library was loaded on the
+ * current device (0 = none).  Bit 0: a kernel's bounded wait on an mbarrier
+ * timed out (after 2 s); the kernel stopped, freed its tensor memory and left
+ * its output incomplete.  Synchronises with the device (reads a __device__
+ * variable).  Returns 0xFFFFFFFF if the read itself fails.
+ */
+AQ_API unsigned aq_device_errors(void);
 
 /* Message for the last non-AQ_OK status on the calling thread ("" if none). */
 AQ_API const char* aq_last_error(void);

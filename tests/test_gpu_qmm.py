@@ -1,0 +1,174 @@
+"""GPU parity for aq_qmm (tcgen05 tensor-core path) against the oracle, within
+|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_affine_quant_b200 import api, inputs
+from tests.gpu_util import DEV, dev_u16, dev_u8, to_dev
+from tests.util import check_matmul
+
+pytestmark = pytest.mark.gpu
+
+BITS = (2, 3, 4, 5, 6, 8)
+
+
+def _case(M, N, K, bits, gs, dt, seed, wstd=0.05, xstd=1.0):
+    g = inputs.gen(seed)
+    w = inputs.normal((N, K), wstd, dt, g)
+    x = inputs.normal((M, K), xstd, dt, g)
+    wq, s, b = api.aq_quantize(to_dev(w), bits, gs)
+    return to_dev(x), wq, s, b
+
+
+def _check(x, wq, s, b, y, bits, gs, dt, mode=0, **kw):
+    N = wq.shape[0]
+    sc = dev_u8(s) if mode == 1 else dev_u16(s)
+    bi = None if b is None else dev_u16(b)
+    yr, den = oracle.qmm(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt)
+    return check_matmul(dev_u16(y), yr, den, dt, **kw)
+
+
+def _check_sampled(x, wq, s, b, y, bits, gs, dt, n_samples=512, seed=0, mode=0, **kw):
+    M, N = y.shape
+    rng = np.random.default_rng(seed)
+    ms = np.concatenate([[0, M - 1, M - 1, 0], rng.integers(0, M, n_samples)])
+    ns = np.concatenate([[0, N - 1, 0, N - 1], rng.integers(0, N, n_samples)])
+    sc = dev_u8(s) if mode == 1 else dev_u16(s)
+    bi = None if b is None else dev_u16(b)
+    yr, den = oracle.qmm_sampled(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt, ms, ns)
+    ys = dev_u16(y)[ms, ns]
+    return check_matmul(ys, yr, den, dt, **kw)
+
+
+def test_qmm_smallest():
+    """One 128 x 16 tile, one K-step."""
+    x, wq, s, b = _case(16, 128, 64, 4, 64, 0, seed=1)
+    y = api.aq_qmm(x, wq, s, b, 4, 64)
+    torch.cuda.synchronize()
+    assert api.aq_last_error() == ""
+    _check(x, wq, s, b, y, 4, 64, 0)
+    assert api.lib().aq_device_errors() == 0
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("dt", [0, 1])
+def test_qmm_all_widths(bits, dt):
+    """Several weight tiles, ragged N and M, K with a 32-element tail."""
+    gs = 32
+    x, wq, s, b = _case(37, 200, 64 * 5 + 32, bits, gs, dt, seed=bits + 10 * dt)
+    y = api.aq_qmm(x, wq, s, b, bits, gs)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, bits, gs, dt)
+
+
+@pytest.mark.parametrize("M", [1, 2, 15, 16, 17, 32, 33, 64, 65, 127, 128, 129, 255, 256, 300])
+def test_qmm_m_sweep(M):
+    """Every token-tile size and its edges (16/32/64/128/256 rows of x)."""
+    dt = M % 2
+    x, wq, s, b = _case(M, 256, 512, 4, 64, dt, seed=M)
+    y = api.aq_qmm(x, wq, s, b, 4, 64)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, 4, 64, dt)
+
+
+@pytest.mark.parametrize("gs", [32, 64, 128])
+@pytest.mark.parametrize("bits", [3, 4, 8])
+def test_qmm_groups(gs, bits):
+    x, wq, s, b = _case(48, 384, 1024, bits, gs, 1, seed=gs + bits)
+    y = api.aq_qmm(x, wq, s, b, bits, gs)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, bits, gs, 1)
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 128, 8192), (1, 256, 4096), (64, 384, 2048 + 32)])
+def test_qmm_split_k_cluster(M, N, K):
+    """Few output tiles: K splits over a cluster and reduces through DSMEM."""
+    x, wq, s, b = _case(M, N, K, 4, 32, 0, seed=K, wstd=0.02)
+    y1 = api.aq_qmm(x, wq, s, b, 4, 32)
+    y2 = api.aq_qmm(x, wq, s, b, 4, 32)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    _check(x, wq, s, b, y1, 4, 32, 0)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 5, 6])
+def test_qmm_narrow_rows(bits):
+    """K % 64 == 32: row strides that are not 16-byte multiples."""
+    x, wq, s, b = _case(20, 130, 32 * 9, bits, 32, 1, seed=bits)
+    y = api.aq_qmm(x, wq, s, b, bits, 32)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, bits, 32, 1)
+
+
+@pytest.mark.parametrize("gs", [16, 32])
+@pytest.mark.parametrize("M", [1, 16, 100, 256])
+@pytest.mark.parametrize("dt", [0, 1])
+def test_qmm_fp4(gs, M, dt):
+    N, K = 256, 1024 + (16 if gs == 16 else 32) * 2
+    codes, scales = inputs.fp4(N, K, gs, seed=gs + M)
+    x = inputs.normal((M, K), 1.0, dt, inputs.gen(M))
+    xd, wq, sc = to_dev(x), codes.to(DEV), scales.to(DEV)
+    y = api.aq_qmm(xd, wq, sc, None, 4, gs)
+    torch.cuda.synchronize()
+    _check(xd, wq, sc, None, y, 4, gs, dt, mode=1)
+
+
+@pytest.mark.parametrize("M", [32, 64])
+@pytest.mark.parametrize("name,N,K", inputs.LLAMA_1B_PROJ)
+def test_qmm_decode_projection(M, name, N, K):
+    """Decode sweep rows M = 32, 64 at full projection size (bf16 4-bit g64)."""
+    x, wq, s, b = _case(M, N, K, 4, 64, 1, seed=N + K + M, wstd=0.02)
+    y = api.aq_qmm(x, wq, s, b, 4, 64)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y, 4, 64, 1)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
+def test_qmm_chained_first_products(bits):
+    """Chained workload, fp16 g64: x[1024,1024] . W1^T (W1 4096x1024) then
+    . W2^T (W2 1024x4096), each checked on sampled outputs against the oracle
+    fed with the device's own input to that product."""
+    x, w1, w2 = inputs.chained()
+    q1 = api.aq_quantize(to_dev(w1), bits, 64)
+    q2 = api.aq_quantize(to_dev(w2), bits, 64)
+    xd = to_dev(x)
+    h = api.aq_qmm(xd, *q1, bits, 64)
+    o = api.aq_qmm(h, *q2, bits, 64)
+    torch.cuda.synchronize()
+    _check_sampled(xd, *q1, h, bits, 64, 0, seed=bits)
+    fin = torch.isfinite(h).all().item()
+    if fin:
+        _check_sampled(h, *q2, o, bits, 64, 0, seed=bits + 1)
+
+
+@pytest.mark.parametrize("gs,scale_range", [(32, "finite"), (16, "finite"), (32, "literal")])
+@pytest.mark.parametrize("M", [256, 4096])
+def test_qmm_fp4_full_size(gs, scale_range, M):
+    """FP4 workload, bf16, K = N = 4096, sampled outputs."""
+    codes, scales = inputs.fp4(4096, 4096, gs, scale_range=scale_range, seed=7)
+    x = inputs.fp4_x(M, 4096)
+    xd, wq, sc = to_dev(x), codes.to(DEV), scales.to(DEV)
+    y = api.aq_qmm(xd, wq, sc, None, 4, gs)
+    torch.cuda.synchronize()
+    _check_sampled(xd, wq, sc, None, y, 4, gs, 1, mode=1,
+                   overflow_any_nonfinite=(scale_range == "literal"))
+
+
+def test_qmm_matches_qmv_small_m():
+    """For M <= 16 both paths agree within twice the bound."""
+    x, wq, s, b = _case(8, 512, 2048, 4, 64, 1, seed=3)
+    y1 = api.aq_qmm(x, wq, s, b, 4, 64)
+    y2 = api.aq_qmv(x, wq, s, b, 4, 64)
+    torch.cuda.synchronize()
+    _check(x, wq, s, b, y1, 4, 64, 1)
+    _check(x, wq, s, b, y2, 4, 64, 1)
+
+
+def test_qmm_empty():
+    x = torch.zeros((0, 64), dtype=torch.float16, device=DEV)
+    wq = torch.zeros((128, 32), dtype=torch.uint8, device=DEV)
+    s = torch.zeros((128, 1), dtype=torch.float16, device=DEV)
+    y = api.aq_qmm(x, wq, s, s, 4, 64)
+    assert y.shape == (0, 128)
