@@ -9,14 +9,17 @@
 //     full 128-row MMA: one wave of tiles covers M = 1..64 at the weight
 //     stream's cost.
 //   * Warp 0 (one thread) loads x tiles with TMA into 128-byte-swizzled shared
-//     memory; warp 1 allocates TMEM and one of its threads issues
-//     tcgen05.mma (kind::f16, fp32 accumulate in TMEM); warps 2-5 are the
-//     dequantizers (one weight row per thread): they stream packed codes and
-//     the group's scale and bias from global memory several stages ahead in
-//     registers, form w_hat = s*q + b in T with packed half2/bfloat162 FMAs
-//     (single rounding, the same value aq_dequantize writes), and store it in
-//     the same swizzled K-major layout.  Stages hand over through mbarriers;
-//     the MMA's commit frees a stage for both producers.
+//     memory; warp 6 streams the packed codes and the words holding each
+//     row's scales and biases into a deep shared-memory ring with cp.async,
+//     completing on an mbarrier; warp 1 allocates TMEM and one of its threads
+//     issues tcgen05.mma (kind::f16, fp32 accumulate in TMEM); warps 2-5 are
+//     the dequantizers (one weight row per thread): from shared memory they
+//     form w_hat = s*q + b in T with packed half2/bfloat162 FMAs (single
+//     rounding, the same value aq_dequantize writes) and store it in the
+//     swizzled K-major layout.  The dequantizers issue no global loads, so
+//     their async-proxy fence before each hand-over never waits on memory
+//     latency.  Stages hand over through mbarriers; the MMA's commit frees an
+//     operand stage for both producers.
 //   * K-step 64 (one 128-byte swizzle atom of 16-bit values); a K tail of 32
 //     reads zero x through TMA's out-of-bounds fill and writes zero w_hat.
 //   * The epilogue (warps 2-5) reads TMEM with tcgen05.ld.  With split-K the
@@ -44,22 +47,27 @@ using namespace sm100;
 
 constexpr int kBK = 64;                  // K elements per stage (128 bytes of T)
 constexpr int kRowsW = 128;              // weight rows per tile (MMA M)
-constexpr int kThreads = 192;            // 6 warps
+constexpr int kThreads = 224;            // 7 warps
 constexpr int kProducerWarp0 = 2;        // warps 2..5 dequantize and run the epilogue
-constexpr int kPrefetch = 4;             // stages of packed codes in flight per thread
+constexpr int kLoaderWarp = 6;           // streams packed codes, scales, biases
 
-template <int BT>
+template <int BT, int BITS>
 struct QmmShape {
-  static constexpr int kStages = BT >= 256 ? 3 : BT >= 128 ? 4 : 6;
-  static constexpr int kABytes = kRowsW * kBK * 2;          // 16 KB
-  static constexpr int kBBytes = BT * kBK * 2;              // BT * 128
+  static constexpr int kStages = BT >= 256 ? 3 : 4;                 // operand stages
+  static constexpr int kPStages = BT >= 256 ? 4 : BT >= 128 ? 6 : BT >= 64 ? 8 : BT >= 32 ? 10 : 12;
+  static constexpr int kABytes = kRowsW * kBK * 2;                   // 16 KB
+  static constexpr int kBBytes = BT * kBK * 2;                       // BT * 128
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kRedBytes = BT * kRowsW * 4;          // split-K parking
+  static constexpr int kPB = 8 * BITS;                               // packed bytes / row / stage
+  static constexpr int kRP = (kPB % 32 == 0) ? kPB + 16 : kPB;       // row pitch (bank spread)
+  static constexpr int kPSlot = kRowsW * kRP + kRowsW * 16;          // packed rows + s/b words
+  static constexpr int kRedBytes = BT * kRowsW * 4;                  // split-K parking
   static constexpr int kRingBytes = kStages * kStageBytes;
-  static constexpr int kDataBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
+  static constexpr int kOpBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
+  static constexpr int kDataBytes = kOpBytes + kPStages * kPSlot;
   static constexpr int kTmemCols = BT < 32 ? 32 : BT;
-  // 1024 for alignment slack + data + barriers
-  static constexpr int kSmem = 1024 + kDataBytes + 256;
+  static constexpr int kSmem = 1024 + kDataBytes + 512;             // align slack, barriers
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
 struct QmmArgs {
@@ -72,9 +80,54 @@ struct QmmArgs {
   int k_tiles;          // ceil(K / 64)
   int k_tiles_split;    // k-tiles per split
   int splits;
-  int narrow;           // 1: 4-byte weight loads (row stride not 16-byte aligned)
+  int vec;              // widest cp.async (16, 8 or 4 bytes) the packed rows allow
   int64_t row_bytes;
 };
+
+// ------------------------------------------------------------ cp.async
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on `bar` when all of this thread's earlier cp.async copies land
+// (the barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Copy the two 4-byte words starting at the 4-byte boundary at or below
+// `p` (a 2- or 1-byte element of an array that ends at `end`) into dst.
+// Words that stick out of the array are filled with byte loads of their
+// in-bounds part (and zeros) and plain shared stores; the function then
+// returns true and the caller must publish the stage with a regular
+// (release) arrive instead of the cp.async-completion arrive.
+__device__ __forceinline__ bool copy_window(uint32_t dst, const uint8_t* p, const uint8_t* begin,
+                                            const uint8_t* end) {
+  bool plain = false;
+  const uint8_t* w0 = reinterpret_cast<const uint8_t*>((uintptr_t)p & ~(uintptr_t)3);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint8_t* w = w0 + 4 * i;
+    if (w >= begin && w + 4 <= end) {
+      cp_async_4(dst + 4 * i, w);
+    } else {
+      uint32_t v = 0;
+      for (int j = 0; j < 4; ++j)
+        if (w + j >= begin && w + j < end) v |= (uint32_t)w[j] << (8 * j);
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst + 4 * i), "r"(v) : "memory");
+      plain = true;
+    }
+  }
+  return plain;
+}
 
 // ------------------------------------------------------------- dequantizer
 // Per thread and stage: the 64 codes of one weight row as 2*BITS words.
@@ -85,34 +138,19 @@ struct Packed {
 };
 
 template <int BITS>
-__device__ __forceinline__ void load_packed(Packed<BITS>& p, const uint8_t* src, bool full,
-                                            bool narrow) {
-  // src: 8*BITS bytes (full stage) or 4*BITS bytes (K tail of 32 codes).
-  // Vector loads need the row stride K*bits/8 to be a multiple of 16 bytes
-  // (8 for 3/5-bit); otherwise (`narrow`) 4-byte loads, which every row and
-  // stage offset satisfies since K % 32 == 0.
-  if (full && narrow) {
+__device__ __forceinline__ void lds_packed(Packed<BITS>& p, const uint8_t* src) {
+  if constexpr ((8 * BITS) % 16 == 0) {
 #pragma unroll
-    for (int i = 0; i < 2 * BITS; ++i) p.w[i] = __ldg(reinterpret_cast<const uint32_t*>(src) + i);
-  } else if (full) {
-    if constexpr (BITS == 2 || BITS == 4 || BITS == 6 || BITS == 8) {
-#pragma unroll
-      for (int i = 0; i < BITS / 2; ++i) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
-        p.w[4 * i] = v.x; p.w[4 * i + 1] = v.y; p.w[4 * i + 2] = v.z; p.w[4 * i + 3] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < BITS; ++i) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + i);
-        p.w[2 * i] = v.x; p.w[2 * i + 1] = v.y;
-      }
+    for (int i = 0; i < BITS / 2; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+      p.w[4 * i] = v.x; p.w[4 * i + 1] = v.y; p.w[4 * i + 2] = v.z; p.w[4 * i + 3] = v.w;
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < BITS; ++i) p.w[i] = __ldg(reinterpret_cast<const uint32_t*>(src) + i);
-#pragma unroll
-    for (int i = BITS; i < 2 * BITS; ++i) p.w[i] = 0u;
+    for (int i = 0; i < BITS; ++i) {
+      const uint2 v = *reinterpret_cast<const uint2*>(src + 8 * i);
+      p.w[2 * i] = v.x; p.w[2 * i + 1] = v.y;
+    }
   }
 }
 
@@ -218,41 +256,54 @@ __device__ __forceinline__ uint32_t splat(T v) {
   return (uint32_t)u | ((uint32_t)u << 16);
 }
 
-// Scale/bias pairs (splatted T) for the two 32-element halves of a stage.
+// Scale/bias pairs (splatted T) for the two 32-element halves of a stage;
+// FP4 at group 16 keeps its four quarter scales in s[0], s[1], b[0], b[1].
 struct StageSB {
   uint32_t s[2], b[2];
 };
 
+__device__ __forceinline__ uint32_t u16_at(uint32_t w0, uint32_t w1, int byte_off) {
+  const uint64_t v = ((uint64_t)w1 << 32) | w0;
+  return (uint32_t)(v >> (8 * byte_off)) & 0xFFFFu;
+}
+__device__ __forceinline__ uint32_t u8_at(uint32_t w0, uint32_t w1, int byte_off) {
+  const uint64_t v = ((uint64_t)w1 << 32) | w0;
+  return (uint32_t)(v >> (8 * byte_off)) & 0xFFu;
+}
+
+// Decode the staged words of one row into the stage's scale/bias pairs.
 template <typename T, bool FP4>
-__device__ __forceinline__ StageSB load_sb(const QmmArgs& a, int64_t row, int kt, int G, bool tail) {
+__device__ __forceinline__ StageSB sb_from_words(const uint4 wv, const QmmArgs& a, int64_t row,
+                                                 int kt, int G, bool tail) {
   StageSB r;
   const int k = kt * kBK;
   const int g0 = k >> a.gs_log2;
-  // the upper half of a K-tail stage has no group (and must not be read)
   const int g1 = tail ? g0 : (k + 32) >> a.gs_log2;
   if constexpr (FP4) {
-    const uint8_t* sp = reinterpret_cast<const uint8_t*>(a.scales) + row * G;
-    const int gs = 1 << a.gs_log2;
-    // group 16: four groups per stage; each 16-element quarter gets its own
-    // scale, handled by the caller through s[] = quarters (0,1) and b[] = (2,3)
-    if (gs == 16) {
-      const int g2 = tail ? g0 : g0 + 2, g3 = tail ? g0 : g0 + 3;
-      r.s[0] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g0), 16)));
-      r.s[1] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g0 + 1), 16)));
-      r.b[0] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g2), 16)));
-      r.b[1] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g3), 16)));
+    const uint8_t* p = reinterpret_cast<const uint8_t*>(a.scales) + row * G + g0;
+    const int off = (int)((uintptr_t)p & 3);
+    auto sc = [&](int d) {
+      return splat(TT<T>::from_f(fp4_scale_t<T>(u8_at(wv.x, wv.y, off + d), 1 << a.gs_log2)));
+    };
+    if (a.gs_log2 == 4) {
+      r.s[0] = sc(0);
+      r.s[1] = sc(1);
+      r.b[0] = tail ? r.s[0] : sc(2);
+      r.b[1] = tail ? r.s[0] : sc(3);
     } else {
-      r.s[0] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g0), 32)));
-      r.s[1] = splat(TT<T>::from_f(fp4_scale_t<T>(__ldg(sp + g1), 32)));
+      r.s[0] = sc(0);
+      r.s[1] = sc(g1 - g0);
       r.b[0] = r.b[1] = 0u;
     }
   } else {
-    const T* sp = reinterpret_cast<const T*>(a.scales) + row * G;
-    const T* bp = reinterpret_cast<const T*>(a.biases) + row * G;
-    r.s[0] = splat(sp[g0]);
-    r.b[0] = splat(bp[g0]);
-    r.s[1] = splat(sp[g1]);
-    r.b[1] = splat(bp[g1]);
+    const int offs = (int)(((uintptr_t)a.scales + 2 * (row * G + g0)) & 3);
+    const int offb = (int)(((uintptr_t)a.biases + 2 * (row * G + g0)) & 3);
+    const uint32_t s0 = u16_at(wv.x, wv.y, offs), s1 = u16_at(wv.x, wv.y, offs + 2 * (g1 - g0));
+    const uint32_t b0 = u16_at(wv.z, wv.w, offb), b1 = u16_at(wv.z, wv.w, offb + 2 * (g1 - g0));
+    r.s[0] = s0 | (s0 << 16);
+    r.s[1] = s1 | (s1 << 16);
+    r.b[0] = b0 | (b0 << 16);
+    r.b[1] = b1 | (b1 << 16);
   }
   return r;
 }
@@ -303,14 +354,16 @@ __device__ __forceinline__ void dequant_stage(const Packed<BITS>& p, const Stage
 template <typename T, int BITS, bool FP4, int BT>
 __global__ void __launch_bounds__(kThreads, 1)
 qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
-  using S = QmmShape<BT>;
+  using S = QmmShape<BT, BITS>;
   constexpr int ST = S::kStages;
+  constexpr int PST = S::kPStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = smem;                                   // [ST] x (A 16 KB | B BT*128)
+  uint8_t* pring = smem + S::kOpBytes;                    // [PST] packed rows | s/b words
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kDataBytes);
-  // bars: full_a[ST], full_b[ST], empty[ST], acc_full
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * ST + 1);
+  // bars: full_a[ST], full_b[ST], empty[ST], full_w[PST], empty_w[PST], acc_full
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * ST + 2 * PST + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -320,17 +373,24 @@ qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
   const int kt0 = split * a.k_tiles_split;
   const int kt1 = min(a.k_tiles, kt0 + a.k_tiles_split);
   const int nkt = kt1 - kt0;                              // >= 1
+  const int G = a.K >> a.gs_log2;
 
   auto full_a = [&](int s) { return smem_u32(bars + s); };
   auto full_b = [&](int s) { return smem_u32(bars + ST + s); };
   auto empty = [&](int s) { return smem_u32(bars + 2 * ST + s); };
-  const uint32_t acc_full = smem_u32(bars + 3 * ST);
+  auto full_w = [&](int s) { return smem_u32(bars + 3 * ST + s); };
+  auto empty_w = [&](int s) { return smem_u32(bars + 3 * ST + PST + s); };
+  const uint32_t acc_full = smem_u32(bars + 3 * ST + 2 * PST);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(full_a(s), 4);          // one arrive per dequantizer warp
       mbar_init(full_b(s), 1);          // TMA producer's arrive + tx bytes
       mbar_init(empty(s), 1);           // MMA commit
+    }
+    for (int s = 0; s < PST; ++s) {
+      mbar_init(full_w(s), 32);         // one cp.async arrival per loader lane
+      mbar_init(empty_w(s), 4);         // one arrive per dequantizer warp
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -356,16 +416,62 @@ qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
                     (kt0 + i) * kBK, m0);
       }
     }
+  } else if (warp == kLoaderWarp) {
+    // ------------------------------------------ packed codes, scales, biases
+    const uint8_t* s_begin = reinterpret_cast<const uint8_t*>(a.scales);
+    const uint8_t* s_end = s_begin + (int64_t)a.N * G * (FP4 ? 1 : 2);
+    const uint8_t* b_begin = reinterpret_cast<const uint8_t*>(a.biases);
+    const uint8_t* b_end = b_begin + (int64_t)a.N * G * 2;
+    for (int i = 0; i < nkt; ++i) {
+      const int ps = i % PST;
+      const uint32_t par = ((i / PST) & 1) ^ 1;
+      if (!mbar_wait(empty_w(ps), par, abort_flag)) break;
+      const int kt = kt0 + i;
+      const bool tail = (kt + 1) * kBK > a.K;
+      const uint32_t slot = smem_u32(pring + ps * S::kPSlot);
+      bool plain = false;
+#pragma unroll
+      for (int j = 0; j < kRowsW / 32; ++j) {
+        const int r = lane + 32 * j;
+        const int64_t row = n0 + r;
+        if (row >= a.N) continue;
+        const uint8_t* src = a.wq + row * a.row_bytes + (int64_t)kt * S::kPB;
+        const uint32_t dst = slot + r * S::kRP;
+        const int nbytes = tail ? S::kPB / 2 : S::kPB;
+        if (a.vec == 16 && !tail) {
+#pragma unroll
+          for (int o = 0; o < S::kPB; o += 16) cp_async_16(dst + o, src + o);
+        } else if (a.vec >= 8 && (nbytes % 8) == 0) {
+          for (int o = 0; o < nbytes; o += 8) cp_async_8(dst + o, src + o);
+        } else {
+          for (int o = 0; o < nbytes; o += 4) cp_async_4(dst + o, src + o);
+        }
+        const uint32_t wdst = slot + kRowsW * S::kRP + r * 16;
+        const int g0 = (kt * kBK) >> a.gs_log2;
+        if constexpr (FP4) {
+          plain |= copy_window(wdst, s_begin + row * G + g0, s_begin, s_end);
+        } else {
+          plain |= copy_window(wdst, s_begin + 2 * (row * G + g0), s_begin, s_end);
+          plain |= copy_window(wdst + 8, b_begin + 2 * (row * G + g0), b_begin, b_end);
+        }
+      }
+      if (plain) {          // rare: a window at the end of the scale arrays
+        cp_async_wait_all();
+        mbar_arrive(full_w(ps));
+      } else {
+        cp_async_arrive(full_w(ps));
+      }
+    }
+    cp_async_wait_all();
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(std::is_same<T, __nv_bfloat16>::value, kRowsW, BT);
-      bool ok = true;
-      for (int i = 0; i < nkt && ok; ++i) {
+      for (int i = 0; i < nkt; ++i) {
         const int s = i % ST;
         const uint32_t par = (i / ST) & 1;
-        ok = mbar_wait(full_a(s), par, abort_flag) && mbar_wait(full_b(s), par, abort_flag);
-        if (!ok) break;
+        if (!(mbar_wait(full_a(s), par, abort_flag) && mbar_wait(full_b(s), par, abort_flag)))
+          break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(ring + s * S::kStageBytes);
         const uint32_t b_addr = a_addr + S::kABytes;
@@ -385,45 +491,39 @@ qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
     const int r = threadIdx.x - kProducerWarp0 * 32;       // weight row in the tile
     const int64_t row = n0 + r;
     const bool row_ok = row < a.N;
-    const int G = a.K >> a.gs_log2;
     const bool fp4_g16 = FP4 && a.gs_log2 == 4;
-    const uint8_t* wrow = a.wq + (row_ok ? row : 0) * a.row_bytes;
-    Packed<BITS> pk[kPrefetch];
-    StageSB sb[kPrefetch];
-    auto issue = [&](int i, Packed<BITS>& p, StageSB& q) {
+    for (int i = 0; i < nkt; ++i) {
+      const int ps = i % PST;
+      if (!mbar_wait(full_w(ps), (i / PST) & 1, abort_flag)) break;
+      const uint8_t* slot = pring + ps * S::kPSlot;
       const int kt = kt0 + i;
-      if (i < nkt && row_ok) {
-        const bool tail = (kt + 1) * kBK > a.K;
-        load_packed<BITS>(p, wrow + (int64_t)kt * (8 * BITS), !tail, a.narrow);
-        q = load_sb<T, FP4>(a, row, kt, G, tail);
-      }
-    };
+      const bool tail = (kt + 1) * kBK > a.K;
+      Packed<BITS> pk;
+      StageSB sb;
+      if (row_ok) {
+        lds_packed<BITS>(pk, slot + r * S::kRP);
+        if (tail) {
 #pragma unroll
-    for (int j = 0; j < kPrefetch; ++j) issue(j, pk[j], sb[j]);
-    bool ok = true;
-    for (int i0 = 0; i0 < nkt && ok; i0 += kPrefetch) {
-#pragma unroll
-      for (int j = 0; j < kPrefetch; ++j) {
-        const int i = i0 + j;
-        if (i >= nkt || !ok) break;
-        const int s = i % ST;
-        const uint32_t par = ((i / ST) & 1) ^ 1;
-        ok = mbar_wait(empty(s), par, abort_flag);
-        if (!ok) break;
-        uint8_t* a_row = ring + s * S::kStageBytes + r * 128;
-        const int kt = kt0 + i;
-        if (row_ok) {
-          dequant_stage<T, BITS, FP4>(pk[j], sb[j], fp4_g16, a_row, r, (kt + 1) * kBK > a.K);
-        } else {
-          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a_row + (c << 4)) = z;
+          for (int w = BITS; w < 2 * BITS; ++w) pk.w[w] = 0u;
         }
-        issue(i + kPrefetch, pk[j], sb[j]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(full_a(s));
+        const uint4 wv = *reinterpret_cast<const uint4*>(slot + kRowsW * S::kRP + r * 16);
+        sb = sb_from_words<T, FP4>(wv, a, row, kt, G, tail);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_w(ps));
+      const int s = i % ST;
+      if (!mbar_wait(empty(s), ((i / ST) & 1) ^ 1, abort_flag)) break;
+      uint8_t* a_row = ring + s * S::kStageBytes + r * 128;
+      if (row_ok) {
+        dequant_stage<T, BITS, FP4>(pk, sb, fp4_g16, a_row, r, tail);
+      } else {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a_row + (c << 4)) = z;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full_a(s));
     }
 
     // ------------------------------------------------------- epilogue
@@ -522,7 +622,7 @@ cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K,
 
 template <typename T, int BITS, bool FP4, int BT>
 cudaError_t launch_tc(const QmmPlan& p, const CUtensorMap& map, const QmmArgs& a, cudaStream_t st) {
-  using S = QmmShape<BT>;
+  using S = QmmShape<BT, BITS>;
   auto kern = qmm_tc_kernel<T, BITS, FP4, BT>;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -630,8 +730,9 @@ cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const v
   a.k_tiles_split = p.k_tiles_split;
   a.splits = p.splits;
   a.row_bytes = K * bits / 8;
-  const int vec = (bits == 3 || bits == 5) ? 8 : 16;
-  a.narrow = (a.row_bytes % vec) != 0;
+  // widest copy that every row start and stage offset (8*bits bytes) allows
+  a.vec = (a.row_bytes % 16 == 0 && (8 * bits) % 16 == 0) ? 16
+          : (a.row_bytes % 8 == 0 && (8 * bits) % 8 == 0) ? 8 : 4;
   return dtype == AQ_F16 ? by_bits_tc<__half>(p, map, a, bits, mode, st)
                          : by_bits_tc<__nv_bfloat16>(p, map, a, bits, mode, st);
 }
