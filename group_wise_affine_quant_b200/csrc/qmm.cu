@@ -30,6 +30,8 @@
 //     flag, every role stops issuing work and the CTA frees its TMEM.
 #include <cooperative_groups.h>
 
+#include <string.h>
+
 #include <type_traits>
 
 #include "common.cuh"
@@ -51,22 +53,32 @@ constexpr int kThreads = 224;            // 7 warps
 constexpr int kProducerWarp0 = 2;        // warps 2..5 dequantize and run the epilogue
 constexpr int kLoaderWarp = 6;           // streams packed codes, scales, biases
 
-template <int BT, int BITS>
+template <int BT, int BITS, bool FAST>
 struct QmmShape {
   static constexpr int kStages = BT >= 256 ? 3 : 4;                 // operand stages
-  static constexpr int kPStages = BT >= 256 ? 4 : BT >= 128 ? 6 : BT >= 64 ? 8 : BT >= 32 ? 10 : 12;
   static constexpr int kABytes = kRowsW * kBK * 2;                   // 16 KB
   static constexpr int kBBytes = BT * kBK * 2;                       // BT * 128
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kPB = 8 * BITS;                               // packed bytes / row / stage
-  static constexpr int kRP = (kPB % 32 == 0) ? kPB + 16 : kPB;       // row pitch (bank spread)
-  static constexpr int kPSlot = kRowsW * kRP + kRowsW * 16;          // packed rows + s/b words
+  // cp.async path: one slot per stage, rows at a bank-spreading pitch.
+  static constexpr int kPStages = BT >= 256 ? 4 : BT >= 128 ? 6 : BT >= 64 ? 8 : BT >= 32 ? 10 : 12;
+  static constexpr int kRP = (kPB % 32 == 0) ? kPB + 16 : kPB;
+  static constexpr int kPSlot = kRowsW * kRP + kRowsW * 16;
+  // TMA path: weight chunks of 128 rows x 128 bytes (128-byte swizzle) and
+  // scale chunks of 128 rows x 16 bytes (scales, then biases).
+  static constexpr int kWChunk = kRowsW * 128;                       // 16 KB
+  static constexpr int kWSlots = BT >= 256 ? 2 : BT >= 128 ? 3 : 4;
+  static constexpr int kSChunk = kRowsW * 16 * 2;                    // 4 KB
+  static constexpr int kSSlots = 4;
+  static constexpr int kLoadBytes = FAST ? kWSlots * kWChunk + kSSlots * kSChunk : kPStages * kPSlot;
   static constexpr int kRedBytes = BT * kRowsW * 4;                  // split-K parking
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kOpBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
-  static constexpr int kDataBytes = kOpBytes + kPStages * kPSlot;
+  static constexpr int kDataBytes = kOpBytes + kLoadBytes;
   static constexpr int kTmemCols = BT < 32 ? 32 : BT;
+  static constexpr int kBars = 3 * kStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
   static constexpr int kSmem = 1024 + kDataBytes + 512;             // align slack, barriers
+  static_assert(kBars * 8 + 16 <= 512, "barrier area");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
@@ -84,6 +96,13 @@ struct QmmArgs {
   int64_t row_bytes;
 };
 
+struct QmmMaps {
+  CUtensorMap x;        // [M, K] T, box {64, BT}, 128-byte swizzle
+  CUtensorMap w;        // [N, row_bytes] u8, box {128, 128}, 128-byte swizzle (TMA path)
+  CUtensorMap s;        // [N, G] scales, box {16 bytes, 128} (TMA path)
+  CUtensorMap b;        // [N, G] biases, likewise (affine)
+};
+
 // ------------------------------------------------------------ cp.async
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -94,10 +113,13 @@ __device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
-// Arrive on `bar` when all of this thread's earlier cp.async copies land
-// (the barrier's expected count includes this arrival).
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -106,12 +128,9 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // Copy the two 4-byte words starting at the 4-byte boundary at or below
 // `p` (a 2- or 1-byte element of an array that ends at `end`) into dst.
 // Words that stick out of the array are filled with byte loads of their
-// in-bounds part (and zeros) and plain shared stores; the function then
-// returns true and the caller must publish the stage with a regular
-// (release) arrive instead of the cp.async-completion arrive.
-__device__ __forceinline__ bool copy_window(uint32_t dst, const uint8_t* p, const uint8_t* begin,
+// in-bounds part (and zeros) and plain shared stores.
+__device__ __forceinline__ void copy_window(uint32_t dst, const uint8_t* p, const uint8_t* begin,
                                             const uint8_t* end) {
-  bool plain = false;
   const uint8_t* w0 = reinterpret_cast<const uint8_t*>((uintptr_t)p & ~(uintptr_t)3);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
@@ -123,10 +142,8 @@ __device__ __forceinline__ bool copy_window(uint32_t dst, const uint8_t* p, cons
       for (int j = 0; j < 4; ++j)
         if (w + j >= begin && w + j < end) v |= (uint32_t)w[j] << (8 * j);
       asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst + 4 * i), "r"(v) : "memory");
-      plain = true;
     }
   }
-  return plain;
 }
 
 // ------------------------------------------------------------- dequantizer
@@ -351,19 +368,32 @@ __device__ __forceinline__ void dequant_stage(const Packed<BITS>& p, const Stage
 }
 
 // -------------------------------------------------------------------- kernel
-template <typename T, int BITS, bool FP4, int BT>
+// Shared memory offset of byte `o` of row r within a chain of 128-byte
+// weight chunks (128-byte swizzle: 16-byte unit u of row r sits at unit
+// u ^ (r % 8)).
+__device__ __forceinline__ uint32_t wchunk_off(int o, int r) {
+  return (uint32_t)(r * 128 + ((((o >> 4) & 7) ^ (r & 7)) << 4) + (o & 15));
+}
+
+template <typename T, int BITS, bool FP4, int BT, bool FAST>
 __global__ void __launch_bounds__(kThreads, 1)
-qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
-  using S = QmmShape<BT, BITS>;
+qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
+  using S = QmmShape<BT, BITS, FAST>;
   constexpr int ST = S::kStages;
   constexpr int PST = S::kPStages;
+  constexpr int WS = S::kWSlots;
+  constexpr int SS = S::kSSlots;
+  constexpr int SGC = FP4 ? 16 : 8;                       // groups per scale chunk (16 bytes)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = smem;                                   // [ST] x (A 16 KB | B BT*128)
-  uint8_t* pring = smem + S::kOpBytes;                    // [PST] packed rows | s/b words
+  uint8_t* pring = smem + S::kOpBytes;                    // loader area
+  uint8_t* wring = pring;                                 // TMA path: [WS] weight chunks
+  uint8_t* sring = pring + WS * S::kWChunk;               // TMA path: [SS] scale chunks
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kDataBytes);
-  // bars: full_a[ST], full_b[ST], empty[ST], full_w[PST], empty_w[PST], acc_full
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * ST + 2 * PST + 1);
+  constexpr int NL = FAST ? WS + SS : PST;                // loader slots
+  // bars: full_a[ST], full_b[ST], empty[ST], full_l[NL], empty_l[NL], acc_full
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -378,9 +408,17 @@ qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
   auto full_a = [&](int s) { return smem_u32(bars + s); };
   auto full_b = [&](int s) { return smem_u32(bars + ST + s); };
   auto empty = [&](int s) { return smem_u32(bars + 2 * ST + s); };
-  auto full_w = [&](int s) { return smem_u32(bars + 3 * ST + s); };
-  auto empty_w = [&](int s) { return smem_u32(bars + 3 * ST + PST + s); };
-  const uint32_t acc_full = smem_u32(bars + 3 * ST + 2 * PST);
+  auto full_l = [&](int s) { return smem_u32(bars + 3 * ST + s); };
+  auto empty_l = [&](int s) { return smem_u32(bars + 3 * ST + NL + s); };
+  const uint32_t acc_full = smem_u32(bars + 3 * ST + 2 * NL);
+
+  // TMA path bookkeeping: weight chunk c covers bytes [wb0 + 128 c, +128) of
+  // every row, scale chunk j covers groups [SGC j, SGC (j + 1)).
+  const int64_t wb0 = (int64_t)kt0 * S::kPB;              // 16-byte aligned (host plan)
+  const int nwc = (int)((nkt * S::kPB + 127) / 128);
+  const int sc0 = ((kt0 * kBK) >> a.gs_log2) / SGC;
+  const int sc1 = (((kt1 * kBK) - 1) >> a.gs_log2) / SGC;
+  const int nsc = sc1 - sc0 + 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -388,9 +426,9 @@ qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
       mbar_init(full_b(s), 1);          // TMA producer's arrive + tx bytes
       mbar_init(empty(s), 1);           // MMA commit
     }
-    for (int s = 0; s < PST; ++s) {
-      mbar_init(full_w(s), 32);         // one cp.async arrival per loader lane
-      mbar_init(empty_w(s), 4);         // one arrive per dequantizer warp
+    for (int s = 0; s < NL; ++s) {
+      mbar_init(full_l(s), FAST ? 1 : 32);   // TMA arrive + tx, or every loader lane
+      mbar_init(empty_l(s), 4);              // one arrive per dequantizer warp
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -412,57 +450,93 @@ qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
         const uint32_t par = ((i / ST) & 1) ^ 1;
         if (!mbar_wait(empty(s), par, abort_flag)) break;
         mbar_arrive_expect_tx(full_b(s), S::kBBytes);
-        tma_load_2d(smem_u32(ring + s * S::kStageBytes + S::kABytes), &tmap_x, full_b(s),
+        tma_load_2d(smem_u32(ring + s * S::kStageBytes + S::kABytes), &maps.x, full_b(s),
                     (kt0 + i) * kBK, m0);
       }
     }
   } else if (warp == kLoaderWarp) {
-    // ------------------------------------------ packed codes, scales, biases
-    const uint8_t* s_begin = reinterpret_cast<const uint8_t*>(a.scales);
-    const uint8_t* s_end = s_begin + (int64_t)a.N * G * (FP4 ? 1 : 2);
-    const uint8_t* b_begin = reinterpret_cast<const uint8_t*>(a.biases);
-    const uint8_t* b_end = b_begin + (int64_t)a.N * G * 2;
-    for (int i = 0; i < nkt; ++i) {
-      const int ps = i % PST;
-      const uint32_t par = ((i / PST) & 1) ^ 1;
-      if (!mbar_wait(empty_w(ps), par, abort_flag)) break;
-      const int kt = kt0 + i;
-      const bool tail = (kt + 1) * kBK > a.K;
-      const uint32_t slot = smem_u32(pring + ps * S::kPSlot);
-      bool plain = false;
-#pragma unroll
-      for (int j = 0; j < kRowsW / 32; ++j) {
-        const int r = lane + 32 * j;
-        const int64_t row = n0 + r;
-        if (row >= a.N) continue;
-        const uint8_t* src = a.wq + row * a.row_bytes + (int64_t)kt * S::kPB;
-        const uint32_t dst = slot + r * S::kRP;
-        const int nbytes = tail ? S::kPB / 2 : S::kPB;
-        if (a.vec == 16 && !tail) {
-#pragma unroll
-          for (int o = 0; o < S::kPB; o += 16) cp_async_16(dst + o, src + o);
-        } else if (a.vec >= 8 && (nbytes % 8) == 0) {
-          for (int o = 0; o < nbytes; o += 8) cp_async_8(dst + o, src + o);
-        } else {
-          for (int o = 0; o < nbytes; o += 4) cp_async_4(dst + o, src + o);
-        }
-        const uint32_t wdst = slot + kRowsW * S::kRP + r * 16;
-        const int g0 = (kt * kBK) >> a.gs_log2;
-        if constexpr (FP4) {
-          plain |= copy_window(wdst, s_begin + row * G + g0, s_begin, s_end);
-        } else {
-          plain |= copy_window(wdst, s_begin + 2 * (row * G + g0), s_begin, s_end);
-          plain |= copy_window(wdst + 8, b_begin + 2 * (row * G + g0), b_begin, b_end);
+    if constexpr (FAST) {
+      // ------------------- weight and scale chunks by TMA, in K order
+      if (lane == 0) {
+        int c = 0, j = 0;
+        while (c < nwc || j < nsc) {
+          // K position (in codes, relative to kt0 * 64) where each chunk starts
+          const int64_t kw = c < nwc ? (int64_t)c * 128 * 8 / BITS : INT64_MAX;
+          const int64_t ks = j < nsc ? (int64_t)(sc0 + j) * SGC * (1 << a.gs_log2) - (int64_t)kt0 * kBK
+                                     : INT64_MAX;
+          if (kw <= ks) {
+            const int slot = c % WS;
+            if (!mbar_wait(empty_l(slot), ((c / WS) & 1) ^ 1, abort_flag)) break;
+            mbar_arrive_expect_tx(full_l(slot), S::kWChunk);
+            tma_load_2d(smem_u32(wring + slot * S::kWChunk), &maps.w, full_l(slot),
+                        (int)(wb0 + 128 * c), n0);
+            ++c;
+          } else {
+            const int slot = j % SS;
+            if (!mbar_wait(empty_l(WS + slot), ((j / SS) & 1) ^ 1, abort_flag)) break;
+            const uint32_t dst = smem_u32(sring + slot * S::kSChunk);
+            mbar_arrive_expect_tx(full_l(WS + slot), FP4 ? kRowsW * 16 : 2 * kRowsW * 16);
+            tma_load_2d(dst, &maps.s, full_l(WS + slot), (sc0 + j) * SGC, n0);
+            if constexpr (!FP4) tma_load_2d(dst + kRowsW * 16, &maps.b, full_l(WS + slot), (sc0 + j) * SGC, n0);
+            ++j;
+          }
         }
       }
-      if (plain) {          // rare: a window at the end of the scale arrays
-        cp_async_wait_all();
-        mbar_arrive(full_w(ps));
-      } else {
-        cp_async_arrive(full_w(ps));
+    } else {
+      // ------------------ packed codes, scales, biases by cp.async
+      // Each lane copies 4 rows per stage, one commit group per stage, and
+      // keeps kLag stages in flight: after committing stage i it waits for
+      // stage i - kLag and publishes it with a release arrive.
+      constexpr int kLag = PST - 1;
+      const uint8_t* s_begin = reinterpret_cast<const uint8_t*>(a.scales);
+      const uint8_t* s_end = s_begin + (int64_t)a.N * G * (FP4 ? 1 : 2);
+      const uint8_t* b_begin = reinterpret_cast<const uint8_t*>(a.biases);
+      const uint8_t* b_end = b_begin + (int64_t)a.N * G * 2;
+      int published = 0;
+      for (int i = 0; i < nkt; ++i) {
+        const int ps = i % PST;
+        const uint32_t par = ((i / PST) & 1) ^ 1;
+        if (!mbar_wait(empty_l(ps), par, abort_flag)) break;
+        const int kt = kt0 + i;
+        const bool tail = (kt + 1) * kBK > a.K;
+        const uint32_t slot = smem_u32(pring + ps * S::kPSlot);
+#pragma unroll
+        for (int jj = 0; jj < kRowsW / 32; ++jj) {
+          const int r = lane + 32 * jj;
+          const int64_t row = n0 + r;
+          if (row >= a.N) continue;
+          const uint8_t* src = a.wq + row * a.row_bytes + (int64_t)kt * S::kPB;
+          const uint32_t dst = slot + r * S::kRP;
+          const int nbytes = tail ? S::kPB / 2 : S::kPB;
+          if (a.vec == 16 && !tail) {
+#pragma unroll
+            for (int o = 0; o < S::kPB; o += 16) cp_async_16(dst + o, src + o);
+          } else if (a.vec >= 8 && (nbytes % 8) == 0) {
+            for (int o = 0; o < nbytes; o += 8) cp_async_8(dst + o, src + o);
+          } else {
+            for (int o = 0; o < nbytes; o += 4) cp_async_4(dst + o, src + o);
+          }
+          const uint32_t wdst = slot + kRowsW * S::kRP + r * 16;
+          const int g0 = (kt * kBK) >> a.gs_log2;
+          if constexpr (FP4) {
+            copy_window(wdst, s_begin + row * G + g0, s_begin, s_end);
+          } else {
+            copy_window(wdst, s_begin + 2 * (row * G + g0), s_begin, s_end);
+            copy_window(wdst + 8, b_begin + 2 * (row * G + g0), b_begin, b_end);
+          }
+        }
+        cp_async_commit();
+        if (i - kLag >= 0) {
+          cp_async_wait_group<kLag>();
+          mbar_arrive(full_l((i - kLag) % PST));
+          published = i - kLag + 1;
+        }
+      }
+      cp_async_wait_all();
+      if (!*abort_flag) {
+        for (int i = published; i < nkt; ++i) mbar_arrive(full_l(i % PST));
       }
     }
-    cp_async_wait_all();
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -492,25 +566,95 @@ qmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const QmmArgs a) {
     const int64_t row = n0 + r;
     const bool row_ok = row < a.N;
     const bool fp4_g16 = FP4 && a.gs_log2 == 4;
+    int w_ready = 0, w_freed = 0;                          // TMA path: chunks waited / released
+    int s_ready = 0, s_freed = 0;
     for (int i = 0; i < nkt; ++i) {
-      const int ps = i % PST;
-      if (!mbar_wait(full_w(ps), (i / PST) & 1, abort_flag)) break;
-      const uint8_t* slot = pring + ps * S::kPSlot;
       const int kt = kt0 + i;
       const bool tail = (kt + 1) * kBK > a.K;
       Packed<BITS> pk;
       StageSB sb;
-      if (row_ok) {
-        lds_packed<BITS>(pk, slot + r * S::kRP);
+      if constexpr (FAST) {
+        const int o0 = i * S::kPB;                         // row byte offset from wb0
+        const int c_hi = (o0 + S::kPB - 1) >> 7;
+        bool ok = true;
+        for (; w_ready <= c_hi && ok; ++w_ready)
+          ok = mbar_wait(full_l(w_ready % WS), (w_ready / WS) & 1, abort_flag);
+        const int sj = (((kt * kBK) >> a.gs_log2) / SGC) - sc0;
+        for (; s_ready <= sj && ok; ++s_ready)
+          ok = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
+        if (!ok) break;
+        if constexpr (S::kPB % 16 == 0) {
+#pragma unroll
+          for (int u = 0; u < S::kPB / 16; ++u) {
+            const int o = o0 + 16 * u;
+            const uint4 v = *reinterpret_cast<const uint4*>(
+                wring + ((o >> 7) % WS) * S::kWChunk + wchunk_off(o & 127, r));
+            pk.w[4 * u] = v.x; pk.w[4 * u + 1] = v.y; pk.w[4 * u + 2] = v.z; pk.w[4 * u + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < S::kPB / 8; ++u) {
+            const int o = o0 + 8 * u;
+            const uint2 v = *reinterpret_cast<const uint2*>(
+                wring + ((o >> 7) % WS) * S::kWChunk + wchunk_off(o & 127, r));
+            pk.w[2 * u] = v.x; pk.w[2 * u + 1] = v.y;
+          }
+        }
         if (tail) {
 #pragma unroll
           for (int w = BITS; w < 2 * BITS; ++w) pk.w[w] = 0u;
         }
-        const uint4 wv = *reinterpret_cast<const uint4*>(slot + kRowsW * S::kRP + r * 16);
-        sb = sb_from_words<T, FP4>(wv, a, row, kt, G, tail);
+        const uint8_t* sslot = sring + ((s_ready - 1) % SS) * S::kSChunk;
+        const int g0 = (kt * kBK) >> a.gs_log2;
+        const int g1 = tail ? g0 : ((kt * kBK + 32) >> a.gs_log2);
+        if constexpr (FP4) {
+          const uint8_t* sp = sslot + r * 16;
+          const int gs = 1 << a.gs_log2;
+          auto sc = [&](int g) { return splat(TT<T>::from_f(fp4_scale_t<T>(sp[g % SGC], gs))); };
+          if (fp4_g16) {
+            sb.s[0] = sc(g0); sb.s[1] = sc(g0 + 1);
+            sb.b[0] = tail ? sb.s[0] : sc(g0 + 2);
+            sb.b[1] = tail ? sb.s[0] : sc(g0 + 3);
+          } else {
+            sb.s[0] = sc(g0); sb.s[1] = sc(g1); sb.b[0] = sb.b[1] = 0u;
+          }
+        } else {
+          const uint16_t* sp = reinterpret_cast<const uint16_t*>(sslot + r * 16);
+          const uint16_t* bp = reinterpret_cast<const uint16_t*>(sslot + kRowsW * 16 + r * 16);
+          const uint32_t s0 = sp[g0 % SGC], s1 = sp[g1 % SGC];
+          const uint32_t b0 = bp[g0 % SGC], b1 = bp[g1 % SGC];
+          sb.s[0] = s0 | (s0 << 16); sb.s[1] = s1 | (s1 << 16);
+          sb.b[0] = b0 | (b0 << 16); sb.b[1] = b1 | (b1 << 16);
+        }
+        // release chunks this stage finished (all of them after the last stage)
+        const bool last = i + 1 == nkt;
+        const int w_done = last ? nwc : ((o0 + S::kPB) >> 7);
+        const int s_done = last ? nsc : ((((kt + 1) * kBK) >> a.gs_log2) / SGC) - sc0;
+        if (w_done > w_freed || s_done > s_freed) {
+          __syncwarp();
+          if (lane == 0) {
+            for (int c = w_freed; c < w_done; ++c) mbar_arrive(empty_l(c % WS));
+            for (int j = s_freed; j < s_done; ++j) mbar_arrive(empty_l(WS + j % SS));
+          }
+          w_freed = w_done > w_freed ? w_done : w_freed;
+          s_freed = s_done > s_freed ? s_done : s_freed;
+        }
+      } else {
+        const int ps = i % PST;
+        if (!mbar_wait(full_l(ps), (i / PST) & 1, abort_flag)) break;
+        const uint8_t* slot = pring + ps * S::kPSlot;
+        if (row_ok) {
+          lds_packed<BITS>(pk, slot + r * S::kRP);
+          if (tail) {
+#pragma unroll
+            for (int w = BITS; w < 2 * BITS; ++w) pk.w[w] = 0u;
+          }
+          const uint4 wv = *reinterpret_cast<const uint4*>(slot + kRowsW * S::kRP + r * 16);
+          sb = sb_from_words<T, FP4>(wv, a, row, kt, G, tail);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_l(ps));
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_w(ps));
       const int s = i % ST;
       if (!mbar_wait(empty(s), ((i / ST) & 1) ^ 1, abort_flag)) break;
       uint8_t* a_row = ring + s * S::kStageBytes + r * 128;
@@ -604,26 +748,27 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// x [rows, K] T, box {64, box_rows}, 128-byte swizzle, zero fill out of bounds.
-cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K, int dtype,
-                       int box_rows) {
+// 2-D tensor map over a row-major [rows, cols] array of 1- or 2-byte
+// elements; zero fill out of bounds.
+cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int esize,
+                     int64_t rows, int64_t cols, int box_cols, int box_rows,
+                     CUtensorMapSwizzle swz) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * esize)};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, dtype == AQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                   2, const_cast<void*>(x), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename T, int BITS, bool FP4, int BT>
-cudaError_t launch_tc(const QmmPlan& p, const CUtensorMap& map, const QmmArgs& a, cudaStream_t st) {
-  using S = QmmShape<BT, BITS>;
-  auto kern = qmm_tc_kernel<T, BITS, FP4, BT>;
+template <typename T, int BITS, bool FP4, int BT, bool FAST>
+cudaError_t launch_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, cudaStream_t st) {
+  using S = QmmShape<BT, BITS, FAST>;
+  auto kern = qmm_tc_kernel<T, BITS, FP4, BT, FAST>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -645,31 +790,31 @@ cudaError_t launch_tc(const QmmPlan& p, const CUtensorMap& map, const QmmArgs& a
   attr[0].val.clusterDim.z = (unsigned)p.splits;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, map, a);
+  return cudaLaunchKernelEx(&cfg, kern, maps, a);
 }
 
-template <typename T, int BITS, bool FP4>
-cudaError_t by_bt(const QmmPlan& p, const CUtensorMap& map, const QmmArgs& a, cudaStream_t st) {
+template <typename T, int BITS, bool FP4, bool FAST>
+cudaError_t by_bt(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, cudaStream_t st) {
   switch (p.bt) {
-    case 16: return launch_tc<T, BITS, FP4, 16>(p, map, a, st);
-    case 32: return launch_tc<T, BITS, FP4, 32>(p, map, a, st);
-    case 64: return launch_tc<T, BITS, FP4, 64>(p, map, a, st);
-    case 128: return launch_tc<T, BITS, FP4, 128>(p, map, a, st);
-    default: return launch_tc<T, BITS, FP4, 256>(p, map, a, st);
+    case 16: return launch_tc<T, BITS, FP4, 16, FAST>(p, maps, a, st);
+    case 32: return launch_tc<T, BITS, FP4, 32, FAST>(p, maps, a, st);
+    case 64: return launch_tc<T, BITS, FP4, 64, FAST>(p, maps, a, st);
+    case 128: return launch_tc<T, BITS, FP4, 128, FAST>(p, maps, a, st);
+    default: return launch_tc<T, BITS, FP4, 256, FAST>(p, maps, a, st);
   }
 }
 
-template <typename T>
-cudaError_t by_bits_tc(const QmmPlan& p, const CUtensorMap& map, const QmmArgs& a, int bits,
+template <typename T, bool FAST>
+cudaError_t by_bits_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, int bits,
                        int mode, cudaStream_t st) {
-  if (mode == AQ_MODE_FP4) return by_bt<T, 4, true>(p, map, a, st);
+  if (mode == AQ_MODE_FP4) return by_bt<T, 4, true, FAST>(p, maps, a, st);
   switch (bits) {
-    case 2: return by_bt<T, 2, false>(p, map, a, st);
-    case 3: return by_bt<T, 3, false>(p, map, a, st);
-    case 4: return by_bt<T, 4, false>(p, map, a, st);
-    case 5: return by_bt<T, 5, false>(p, map, a, st);
-    case 6: return by_bt<T, 6, false>(p, map, a, st);
-    case 8: return by_bt<T, 8, false>(p, map, a, st);
+    case 2: return by_bt<T, 2, false, FAST>(p, maps, a, st);
+    case 3: return by_bt<T, 3, false, FAST>(p, maps, a, st);
+    case 4: return by_bt<T, 4, false, FAST>(p, maps, a, st);
+    case 5: return by_bt<T, 5, false, FAST>(p, maps, a, st);
+    case 6: return by_bt<T, 6, false, FAST>(p, maps, a, st);
+    case 8: return by_bt<T, 8, false, FAST>(p, maps, a, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -683,7 +828,7 @@ int ilog2i(int v) {
 }  // namespace
 
 QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
-  (void)bits; (void)gs; (void)mode;
+  (void)gs; (void)mode;
   QmmPlan p{};
   const int64_t n_tiles = (N + kRowsW - 1) / kRowsW;
   const int64_t k_tiles = (K + kBK - 1) / kBK;
@@ -706,6 +851,8 @@ QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
   const int64_t tiles = p.n_tiles * p.m_tiles;
   while (splits < 8 && tiles * splits * 2 <= sms && k_tiles / (splits * 2) >= 2) splits *= 2;
   p.k_tiles_split = (int)((k_tiles + splits - 1) / splits);
+  // a K-slice must start on a 16-byte boundary of the packed rows
+  if (bits & 1) p.k_tiles_split += p.k_tiles_split & 1;
   p.splits = (int)((k_tiles + p.k_tiles_split - 1) / p.k_tiles_split);
   p.k_tiles = (int)k_tiles;
   return p;
@@ -714,8 +861,11 @@ QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
 cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const void* scales,
                        const void* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                        int gs, int mode, int dtype, cudaStream_t st) {
-  CUtensorMap map;
-  cudaError_t e = make_x_map(&map, x, M, K, dtype, p.bt);
+  QmmMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const CUtensorMapDataType tt =
+      dtype == AQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cudaError_t e = make_map(&maps.x, x, tt, 2, M, K, kBK, p.bt, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   QmmArgs a;
   a.wq = (const uint8_t*)w_q;
@@ -733,8 +883,29 @@ cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const v
   // widest copy that every row start and stage offset (8*bits bytes) allows
   a.vec = (a.row_bytes % 16 == 0 && (8 * bits) % 16 == 0) ? 16
           : (a.row_bytes % 8 == 0 && (8 * bits) % 8 == 0) ? 8 : 4;
-  return dtype == AQ_F16 ? by_bits_tc<__half>(p, map, a, bits, mode, st)
-                         : by_bits_tc<__nv_bfloat16>(p, map, a, bits, mode, st);
+  // TMA path: packed rows, scale rows and bias rows 16-byte strided and based.
+  const int64_t G = K / gs;
+  const int esz = mode == AQ_MODE_FP4 ? 1 : 2;
+  const bool fast = a.row_bytes % 16 == 0 && (G * esz) % 16 == 0 &&
+                    ((uintptr_t)scales & 15) == 0 &&
+                    (mode == AQ_MODE_FP4 || ((uintptr_t)biases & 15) == 0);
+  if (fast) {
+    e = make_map(&maps.w, w_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, a.row_bytes, 128, kRowsW,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    const CUtensorMapDataType st_t =
+        mode == AQ_MODE_FP4 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+    e = make_map(&maps.s, scales, st_t, esz, N, G, 16 / esz, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+    if (mode != AQ_MODE_FP4) {
+      e = make_map(&maps.b, biases, st_t, esz, N, G, 16 / esz, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (e != cudaSuccess) return e;
+    }
+    return dtype == AQ_F16 ? by_bits_tc<__half, true>(p, maps, a, bits, mode, st)
+                           : by_bits_tc<__nv_bfloat16, true>(p, maps, a, bits, mode, st);
+  }
+  return dtype == AQ_F16 ? by_bits_tc<__half, false>(p, maps, a, bits, mode, st)
+                         : by_bits_tc<__nv_bfloat16, false>(p, maps, a, bits, mode, st);
 }
 
 cudaError_t read_device_error(unsigned* out) {
