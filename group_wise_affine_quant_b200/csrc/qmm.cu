@@ -49,9 +49,10 @@ using namespace sm100;
 
 constexpr int kBK = 64;                  // K elements per stage (128 bytes of T)
 constexpr int kRowsW = 128;              // weight rows per tile (MMA M)
-constexpr int kThreads = 224;            // 7 warps
-constexpr int kProducerWarp0 = 2;        // warps 2..5 dequantize and run the epilogue
-constexpr int kLoaderWarp = 6;           // streams packed codes, scales, biases
+constexpr int kThreads = 352;            // 11 warps
+constexpr int kProducerWarp0 = 2;        // warps 2..9: two groups of 4 dequantizer warps
+constexpr int kDqGroups = 2;             // group g takes K-stages i with i % 2 == g
+constexpr int kLoaderWarp = 10;          // streams packed codes, scales, biases
 
 template <int BT, int BITS, bool FAST>
 struct QmmShape {
@@ -428,7 +429,9 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     }
     for (int s = 0; s < NL; ++s) {
       mbar_init(full_l(s), FAST ? 1 : 32);   // TMA arrive + tx, or every loader lane
-      mbar_init(empty_l(s), 4);              // one arrive per dequantizer warp
+      // TMA path: every chunk spans >= 2 K-stages, so both dequantizer
+      // groups release it; cp.async path: one stage, one group.
+      mbar_init(empty_l(s), FAST ? 4 * kDqGroups : 4);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -562,13 +565,14 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     }
   } else {
     // ------------------------------------------- dequantizers (warps 2..5)
-    const int r = threadIdx.x - kProducerWarp0 * 32;       // weight row in the tile
+    const int grp = (warp - kProducerWarp0) >> 2;          // dequantizer group
+    const int r = ((warp - kProducerWarp0) & 3) * 32 + lane; // weight row in the tile
     const int64_t row = n0 + r;
     const bool row_ok = row < a.N;
     const bool fp4_g16 = FP4 && a.gs_log2 == 4;
     int w_ready = 0, w_freed = 0;                          // TMA path: chunks waited / released
     int s_ready = 0, s_freed = 0;
-    for (int i = 0; i < nkt; ++i) {
+    for (int i = grp; i < nkt; i += kDqGroups) {
       const int kt = kt0 + i;
       const bool tail = (kt + 1) * kBK > a.K;
       Packed<BITS> pk;
@@ -626,10 +630,12 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
           sb.s[0] = s0 | (s0 << 16); sb.s[1] = s1 | (s1 << 16);
           sb.b[0] = b0 | (b0 << 16); sb.b[1] = b1 | (b1 << 16);
         }
-        // release chunks this stage finished (all of them after the last stage)
-        const bool last = i + 1 == nkt;
-        const int w_done = last ? nwc : ((o0 + S::kPB) >> 7);
-        const int s_done = last ? nsc : ((((kt + 1) * kBK) >> a.gs_log2) / SGC) - sc0;
+        // release the chunks this group is done with: those that end before
+        // its next stage starts (all of them after its last stage)
+        const bool last = i + kDqGroups >= nkt;
+        const int w_done = last ? nwc : (((i + kDqGroups) * S::kPB) >> 7);
+        const int s_done =
+            last ? nsc : ((((kt + kDqGroups) * kBK) >> a.gs_log2) / SGC) - sc0;
         if (w_done > w_freed || s_done > s_freed) {
           __syncwarp();
           if (lane == 0) {
@@ -669,6 +675,24 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(full_a(s));
     }
+    if constexpr (FAST) {
+      // Chunks past this group's last stage are released too (both groups
+      // release every chunk), but only after their data has landed: the
+      // landing proves the slot's previous chunk was released by both
+      // groups, so this arrival counts toward the right phase.
+      bool ok = !*abort_flag;
+      for (; w_ready < nwc && ok; ++w_ready)
+        ok = mbar_wait(full_l(w_ready % WS), (w_ready / WS) & 1, abort_flag);
+      for (; s_ready < nsc && ok; ++s_ready)
+        ok = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
+      if (ok && (w_freed < nwc || s_freed < nsc)) {
+        __syncwarp();
+        if (lane == 0) {
+          for (int c = w_freed; c < nwc; ++c) mbar_arrive(empty_l(c % WS));
+          for (int j = s_freed; j < nsc; ++j) mbar_arrive(empty_l(WS + j % SS));
+        }
+      }
+    }
 
     // ------------------------------------------------------- epilogue
     const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, 4000000000ull);
@@ -679,7 +703,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     float* red = reinterpret_cast<float*>(ring);            // [BT][128] when split
     if (acc_ok && !*abort_flag) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < BT; c0 += 16) {
+      for (int c0 = 16 * grp; c0 < BT; c0 += 16 * kDqGroups) {
         uint32_t v[16];
         tmem_ld_16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
         tmem_ld_wait();
