@@ -161,9 +161,10 @@ aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void*
 }
 
 unsigned aq_device_errors(void) {
-  unsigned v = 0;
-  if (aq::read_device_error(&v) != cudaSuccess) return 0xFFFFFFFFu;
-  return v;
+  unsigned v = 0, w = 0;
+  if (aq::read_device_error_qmm(&v) != cudaSuccess) return 0xFFFFFFFFu;
+  if (aq::read_device_error_conv(&w) != cudaSuccess) return 0xFFFFFFFFu;
+  return v | w;
 }
 
 aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* scales,
@@ -172,11 +173,36 @@ aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* scales,
                           int pad_w, int groups, int bits, int group_size, aq_dtype dtype,
                           void* workspace, size_t workspace_bytes, aq_stream_t stream) {
   g_err[0] = 0;
-  (void)x; (void)w_q; (void)scales; (void)biases; (void)y; (void)B; (void)H; (void)W;
-  (void)Cin; (void)Cout; (void)kh; (void)kw; (void)stride_h; (void)stride_w; (void)pad_h;
-  (void)pad_w; (void)groups; (void)bits; (void)group_size; (void)dtype; (void)workspace;
-  (void)workspace_bytes; (void)stream;
-  return fail(AQ_ERR_UNSUPPORTED, "aq_qconv2d_nhwc is not built yet");
+  (void)workspace; (void)workspace_bytes;
+  aq_status st = check_format(bits, group_size, AQ_MODE_AFFINE, dtype);
+  if (st != AQ_OK) return st;
+  if (B < 0 || H < 0 || W < 0 || Cin <= 0 || Cout <= 0 || kh <= 0 || kw <= 0 ||
+      stride_h <= 0 || stride_w <= 0 || pad_h < 0 || pad_w < 0 || groups <= 0)
+    return fail(AQ_ERR_INVALID_ARG, "conv sizes must be positive (pads >= 0)");
+  if (Cin % groups || Cout % groups)
+    return fail(AQ_ERR_INVALID_ARG, "Cin=%d and Cout=%d must be multiples of groups=%d", Cin, Cout, groups);
+  if ((Cin / groups) % 8)
+    return fail(AQ_ERR_UNSUPPORTED, "Cin/groups=%d must be a multiple of 8 (16-byte channel runs)", Cin / groups);
+  const int64_t Ho = ((int64_t)H + 2 * pad_h - kh) / stride_h + 1;
+  const int64_t Wo = ((int64_t)W + 2 * pad_w - kw) / stride_w + 1;
+  if (H + 2 * pad_h < kh || W + 2 * pad_w < kw)
+    return fail(AQ_ERR_INVALID_ARG, "kernel %dx%d larger than the padded input", kh, kw);
+  const int64_t M = (int64_t)B * Ho * Wo;
+  const int64_t Kreal = (int64_t)kh * kw * (Cin / groups);
+  const int64_t Kp = (Kreal + group_size - 1) / group_size * group_size;
+  if (M > kMaxDim || Kp > kMaxDim || (int64_t)B * H * W * Cin > ((int64_t)1 << 40))
+    return fail(AQ_ERR_INVALID_ARG, "conv problem too large");
+  if (M == 0) return AQ_OK;
+  if (!x || !y || !w_q || !scales || !biases)
+    return fail(AQ_ERR_INVALID_ARG, "x, y, w_q, scales and biases must not be NULL");
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(w_q, 16))
+    return fail(AQ_ERR_MISALIGNED, "x, y and w_q must be 16-byte aligned");
+  if (!aligned(scales, 2) || !aligned(biases, 2))
+    return fail(AQ_ERR_MISALIGNED, "scales and biases must be 2-byte aligned");
+  return cuda_status(aq::launch_qconv(x, w_q, scales, biases, y, B, H, W, Cin, Cout, kh, kw,
+                                      stride_h, stride_w, pad_h, pad_w, groups, bits, group_size,
+                                      dtype, (cudaStream_t)stream),
+                     "aq_qconv2d_nhwc launch");
 }
 
 size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size,

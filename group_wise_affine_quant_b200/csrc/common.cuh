@@ -117,5 +117,10 @@ QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode);
 cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const void* scales,
                        const void* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                        int gs, int mode, int dtype, cudaStream_t st);
-cudaError_t read_device_error(unsigned* out);
+cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, const void* biases,
+                         void* y, int Bn, int H, int W, int Cin, int Cout, int kh, int kw,
+                         int sh, int sw, int ph, int pw, int groups, int bits, int gs, int dtype,
+                         cudaStream_t st);
+cudaError_t read_device_error_qmm(unsigned* out);
+cudaError_t read_device_error_conv(unsigned* out);
 }  // namespace aq

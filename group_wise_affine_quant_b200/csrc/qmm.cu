@@ -1,855 +1,9 @@
-// qmm.cu — tensor-core quantized matmul y = x . dequant(W)^T (tcgen05 + TMEM).
-//
-// Prior art: affine_packed_qmm_t in "Add the 3bit packed qmm_t" (a block
-// loader dequantizes a weight tile into threadgroup memory, then a simdgroup
-// MMA).  The B200 design, per CTA and output tile of 128 weight rows x BT
-// rows of x:
-//   * The weight is the MMA's A operand (M = 128 rows of N) and x is the B
-//     operand (N = BT in 16..256 rows of M), so a decode-sized M still fills a
-//     full 128-row MMA: one wave of tiles covers M = 1..64 at the weight
-//     stream's cost.
-//   * Warp 0 (one thread) loads x tiles with TMA into 128-byte-swizzled shared
-//     memory; warp 6 streams the packed codes and the words holding each
-//     row's scales and biases into a deep shared-memory ring with cp.async,
-//     completing on an mbarrier; warp 1 allocates TMEM and one of its threads
-//     issues tcgen05.mma (kind::f16, fp32 accumulate in TMEM); warps 2-5 are
-//     the dequantizers (one weight row per thread): from shared memory they
-//     form w_hat = s*q + b in T with packed half2/bfloat162 FMAs (single
-//     rounding, the same value aq_dequantize writes) and store it in the
-//     swizzled K-major layout.  The dequantizers issue no global loads, so
-//     their async-proxy fence before each hand-over never waits on memory
-//     latency.  Stages hand over through mbarriers; the MMA's commit frees an
-//     operand stage for both producers.
-//   * K-step 64 (one 128-byte swizzle atom of 16-bit values); a K tail of 32
-//     reads zero x through TMA's out-of-bounds fill and writes zero w_hat.
-//   * The epilogue (warps 2-5) reads TMEM with tcgen05.ld.  With split-K the
-//     K-slices of a tile form a thread block cluster: each CTA parks its fp32
-//     tile in shared memory and the slices are added in slice order through
-//     distributed shared memory.  No workspace, no global atomics.
-//   * Every mbarrier wait is bounded (2 s); a timeout sets a device error
-//     flag, every role stops issuing work and the CTA frees its TMEM.
-#include <cooperative_groups.h>
-
-#include <string.h>
-
-#include <type_traits>
-
-#include "common.cuh"
-#include "sm100.cuh"
-
-namespace cg = cooperative_groups;
+// qmm.cu — dense entry of the tensor-core quantized matmul: plan and launch
+// of y = x . dequant(W)^T with x [M, K] read by 2-D TMA (kernel template in
+// qmm_kernel.cuh).
+#include "qmm_kernel.cuh"
 
 namespace aq {
-
-__device__ unsigned int g_aq_device_error = 0u;   // bit 0: a wait timed out
-
-namespace {
-
-using namespace sm100;
-
-constexpr int kBK = 64;                  // K elements per stage (128 bytes of T)
-constexpr int kRowsW = 128;              // weight rows per tile (MMA M)
-constexpr int kThreads = 352;            // 11 warps
-constexpr int kProducerWarp0 = 2;        // warps 2..9: two groups of 4 dequantizer warps
-constexpr int kDqGroups = 2;             // group g takes K-stages i with i % 2 == g
-constexpr int kLoaderWarp = 10;          // streams packed codes, scales, biases
-
-template <int BT, int BITS, bool FAST>
-struct QmmShape {
-  static constexpr int kStages = BT >= 256 ? 3 : 4;                 // operand stages
-  static constexpr int kABytes = kRowsW * kBK * 2;                   // 16 KB
-  static constexpr int kBBytes = BT * kBK * 2;                       // BT * 128
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kPB = 8 * BITS;                               // packed bytes / row / stage
-  // cp.async path: one slot per stage, rows at a bank-spreading pitch.
-  static constexpr int kPStages = BT >= 256 ? 4 : BT >= 128 ? 6 : BT >= 64 ? 8 : BT >= 32 ? 10 : 12;
-  static constexpr int kRP = (kPB % 32 == 0) ? kPB + 16 : kPB;
-  static constexpr int kPSlot = kRowsW * kRP + kRowsW * 16;
-  // TMA path: weight chunks of 128 rows x 128 bytes (128-byte swizzle) and
-  // scale chunks of 128 rows x 16 bytes (scales, then biases).
-  static constexpr int kWChunk = kRowsW * 128;                       // 16 KB
-  static constexpr int kWSlots = BT >= 256 ? 2 : BT >= 128 ? 3 : 4;
-  static constexpr int kSChunk = kRowsW * 16 * 2;                    // 4 KB
-  static constexpr int kSSlots = 4;
-  static constexpr int kLoadBytes = FAST ? kWSlots * kWChunk + kSSlots * kSChunk : kPStages * kPSlot;
-  static constexpr int kRedBytes = BT * kRowsW * 4;                  // split-K parking
-  static constexpr int kRingBytes = kStages * kStageBytes;
-  static constexpr int kOpBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
-  static constexpr int kDataBytes = kOpBytes + kLoadBytes;
-  static constexpr int kTmemCols = BT < 32 ? 32 : BT;
-  static constexpr int kBars = 3 * kStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
-  static constexpr int kSmem = 1024 + kDataBytes + 512;             // align slack, barriers
-  static_assert(kBars * 8 + 16 <= 512, "barrier area");
-  static_assert(kSmem <= 227 * 1024, "shared memory budget");
-};
-
-struct QmmArgs {
-  const uint8_t* wq;
-  const void* scales;
-  const void* biases;
-  void* y;
-  int M, N, K;
-  int gs_log2;
-  int k_tiles;          // ceil(K / 64)
-  int k_tiles_split;    // k-tiles per split
-  int splits;
-  int vec;              // widest cp.async (16, 8 or 4 bytes) the packed rows allow
-  int64_t row_bytes;
-};
-
-struct QmmMaps {
-  CUtensorMap x;        // [M, K] T, box {64, BT}, 128-byte swizzle
-  CUtensorMap w;        // [N, row_bytes] u8, box {128, 128}, 128-byte swizzle (TMA path)
-  CUtensorMap s;        // [N, G] scales, box {16 bytes, 128} (TMA path)
-  CUtensorMap b;        // [N, G] biases, likewise (affine)
-};
-
-// ------------------------------------------------------------ cp.async
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-// Wait until at most N of this thread's committed groups are still in flight.
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
-// Copy the two 4-byte words starting at the 4-byte boundary at or below
-// `p` (a 2- or 1-byte element of an array that ends at `end`) into dst.
-// Words that stick out of the array are filled with byte loads of their
-// in-bounds part (and zeros) and plain shared stores.
-__device__ __forceinline__ void copy_window(uint32_t dst, const uint8_t* p, const uint8_t* begin,
-                                            const uint8_t* end) {
-  const uint8_t* w0 = reinterpret_cast<const uint8_t*>((uintptr_t)p & ~(uintptr_t)3);
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const uint8_t* w = w0 + 4 * i;
-    if (w >= begin && w + 4 <= end) {
-      cp_async_4(dst + 4 * i, w);
-    } else {
-      uint32_t v = 0;
-      for (int j = 0; j < 4; ++j)
-        if (w + j >= begin && w + j < end) v |= (uint32_t)w[j] << (8 * j);
-      asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst + 4 * i), "r"(v) : "memory");
-    }
-  }
-}
-
-// ------------------------------------------------------------- dequantizer
-// Per thread and stage: the 64 codes of one weight row as 2*BITS words.
-template <int BITS>
-struct Packed {
-  static constexpr int kWords = 2 * BITS;
-  uint32_t w[kWords];
-};
-
-template <int BITS>
-__device__ __forceinline__ void lds_packed(Packed<BITS>& p, const uint8_t* src) {
-  if constexpr ((8 * BITS) % 16 == 0) {
-#pragma unroll
-    for (int i = 0; i < BITS / 2; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
-      p.w[4 * i] = v.x; p.w[4 * i + 1] = v.y; p.w[4 * i + 2] = v.z; p.w[4 * i + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < BITS; ++i) {
-      const uint2 v = *reinterpret_cast<const uint2*>(src + 8 * i);
-      p.w[2 * i] = v.x; p.w[2 * i + 1] = v.y;
-    }
-  }
-}
-
-template <typename T> struct Pair;
-template <> struct Pair<__half> {
-  static constexpr uint32_t kMagic = 0x64006400u;            // 1024.0 in each half
-  static __device__ __forceinline__ uint32_t sub_magic(uint32_t v) {
-    __half2 h = *reinterpret_cast<__half2*>(&v);
-    h = __hsub2(h, __half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
-    return *reinterpret_cast<uint32_t*>(&h);
-  }
-  static __device__ __forceinline__ uint32_t fma(uint32_t q, uint32_t s, uint32_t b) {
-    __half2 r = __hfma2(*reinterpret_cast<__half2*>(&q), *reinterpret_cast<__half2*>(&s),
-                        *reinterpret_cast<__half2*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-  }
-  static __device__ __forceinline__ uint32_t mul(uint32_t a, uint32_t b) {
-    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-  }
-  static __device__ __forceinline__ uint32_t from_f2(float lo, float hi) {
-    __half2 r = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&r);
-  }
-  static constexpr int kMagicMaxCode = 1023;
-};
-template <> struct Pair<__nv_bfloat16> {
-  static constexpr uint32_t kMagic = 0x43004300u;            // 128.0 in each half
-  static __device__ __forceinline__ uint32_t sub_magic(uint32_t v) {
-    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
-    h = __hsub2(h, __nv_bfloat162(__ushort_as_bfloat16(0x4300), __ushort_as_bfloat16(0x4300)));
-    return *reinterpret_cast<uint32_t*>(&h);
-  }
-  static __device__ __forceinline__ uint32_t fma(uint32_t q, uint32_t s, uint32_t b) {
-    __nv_bfloat162 r = __hfma2(*reinterpret_cast<__nv_bfloat162*>(&q),
-                               *reinterpret_cast<__nv_bfloat162*>(&s),
-                               *reinterpret_cast<__nv_bfloat162*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-  }
-  static __device__ __forceinline__ uint32_t mul(uint32_t a, uint32_t b) {
-    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a),
-                               *reinterpret_cast<__nv_bfloat162*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-  }
-  static __device__ __forceinline__ uint32_t from_f2(float lo, float hi) {
-    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&r);
-  }
-  static constexpr int kMagicMaxCode = 127;
-};
-
-// Exact codes of elements (2j, 2j+1) of chunk c as a T pair.
-template <typename T, int BITS, int C, int J>
-__device__ __forceinline__ uint32_t code_pair(const Packed<BITS>& p) {
-  constexpr int k0 = 8 * C + 2 * J;
-  if constexpr (BITS == 4) {
-    // byte J of word C holds codes 2J (low nibble) and 2J+1 (high nibble):
-    // put byte J of w at byte 0 and byte J of w >> 4 at byte 2, keep the low
-    // nibbles, OR in the magic exponent and subtract it.
-    const uint32_t w = p.w[C];
-    constexpr uint32_t sel = (uint32_t)J | ((uint32_t)J << 4) | ((uint32_t)(J + 4) << 8) |
-                             ((uint32_t)(J + 4) << 12);
-    const uint32_t t = __byte_perm(w, w >> 4, sel);
-    return Pair<T>::sub_magic((t & 0x000F000Fu) | Pair<T>::kMagic);
-  } else if constexpr (BITS == 8 && std::is_same<T, __nv_bfloat16>::value) {
-    const float lo = u_to_f_exact(code_at<8, k0>(p.w));
-    const float hi = u_to_f_exact(code_at<8, k0 + 1>(p.w));
-    return Pair<T>::from_f2(lo, hi);
-  } else {
-    const uint32_t lo = code_at<BITS, k0>(p.w);
-    const uint32_t hi = code_at<BITS, k0 + 1>(p.w);
-    return Pair<T>::sub_magic(lo | (hi << 16) | Pair<T>::kMagic);
-  }
-}
-
-template <typename T, int C, int J>
-__device__ __forceinline__ uint32_t fp4_pair(const Packed<4>& p) {
-  constexpr int k0 = 8 * C + 2 * J;
-  return Pair<T>::from_f2(e2m1_to_float(code_at<4, k0>(p.w)), e2m1_to_float(code_at<4, k0 + 1>(p.w)));
-}
-
-// Dequantize chunk C (8 elements) into 16 bytes.
-template <typename T, int BITS, bool FP4, int C>
-__device__ __forceinline__ uint4 dequant_chunk(const Packed<BITS>& p, uint32_t s2, uint32_t b2) {
-  uint4 o;
-  if constexpr (FP4) {
-    o.x = Pair<T>::mul(fp4_pair<T, C, 0>(p), s2);
-    o.y = Pair<T>::mul(fp4_pair<T, C, 1>(p), s2);
-    o.z = Pair<T>::mul(fp4_pair<T, C, 2>(p), s2);
-    o.w = Pair<T>::mul(fp4_pair<T, C, 3>(p), s2);
-  } else {
-    o.x = Pair<T>::fma(code_pair<T, BITS, C, 0>(p), s2, b2);
-    o.y = Pair<T>::fma(code_pair<T, BITS, C, 1>(p), s2, b2);
-    o.z = Pair<T>::fma(code_pair<T, BITS, C, 2>(p), s2, b2);
-    o.w = Pair<T>::fma(code_pair<T, BITS, C, 3>(p), s2, b2);
-  }
-  return o;
-}
-
-template <typename T>
-__device__ __forceinline__ uint32_t splat(T v) {
-  const uint16_t u = *reinterpret_cast<const uint16_t*>(&v);
-  return (uint32_t)u | ((uint32_t)u << 16);
-}
-
-// Scale/bias pairs (splatted T) for the two 32-element halves of a stage;
-// FP4 at group 16 keeps its four quarter scales in s[0], s[1], b[0], b[1].
-struct StageSB {
-  uint32_t s[2], b[2];
-};
-
-__device__ __forceinline__ uint32_t u16_at(uint32_t w0, uint32_t w1, int byte_off) {
-  const uint64_t v = ((uint64_t)w1 << 32) | w0;
-  return (uint32_t)(v >> (8 * byte_off)) & 0xFFFFu;
-}
-__device__ __forceinline__ uint32_t u8_at(uint32_t w0, uint32_t w1, int byte_off) {
-  const uint64_t v = ((uint64_t)w1 << 32) | w0;
-  return (uint32_t)(v >> (8 * byte_off)) & 0xFFu;
-}
-
-// Decode the staged words of one row into the stage's scale/bias pairs.
-template <typename T, bool FP4>
-__device__ __forceinline__ StageSB sb_from_words(const uint4 wv, const QmmArgs& a, int64_t row,
-                                                 int kt, int G, bool tail) {
-  StageSB r;
-  const int k = kt * kBK;
-  const int g0 = k >> a.gs_log2;
-  const int g1 = tail ? g0 : (k + 32) >> a.gs_log2;
-  if constexpr (FP4) {
-    const uint8_t* p = reinterpret_cast<const uint8_t*>(a.scales) + row * G + g0;
-    const int off = (int)((uintptr_t)p & 3);
-    auto sc = [&](int d) {
-      return splat(TT<T>::from_f(fp4_scale_t<T>(u8_at(wv.x, wv.y, off + d), 1 << a.gs_log2)));
-    };
-    if (a.gs_log2 == 4) {
-      r.s[0] = sc(0);
-      r.s[1] = sc(1);
-      r.b[0] = tail ? r.s[0] : sc(2);
-      r.b[1] = tail ? r.s[0] : sc(3);
-    } else {
-      r.s[0] = sc(0);
-      r.s[1] = sc(g1 - g0);
-      r.b[0] = r.b[1] = 0u;
-    }
-  } else {
-    const int offs = (int)(((uintptr_t)a.scales + 2 * (row * G + g0)) & 3);
-    const int offb = (int)(((uintptr_t)a.biases + 2 * (row * G + g0)) & 3);
-    const uint32_t s0 = u16_at(wv.x, wv.y, offs), s1 = u16_at(wv.x, wv.y, offs + 2 * (g1 - g0));
-    const uint32_t b0 = u16_at(wv.z, wv.w, offb), b1 = u16_at(wv.z, wv.w, offb + 2 * (g1 - g0));
-    r.s[0] = s0 | (s0 << 16);
-    r.s[1] = s1 | (s1 << 16);
-    r.b[0] = b0 | (b0 << 16);
-    r.b[1] = b1 | (b1 << 16);
-  }
-  return r;
-}
-
-template <typename T, int BITS, bool FP4>
-__device__ __forceinline__ void dequant_stage(const Packed<BITS>& p, const StageSB& sb, bool fp4_g16,
-                                              uint8_t* a_row, int r, bool tail) {
-  // chunk c of 8 elements lands at 16-byte slot c ^ (r & 7) of the row
-  const int sw = r & 7;
-  auto put = [&](int c, uint4 v) {
-    *reinterpret_cast<uint4*>(a_row + ((c ^ sw) << 4)) = v;
-  };
-  if constexpr (FP4) {
-    // quarters of 16 elements: scales s0 s1 (g16: b0 b1 hold quarters 2, 3)
-    const uint32_t q0 = sb.s[0];
-    const uint32_t q1 = fp4_g16 ? sb.s[1] : sb.s[0];
-    const uint32_t q2 = fp4_g16 ? sb.b[0] : sb.s[1];
-    const uint32_t q3 = fp4_g16 ? sb.b[1] : sb.s[1];
-    put(0, dequant_chunk<T, BITS, FP4, 0>(p, q0, 0u));
-    put(1, dequant_chunk<T, BITS, FP4, 1>(p, q0, 0u));
-    put(2, dequant_chunk<T, BITS, FP4, 2>(p, q1, 0u));
-    put(3, dequant_chunk<T, BITS, FP4, 3>(p, q1, 0u));
-    if (!tail) {
-      put(4, dequant_chunk<T, BITS, FP4, 4>(p, q2, 0u));
-      put(5, dequant_chunk<T, BITS, FP4, 5>(p, q2, 0u));
-      put(6, dequant_chunk<T, BITS, FP4, 6>(p, q3, 0u));
-      put(7, dequant_chunk<T, BITS, FP4, 7>(p, q3, 0u));
-    }
-  } else {
-    put(0, dequant_chunk<T, BITS, FP4, 0>(p, sb.s[0], sb.b[0]));
-    put(1, dequant_chunk<T, BITS, FP4, 1>(p, sb.s[0], sb.b[0]));
-    put(2, dequant_chunk<T, BITS, FP4, 2>(p, sb.s[0], sb.b[0]));
-    put(3, dequant_chunk<T, BITS, FP4, 3>(p, sb.s[0], sb.b[0]));
-    if (!tail) {
-      put(4, dequant_chunk<T, BITS, FP4, 4>(p, sb.s[1], sb.b[1]));
-      put(5, dequant_chunk<T, BITS, FP4, 5>(p, sb.s[1], sb.b[1]));
-      put(6, dequant_chunk<T, BITS, FP4, 6>(p, sb.s[1], sb.b[1]));
-      put(7, dequant_chunk<T, BITS, FP4, 7>(p, sb.s[1], sb.b[1]));
-    }
-  }
-  if (tail) {
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    put(4, z); put(5, z); put(6, z); put(7, z);
-  }
-}
-
-// -------------------------------------------------------------------- kernel
-// Shared memory offset of byte `o` of row r within a chain of 128-byte
-// weight chunks (128-byte swizzle: 16-byte unit u of row r sits at unit
-// u ^ (r % 8)).
-__device__ __forceinline__ uint32_t wchunk_off(int o, int r) {
-  return (uint32_t)(r * 128 + ((((o >> 4) & 7) ^ (r & 7)) << 4) + (o & 15));
-}
-
-template <typename T, int BITS, bool FP4, int BT, bool FAST>
-__global__ void __launch_bounds__(kThreads, 1)
-qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
-  using S = QmmShape<BT, BITS, FAST>;
-  constexpr int ST = S::kStages;
-  constexpr int PST = S::kPStages;
-  constexpr int WS = S::kWSlots;
-  constexpr int SS = S::kSSlots;
-  constexpr int SGC = FP4 ? 16 : 8;                       // groups per scale chunk (16 bytes)
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* ring = smem;                                   // [ST] x (A 16 KB | B BT*128)
-  uint8_t* pring = smem + S::kOpBytes;                    // loader area
-  uint8_t* wring = pring;                                 // TMA path: [WS] weight chunks
-  uint8_t* sring = pring + WS * S::kWChunk;               // TMA path: [SS] scale chunks
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kDataBytes);
-  constexpr int NL = FAST ? WS + SS : PST;                // loader slots
-  // bars: full_a[ST], full_b[ST], empty[ST], full_l[NL], empty_l[NL], acc_full
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kRowsW;
-  const int m0 = blockIdx.y * BT;
-  const int split = blockIdx.z;
-  const int kt0 = split * a.k_tiles_split;
-  const int kt1 = min(a.k_tiles, kt0 + a.k_tiles_split);
-  const int nkt = kt1 - kt0;                              // >= 1
-  const int G = a.K >> a.gs_log2;
-
-  auto full_a = [&](int s) { return smem_u32(bars + s); };
-  auto full_b = [&](int s) { return smem_u32(bars + ST + s); };
-  auto empty = [&](int s) { return smem_u32(bars + 2 * ST + s); };
-  auto full_l = [&](int s) { return smem_u32(bars + 3 * ST + s); };
-  auto empty_l = [&](int s) { return smem_u32(bars + 3 * ST + NL + s); };
-  const uint32_t acc_full = smem_u32(bars + 3 * ST + 2 * NL);
-
-  // TMA path bookkeeping: weight chunk c covers bytes [wb0 + 128 c, +128) of
-  // every row, scale chunk j covers groups [SGC j, SGC (j + 1)).
-  const int64_t wb0 = (int64_t)kt0 * S::kPB;              // 16-byte aligned (host plan)
-  const int nwc = (int)((nkt * S::kPB + 127) / 128);
-  const int sc0 = ((kt0 * kBK) >> a.gs_log2) / SGC;
-  const int sc1 = (((kt1 * kBK) - 1) >> a.gs_log2) / SGC;
-  const int nsc = sc1 - sc0 + 1;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(full_a(s), 4);          // one arrive per dequantizer warp
-      mbar_init(full_b(s), 1);          // TMA producer's arrive + tx bytes
-      mbar_init(empty(s), 1);           // MMA commit
-    }
-    for (int s = 0; s < NL; ++s) {
-      mbar_init(full_l(s), FAST ? 1 : 32);   // TMA arrive + tx, or every loader lane
-      // TMA path: every chunk spans >= 2 K-stages, so both dequantizer
-      // groups release it; cp.async path: one stage, one group.
-      mbar_init(empty_l(s), FAST ? 4 * kDqGroups : 4);
-    }
-    mbar_init(acc_full, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
-    tc_fence_before();
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ---------------------------------------------------- TMA producer (x)
-    if (lane == 0) {
-      for (int i = 0; i < nkt; ++i) {
-        const int s = i % ST;
-        const uint32_t par = ((i / ST) & 1) ^ 1;
-        if (!mbar_wait(empty(s), par, abort_flag)) break;
-        mbar_arrive_expect_tx(full_b(s), S::kBBytes);
-        tma_load_2d(smem_u32(ring + s * S::kStageBytes + S::kABytes), &maps.x, full_b(s),
-                    (kt0 + i) * kBK, m0);
-      }
-    }
-  } else if (warp == kLoaderWarp) {
-    if constexpr (FAST) {
-      // ------------------- weight and scale chunks by TMA, in K order
-      if (lane == 0) {
-        int c = 0, j = 0;
-        while (c < nwc || j < nsc) {
-          // K position (in codes, relative to kt0 * 64) where each chunk starts
-          const int64_t kw = c < nwc ? (int64_t)c * 128 * 8 / BITS : INT64_MAX;
-          const int64_t ks = j < nsc ? (int64_t)(sc0 + j) * SGC * (1 << a.gs_log2) - (int64_t)kt0 * kBK
-                                     : INT64_MAX;
-          if (kw <= ks) {
-            const int slot = c % WS;
-            if (!mbar_wait(empty_l(slot), ((c / WS) & 1) ^ 1, abort_flag)) break;
-            mbar_arrive_expect_tx(full_l(slot), S::kWChunk);
-            tma_load_2d(smem_u32(wring + slot * S::kWChunk), &maps.w, full_l(slot),
-                        (int)(wb0 + 128 * c), n0);
-            ++c;
-          } else {
-            const int slot = j % SS;
-            if (!mbar_wait(empty_l(WS + slot), ((j / SS) & 1) ^ 1, abort_flag)) break;
-            const uint32_t dst = smem_u32(sring + slot * S::kSChunk);
-            mbar_arrive_expect_tx(full_l(WS + slot), FP4 ? kRowsW * 16 : 2 * kRowsW * 16);
-            tma_load_2d(dst, &maps.s, full_l(WS + slot), (sc0 + j) * SGC, n0);
-            if constexpr (!FP4) tma_load_2d(dst + kRowsW * 16, &maps.b, full_l(WS + slot), (sc0 + j) * SGC, n0);
-            ++j;
-          }
-        }
-      }
-    } else {
-      // ------------------ packed codes, scales, biases by cp.async
-      // Each lane copies 4 rows per stage, one commit group per stage, and
-      // keeps kLag stages in flight: after committing stage i it waits for
-      // stage i - kLag and publishes it with a release arrive.
-      constexpr int kLag = PST - 1;
-      const uint8_t* s_begin = reinterpret_cast<const uint8_t*>(a.scales);
-      const uint8_t* s_end = s_begin + (int64_t)a.N * G * (FP4 ? 1 : 2);
-      const uint8_t* b_begin = reinterpret_cast<const uint8_t*>(a.biases);
-      const uint8_t* b_end = b_begin + (int64_t)a.N * G * 2;
-      int published = 0;
-      for (int i = 0; i < nkt; ++i) {
-        const int ps = i % PST;
-        const uint32_t par = ((i / PST) & 1) ^ 1;
-        if (!mbar_wait(empty_l(ps), par, abort_flag)) break;
-        const int kt = kt0 + i;
-        const bool tail = (kt + 1) * kBK > a.K;
-        const uint32_t slot = smem_u32(pring + ps * S::kPSlot);
-#pragma unroll
-        for (int jj = 0; jj < kRowsW / 32; ++jj) {
-          const int r = lane + 32 * jj;
-          const int64_t row = n0 + r;
-          if (row >= a.N) continue;
-          const uint8_t* src = a.wq + row * a.row_bytes + (int64_t)kt * S::kPB;
-          const uint32_t dst = slot + r * S::kRP;
-          const int nbytes = tail ? S::kPB / 2 : S::kPB;
-          if (a.vec == 16 && !tail) {
-#pragma unroll
-            for (int o = 0; o < S::kPB; o += 16) cp_async_16(dst + o, src + o);
-          } else if (a.vec >= 8 && (nbytes % 8) == 0) {
-            for (int o = 0; o < nbytes; o += 8) cp_async_8(dst + o, src + o);
-          } else {
-            for (int o = 0; o < nbytes; o += 4) cp_async_4(dst + o, src + o);
-          }
-          const uint32_t wdst = slot + kRowsW * S::kRP + r * 16;
-          const int g0 = (kt * kBK) >> a.gs_log2;
-          if constexpr (FP4) {
-            copy_window(wdst, s_begin + row * G + g0, s_begin, s_end);
-          } else {
-            copy_window(wdst, s_begin + 2 * (row * G + g0), s_begin, s_end);
-            copy_window(wdst + 8, b_begin + 2 * (row * G + g0), b_begin, b_end);
-          }
-        }
-        cp_async_commit();
-        if (i - kLag >= 0) {
-          cp_async_wait_group<kLag>();
-          mbar_arrive(full_l((i - kLag) % PST));
-          published = i - kLag + 1;
-        }
-      }
-      cp_async_wait_all();
-      if (!*abort_flag) {
-        for (int i = published; i < nkt; ++i) mbar_arrive(full_l(i % PST));
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(std::is_same<T, __nv_bfloat16>::value, kRowsW, BT);
-      for (int i = 0; i < nkt; ++i) {
-        const int s = i % ST;
-        const uint32_t par = (i / ST) & 1;
-        if (!(mbar_wait(full_a(s), par, abort_flag) && mbar_wait(full_b(s), par, abort_flag)))
-          break;
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(ring + s * S::kStageBytes);
-        const uint32_t b_addr = a_addr + S::kABytes;
-#pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          mma_f16(tmem, sdesc_sw128(a_addr + k * 32), sdesc_sw128(b_addr + k * 32), idesc,
-                  (i > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(empty(s));
-      }
-      // Signals the epilogue once every issued MMA has completed (also on
-      // abort, so nothing is in flight when TMEM is freed).
-      mma_commit(acc_full);
-    }
-  } else {
-    // ------------------------------------------- dequantizers (warps 2..5)
-    const int grp = (warp - kProducerWarp0) >> 2;          // dequantizer group
-    const int r = ((warp - kProducerWarp0) & 3) * 32 + lane; // weight row in the tile
-    const int64_t row = n0 + r;
-    const bool row_ok = row < a.N;
-    const bool fp4_g16 = FP4 && a.gs_log2 == 4;
-    int w_ready = 0, w_freed = 0;                          // TMA path: chunks waited / released
-    int s_ready = 0, s_freed = 0;
-    for (int i = grp; i < nkt; i += kDqGroups) {
-      const int kt = kt0 + i;
-      const bool tail = (kt + 1) * kBK > a.K;
-      Packed<BITS> pk;
-      StageSB sb;
-      if constexpr (FAST) {
-        const int o0 = i * S::kPB;                         // row byte offset from wb0
-        const int c_hi = (o0 + S::kPB - 1) >> 7;
-        bool ok = true;
-        for (; w_ready <= c_hi && ok; ++w_ready)
-          ok = mbar_wait(full_l(w_ready % WS), (w_ready / WS) & 1, abort_flag);
-        const int sj = (((kt * kBK) >> a.gs_log2) / SGC) - sc0;
-        for (; s_ready <= sj && ok; ++s_ready)
-          ok = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
-        if (!ok) break;
-        if constexpr (S::kPB % 16 == 0) {
-#pragma unroll
-          for (int u = 0; u < S::kPB / 16; ++u) {
-            const int o = o0 + 16 * u;
-            const uint4 v = *reinterpret_cast<const uint4*>(
-                wring + ((o >> 7) % WS) * S::kWChunk + wchunk_off(o & 127, r));
-            pk.w[4 * u] = v.x; pk.w[4 * u + 1] = v.y; pk.w[4 * u + 2] = v.z; pk.w[4 * u + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int u = 0; u < S::kPB / 8; ++u) {
-            const int o = o0 + 8 * u;
-            const uint2 v = *reinterpret_cast<const uint2*>(
-                wring + ((o >> 7) % WS) * S::kWChunk + wchunk_off(o & 127, r));
-            pk.w[2 * u] = v.x; pk.w[2 * u + 1] = v.y;
-          }
-        }
-        if (tail) {
-#pragma unroll
-          for (int w = BITS; w < 2 * BITS; ++w) pk.w[w] = 0u;
-        }
-        const uint8_t* sslot = sring + ((s_ready - 1) % SS) * S::kSChunk;
-        const int g0 = (kt * kBK) >> a.gs_log2;
-        const int g1 = tail ? g0 : ((kt * kBK + 32) >> a.gs_log2);
-        if constexpr (FP4) {
-          const uint8_t* sp = sslot + r * 16;
-          const int gs = 1 << a.gs_log2;
-          auto sc = [&](int g) { return splat(TT<T>::from_f(fp4_scale_t<T>(sp[g % SGC], gs))); };
-          if (fp4_g16) {
-            sb.s[0] = sc(g0); sb.s[1] = sc(g0 + 1);
-            sb.b[0] = tail ? sb.s[0] : sc(g0 + 2);
-            sb.b[1] = tail ? sb.s[0] : sc(g0 + 3);
-          } else {
-            sb.s[0] = sc(g0); sb.s[1] = sc(g1); sb.b[0] = sb.b[1] = 0u;
-          }
-        } else {
-          const uint16_t* sp = reinterpret_cast<const uint16_t*>(sslot + r * 16);
-          const uint16_t* bp = reinterpret_cast<const uint16_t*>(sslot + kRowsW * 16 + r * 16);
-          const uint32_t s0 = sp[g0 % SGC], s1 = sp[g1 % SGC];
-          const uint32_t b0 = bp[g0 % SGC], b1 = bp[g1 % SGC];
-          sb.s[0] = s0 | (s0 << 16); sb.s[1] = s1 | (s1 << 16);
-          sb.b[0] = b0 | (b0 << 16); sb.b[1] = b1 | (b1 << 16);
-        }
-        // release the chunks this group is done with: those that end before
-        // its next stage starts (all of them after its last stage)
-        const bool last = i + kDqGroups >= nkt;
-        const int w_done = last ? nwc : (((i + kDqGroups) * S::kPB) >> 7);
-        const int s_done =
-            last ? nsc : ((((kt + kDqGroups) * kBK) >> a.gs_log2) / SGC) - sc0;
-        if (w_done > w_freed || s_done > s_freed) {
-          __syncwarp();
-          if (lane == 0) {
-            for (int c = w_freed; c < w_done; ++c) mbar_arrive(empty_l(c % WS));
-            for (int j = s_freed; j < s_done; ++j) mbar_arrive(empty_l(WS + j % SS));
-          }
-          w_freed = w_done > w_freed ? w_done : w_freed;
-          s_freed = s_done > s_freed ? s_done : s_freed;
-        }
-      } else {
-        const int ps = i % PST;
-        if (!mbar_wait(full_l(ps), (i / PST) & 1, abort_flag)) break;
-        const uint8_t* slot = pring + ps * S::kPSlot;
-        if (row_ok) {
-          lds_packed<BITS>(pk, slot + r * S::kRP);
-          if (tail) {
-#pragma unroll
-            for (int w = BITS; w < 2 * BITS; ++w) pk.w[w] = 0u;
-          }
-          const uint4 wv = *reinterpret_cast<const uint4*>(slot + kRowsW * S::kRP + r * 16);
-          sb = sb_from_words<T, FP4>(wv, a, row, kt, G, tail);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty_l(ps));
-      }
-      const int s = i % ST;
-      if (!mbar_wait(empty(s), ((i / ST) & 1) ^ 1, abort_flag)) break;
-      uint8_t* a_row = ring + s * S::kStageBytes + r * 128;
-      if (row_ok) {
-        dequant_stage<T, BITS, FP4>(pk, sb, fp4_g16, a_row, r, tail);
-      } else {
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a_row + (c << 4)) = z;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(full_a(s));
-    }
-    if constexpr (FAST) {
-      // Chunks past this group's last stage are released too (both groups
-      // release every chunk), but only after their data has landed: the
-      // landing proves the slot's previous chunk was released by both
-      // groups, so this arrival counts toward the right phase.
-      bool ok = !*abort_flag;
-      for (; w_ready < nwc && ok; ++w_ready)
-        ok = mbar_wait(full_l(w_ready % WS), (w_ready / WS) & 1, abort_flag);
-      for (; s_ready < nsc && ok; ++s_ready)
-        ok = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
-      if (ok && (w_freed < nwc || s_freed < nsc)) {
-        __syncwarp();
-        if (lane == 0) {
-          for (int c = w_freed; c < nwc; ++c) mbar_arrive(empty_l(c % WS));
-          for (int j = s_freed; j < nsc; ++j) mbar_arrive(empty_l(WS + j % SS));
-        }
-      }
-    }
-
-    // ------------------------------------------------------- epilogue
-    const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, 4000000000ull);
-    tc_fence_after();
-    const int q = warp & 3;                                 // TMEM lane quarter
-    const int rr = q * 32 + lane;                           // tile row of this thread
-    const int64_t orow = n0 + rr;
-    float* red = reinterpret_cast<float*>(ring);            // [BT][128] when split
-    if (acc_ok && !*abort_flag) {
-#pragma unroll 1
-      for (int c0 = 16 * grp; c0 < BT; c0 += 16 * kDqGroups) {
-        uint32_t v[16];
-        tmem_ld_16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
-        tmem_ld_wait();
-        if (a.splits == 1) {
-          if (orow < a.N) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int m = m0 + c0 + j;
-              if (m < a.M)
-                reinterpret_cast<T*>(a.y)[(int64_t)m * a.N + orow] = TT<T>::from_f(__uint_as_float(v[j]));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) red[(c0 + j) * kRowsW + rr] = __uint_as_float(v[j]);
-        }
-      }
-    }
-  }
-
-  // --------------------------------------------------------- split-K reduce
-  if (a.splits > 1) {
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    if (!*abort_flag) {
-      const float* red = reinterpret_cast<const float*>(ring);
-      for (int i = threadIdx.x; i < BT * kRowsW; i += kThreads) {
-        if (i % a.splits != split) continue;
-        const int j = i / kRowsW, rr = i - j * kRowsW;
-        const int m = m0 + j;
-        const int64_t orow = n0 + rr;
-        if (m >= a.M || orow >= a.N) continue;
-        float sum = 0.0f;
-        for (int q = 0; q < a.splits; ++q) sum += cluster.map_shared_rank(red, q)[i];
-        reinterpret_cast<T*>(a.y)[(int64_t)m * a.N + orow] = TT<T>::from_f(sum);
-      }
-    }
-    cluster.sync();
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) atomicOr(&g_aq_device_error, 1u);
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, S::kTmemCols);
-  }
-}
-
-// -------------------------------------------------------------------- host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 2-D tensor map over a row-major [rows, cols] array of 1- or 2-byte
-// elements; zero fill out of bounds.
-cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int esize,
-                     int64_t rows, int64_t cols, int box_cols, int box_rows,
-                     CUtensorMapSwizzle swz) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return cudaErrorNotSupported;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(cols * esize)};
-  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-template <typename T, int BITS, bool FP4, int BT, bool FAST>
-cudaError_t launch_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, cudaStream_t st) {
-  using S = QmmShape<BT, BITS, FAST>;
-  auto kern = qmm_tc_kernel<T, BITS, FP4, BT, FAST>;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 64 || !attr_done[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
-    if (e != cudaSuccess) return e;
-    if (dev < 64) attr_done[dev] = true;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.n_tiles, (unsigned)p.m_tiles, (unsigned)p.splits);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = S::kSmem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = (unsigned)p.splits;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, maps, a);
-}
-
-template <typename T, int BITS, bool FP4, bool FAST>
-cudaError_t by_bt(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, cudaStream_t st) {
-  switch (p.bt) {
-    case 16: return launch_tc<T, BITS, FP4, 16, FAST>(p, maps, a, st);
-    case 32: return launch_tc<T, BITS, FP4, 32, FAST>(p, maps, a, st);
-    case 64: return launch_tc<T, BITS, FP4, 64, FAST>(p, maps, a, st);
-    case 128: return launch_tc<T, BITS, FP4, 128, FAST>(p, maps, a, st);
-    default: return launch_tc<T, BITS, FP4, 256, FAST>(p, maps, a, st);
-  }
-}
-
-template <typename T, bool FAST>
-cudaError_t by_bits_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, int bits,
-                       int mode, cudaStream_t st) {
-  if (mode == AQ_MODE_FP4) return by_bt<T, 4, true, FAST>(p, maps, a, st);
-  switch (bits) {
-    case 2: return by_bt<T, 2, false, FAST>(p, maps, a, st);
-    case 3: return by_bt<T, 3, false, FAST>(p, maps, a, st);
-    case 4: return by_bt<T, 4, false, FAST>(p, maps, a, st);
-    case 5: return by_bt<T, 5, false, FAST>(p, maps, a, st);
-    case 6: return by_bt<T, 6, false, FAST>(p, maps, a, st);
-    case 8: return by_bt<T, 8, false, FAST>(p, maps, a, st);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-int ilog2i(int v) {
-  int r = 0;
-  while ((1 << (r + 1)) <= v) ++r;
-  return r;
-}
-
-}  // namespace
 
 QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
   (void)gs; (void)mode;
@@ -892,10 +46,12 @@ cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const v
   cudaError_t e = make_map(&maps.x, x, tt, 2, M, K, kBK, p.bt, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   QmmArgs a;
+  memset(&a, 0, sizeof(a));
   a.wq = (const uint8_t*)w_q;
   a.scales = scales;
   a.biases = biases;
   a.y = y;
+  a.x = x;
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
@@ -903,37 +59,19 @@ cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const v
   a.k_tiles = p.k_tiles;
   a.k_tiles_split = p.k_tiles_split;
   a.splits = p.splits;
-  a.row_bytes = K * bits / 8;
-  // widest copy that every row start and stage offset (8*bits bytes) allows
-  a.vec = (a.row_bytes % 16 == 0 && (8 * bits) % 16 == 0) ? 16
-          : (a.row_bytes % 8 == 0 && (8 * bits) % 8 == 0) ? 8 : 4;
-  // TMA path: packed rows, scale rows and bias rows 16-byte strided and based.
-  const int64_t G = K / gs;
-  const int esz = mode == AQ_MODE_FP4 ? 1 : 2;
-  const bool fast = a.row_bytes % 16 == 0 && (G * esz) % 16 == 0 &&
-                    ((uintptr_t)scales & 15) == 0 &&
-                    (mode == AQ_MODE_FP4 || ((uintptr_t)biases & 15) == 0);
-  if (fast) {
-    e = make_map(&maps.w, w_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, a.row_bytes, 128, kRowsW,
-                 CU_TENSOR_MAP_SWIZZLE_128B);
-    if (e != cudaSuccess) return e;
-    const CUtensorMapDataType st_t =
-        mode == AQ_MODE_FP4 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
-    e = make_map(&maps.s, scales, st_t, esz, N, G, 16 / esz, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (e != cudaSuccess) return e;
-    if (mode != AQ_MODE_FP4) {
-      e = make_map(&maps.b, biases, st_t, esz, N, G, 16 / esz, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE);
-      if (e != cudaSuccess) return e;
-    }
-    return dtype == AQ_F16 ? by_bits_tc<__half, true>(p, maps, a, bits, mode, st)
-                           : by_bits_tc<__nv_bfloat16, true>(p, maps, a, bits, mode, st);
-  }
-  return dtype == AQ_F16 ? by_bits_tc<__half, false>(p, maps, a, bits, mode, st)
-                         : by_bits_tc<__nv_bfloat16, false>(p, maps, a, bits, mode, st);
+  a.ldy = (int)N;
+  a.n_limit = (int)N;
+  a.ntg = (int)p.n_tiles;
+  bool fast = false;
+  e = weight_maps(maps, a, w_q, scales, biases, N, K, bits, gs, mode, &fast);
+  if (e != cudaSuccess) return e;
+  if (fast)
+    return dtype == AQ_F16 ? by_bits_tc<__half, true, 0>(p, maps, a, bits, mode, st)
+                           : by_bits_tc<__nv_bfloat16, true, 0>(p, maps, a, bits, mode, st);
+  return dtype == AQ_F16 ? by_bits_tc<__half, false, 0>(p, maps, a, bits, mode, st)
+                         : by_bits_tc<__nv_bfloat16, false, 0>(p, maps, a, bits, mode, st);
 }
 
-cudaError_t read_device_error(unsigned* out) {
-  return cudaMemcpyFromSymbol(out, g_aq_device_error, sizeof(unsigned));
-}
+cudaError_t read_device_error_qmm(unsigned* out) { return read_tu_error(out); }
 
 }  // namespace aq
