@@ -40,10 +40,10 @@ def lib():
         _lib.orc_quantize.argtypes = [P, I64, I64, I, I, I, P, P, P]
         _lib.orc_unpack.argtypes = [P, I64, I64, I, P]
         _lib.orc_dequantize.argtypes = [P, P, P, I64, I64, I, I, I, I, P, P]
-        _lib.orc_qmm.argtypes = [P, P, P, P, I64, I64, I64, I, I, I, I, P, P]
-        _lib.orc_qmm_sampled.argtypes = [P, P, P, P, I64, I64, I64, I, I, I, I,
+        _lib.orc_qmm.argtypes = [P, P, P, P, I64, I64, I64, I, I, I, I, I, P, P]
+        _lib.orc_qmm_sampled.argtypes = [P, P, P, P, I64, I64, I64, I, I, I, I, I,
                                          P, P, I64, P, P]
-        _lib.orc_qconv2d_nhwc.argtypes = [P, P, P, P] + [I] * 15 + [P, P, I64, P, P]
+        _lib.orc_qconv2d_nhwc.argtypes = [P, P, P, P] + [I] * 16 + [P, P, I64, P, P]
         for name in ("orc_quantize", "orc_unpack", "orc_dequantize", "orc_qmm",
                      "orc_qmm_sampled", "orc_qconv2d_nhwc"):
             getattr(_lib, name).restype = I
@@ -122,8 +122,9 @@ def dequantize(wq, scales, biases, N, K, bits, gs, mode, dt):
     return wh, wt
 
 
-def qmm(x16, wq, scales, biases, N, bits, gs, mode, dt):
-    """y = x . w_hat^T in fp64 -> (y [M, N], den [M, N] = sum |x w_hat|)."""
+def qmm(x16, wq, scales, biases, N, bits, gs, mode, dt, w_in_t=False):
+    """y = x . w_hat^T in fp64 -> (y [M, N], den [M, N] = sum |x w_hat|).
+    w_in_t: multiply by w_hat rounded once to T (the dequantize output)."""
     x16 = _c(x16, np.uint16)
     M, K = x16.shape
     wq = _c(wq, np.uint8)
@@ -132,11 +133,11 @@ def qmm(x16, wq, scales, biases, N, bits, gs, mode, dt):
     y = np.zeros((M, N), np.float64)
     den = np.zeros((M, N), np.float64)
     _check(lib().orc_qmm(_p(x16), _p(wq), _p(scales), _p(biases), M, N, K, bits, gs, mode, dt,
-                         _p(y), _p(den)), "qmm")
+                         int(w_in_t), _p(y), _p(den)), "qmm")
     return y, den
 
 
-def qmm_sampled(x16, wq, scales, biases, N, bits, gs, mode, dt, ms, ns):
+def qmm_sampled(x16, wq, scales, biases, N, bits, gs, mode, dt, ms, ns, w_in_t=False):
     x16 = _c(x16, np.uint16)
     M, K = x16.shape
     wq = _c(wq, np.uint8)
@@ -147,7 +148,7 @@ def qmm_sampled(x16, wq, scales, biases, N, bits, gs, mode, dt, ms, ns):
     y = np.zeros(len(ms), np.float64)
     den = np.zeros(len(ms), np.float64)
     _check(lib().orc_qmm_sampled(_p(x16), _p(wq), _p(scales), _p(biases), M, N, K, bits, gs,
-                                 mode, dt, _p(ms), _p(ns), len(ms), _p(y), _p(den)),
+                                 mode, dt, int(w_in_t), _p(ms), _p(ns), len(ms), _p(y), _p(den)),
            "qmm_sampled")
     return y, den
 
@@ -157,7 +158,7 @@ def conv_out_hw(H, W, kh, kw, sh, sw, ph, pw):
 
 
 def qconv2d_nhwc(x16, wq, scales, biases, Cout, kh, kw, stride, pad, groups, bits, gs, dt,
-                 ms=None, cos=None):
+                 ms=None, cos=None, w_in_t=False):
     """x16 [B, H, W, Cin] -> (y, den) as [B, Ho, Wo, Cout] fp64, or at sampled (m, co)."""
     x16 = _c(x16, np.uint16)
     B, H, W, Cin = x16.shape
@@ -178,6 +179,6 @@ def qconv2d_nhwc(x16, wq, scales, biases, Cout, kh, kw, stride, pad, groups, bit
         den = np.zeros((B, Ho, Wo, Cout), np.float64)
         cnt = 0
     _check(lib().orc_qconv2d_nhwc(_p(x16), _p(wq), _p(scales), _p(biases), B, H, W, Cin, Cout,
-                                  kh, kw, sh, sw, ph, pw, groups, bits, gs, dt,
+                                  kh, kw, sh, sw, ph, pw, groups, bits, gs, dt, int(w_in_t),
                                   _p(ms), _p(cos), cnt, _p(y), _p(den)), "qconv2d_nhwc")
     return y, den

@@ -206,6 +206,14 @@ void dequant_row(const uint8_t* wq, const void* scales, const uint16_t* biases,
   }
 }
 
+// w_hat rounded once to T: the dequantize operation's output ("Add the 3bit
+// packed qmm_t", dequantize returns an array of the scales' type; the
+// pages' Metal loader and CPU _qmm_t form scale * w + bias in T before the
+// multiply).  Used for the products of kernels that dequantize into T tiles.
+void round_row_to_t(double* row, int64_t K, int dt) {
+  for (int64_t k = 0; k < K; ++k) row[k] = t_to_double(round_to_t(row[k], dt), dt);
+}
+
 int check_common(int64_t N, int64_t K, int bits, int gs, int mode, int dt) {
   if (dt != DT_F16 && dt != DT_BF16) return 1;
   if (N < 0 || K < 0) return 1;
@@ -329,12 +337,13 @@ int orc_dequantize(const uint8_t* w_q, const void* scales, const uint16_t* biase
 }
 
 // y = x . w_hat^T in fp64 ([P2] quantized_matmul with transpose=true), and
-// den = sum_k |x[m,k] * w_hat[n,k]| for the error bound.  x is [M, K] T;
+// den = sum_k |x[m,k] * w_hat[n,k]| for the error bound.  With w_in_t the
+// product uses w_hat rounded once to T (see round_row_to_t).  x is [M, K] T;
 // y, den are [M, N] doubles.  The outer loop over n may run on several
 // threads; each output is one sequential fp64 sum over k.
 int orc_qmm(const uint16_t* x, const uint8_t* w_q, const void* scales,
             const uint16_t* biases, int64_t M, int64_t N, int64_t K, int bits,
-            int gs, int mode, int dt, double* y, double* den) {
+            int gs, int mode, int dt, int w_in_t, double* y, double* den) {
   if (check_common(N, K, bits, gs, mode, dt) || M < 0) return 1;
   std::vector<double> xd((size_t)(M * K));
   for (int64_t i = 0; i < M * K; ++i) xd[(size_t)i] = t_to_double(x[i], dt);
@@ -344,6 +353,7 @@ int orc_qmm(const uint16_t* x, const uint8_t* w_q, const void* scales,
 #pragma omp for schedule(dynamic, 4)
     for (int64_t n = 0; n < N; ++n) {
       dequant_row(w_q, scales, biases, n, K, bits, gs, mode, dt, row.data());
+      if (w_in_t) round_row_to_t(row.data(), K, dt);
       for (int64_t m = 0; m < M; ++m) {
         const double* xr = xd.data() + m * K;
         double acc = 0.0, mag = 0.0;
@@ -363,13 +373,14 @@ int orc_qmm(const uint16_t* x, const uint8_t* w_q, const void* scales,
 // The same products at `count` sampled (m, n) positions only.
 int orc_qmm_sampled(const uint16_t* x, const uint8_t* w_q, const void* scales,
                     const uint16_t* biases, int64_t M, int64_t N, int64_t K, int bits,
-                    int gs, int mode, int dt, const int64_t* ms, const int64_t* ns,
-                    int64_t count, double* y, double* den) {
+                    int gs, int mode, int dt, int w_in_t, const int64_t* ms,
+                    const int64_t* ns, int64_t count, double* y, double* den) {
   if (check_common(N, K, bits, gs, mode, dt) || M < 0) return 1;
   std::vector<double> row((size_t)K);
   for (int64_t i = 0; i < count; ++i) {
     if (ms[i] < 0 || ms[i] >= M || ns[i] < 0 || ns[i] >= N) return 1;
     dequant_row(w_q, scales, biases, ns[i], K, bits, gs, mode, dt, row.data());
+    if (w_in_t) round_row_to_t(row.data(), K, dt);
     double acc = 0.0, mag = 0.0;
     for (int64_t k = 0; k < K; ++k) {
       double p = t_to_double(x[ms[i] * K + k], dt) * row[(size_t)k];
@@ -398,8 +409,8 @@ int orc_qmm_sampled(const uint16_t* x, const uint8_t* w_q, const void* scales,
 int orc_qconv2d_nhwc(const uint16_t* x, const uint8_t* w_q, const uint16_t* scales,
                      const uint16_t* biases, int B, int H, int W, int Cin, int Cout,
                      int kh, int kw, int sh, int sw, int ph, int pw, int groups,
-                     int bits, int gs, int dt, const int64_t* ms, const int64_t* cos,
-                     int64_t count, double* y, double* den) {
+                     int bits, int gs, int dt, int w_in_t, const int64_t* ms,
+                     const int64_t* cos, int64_t count, double* y, double* den) {
   if (groups <= 0 || Cin % groups || Cout % groups || kh <= 0 || kw <= 0 ||
       sh <= 0 || sw <= 0 || ph < 0 || pw < 0 || B < 0 || H < 0 || W < 0)
     return 1;
@@ -432,6 +443,7 @@ int orc_qconv2d_nhwc(const uint16_t* x, const uint8_t* w_q, const uint16_t* scal
       const int g = (int)(cos[i] / Ng);
       im2col_row(ms[i], g, a.data());
       dequant_row(w_q, scales, biases, cos[i], Kp, bits, gs, MODE_AFFINE, dt, wrow.data());
+      if (w_in_t) round_row_to_t(wrow.data(), Kp, dt);
       double acc = 0.0, mag = 0.0;
       for (int64_t k = 0; k < Kp; ++k) {
         double p = a[(size_t)k] * wrow[(size_t)k];
@@ -453,6 +465,7 @@ int orc_qconv2d_nhwc(const uint16_t* x, const uint8_t* w_q, const uint16_t* scal
     for (int n = 0; n < Ng; ++n) {
       const int co = g * Ng + n;
       dequant_row(w_q, scales, biases, co, Kp, bits, gs, MODE_AFFINE, dt, wrow.data());
+      if (w_in_t) round_row_to_t(wrow.data(), Kp, dt);
       for (int64_t m = 0; m < Mtot; ++m) {
         const double* a = A.data() + m * Kp;
         double acc = 0.0, mag = 0.0;

@@ -1,6 +1,7 @@
 """GPU parity for aq_qconv2d_nhwc (implicit GEMM on the tcgen05 kernel)
 against the oracle's explicit-im2col convolution, within
-|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref)."""
+|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref), with w_hat rounded
+once to T in the reference (the kernel multiplies T-valued weight tiles)."""
 import numpy as np
 import pytest
 import torch
@@ -26,7 +27,7 @@ def _conv_case(B, H, W, Cin, Cout, k, stride, pad, groups, bits, gs, dt, seed):
 
 def _check_full(xd, wq, s, b, y, Cout, k, stride, pad, groups, bits, gs, dt):
     yr, den = oracle.qconv2d_nhwc(dev_u16(xd), dev_u8(wq), dev_u16(s), dev_u16(b), Cout, k, k,
-                                  (stride, stride), (pad, pad), groups, bits, gs, dt)
+                                  (stride, stride), (pad, pad), groups, bits, gs, dt, w_in_t=True)
     return check_matmul(dev_u16(y).reshape(yr.shape), yr, den, dt)
 
 
@@ -58,7 +59,8 @@ def test_conv_full_size(groups, bits):
     ms = np.concatenate([[0, M - 1, 63, 64, 4095, 4096], rng.integers(0, M, 600)])
     cos = np.concatenate([[0, 319, 79, 80, 160, 240], rng.integers(0, 320, 600)])
     yr, den = oracle.qconv2d_nhwc(dev_u16(xd), dev_u8(wq), dev_u16(s), dev_u16(b), 320, 3, 3,
-                                  (1, 1), (1, 1), groups, bits, gs, dt, ms=ms, cos=cos)
+                                  (1, 1), (1, 1), groups, bits, gs, dt, ms=ms, cos=cos,
+                                  w_in_t=True)
     ys = dev_u16(y).reshape(M, 320)[ms, cos]
     check_matmul(ys, yr, den, dt)
 

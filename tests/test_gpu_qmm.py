@@ -1,5 +1,9 @@
 """GPU parity for aq_qmm (tcgen05 tensor-core path) against the oracle, within
-|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref)."""
+|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref).
+
+The kernel dequantizes each weight tile into T (the values aq_dequantize
+writes, as the pages' kernels do) before the tensor-core product, so y_ref is
+the oracle's fp64 product with w_hat rounded once to T (w_in_t)."""
 import numpy as np
 import pytest
 import torch
@@ -22,11 +26,11 @@ def _case(M, N, K, bits, gs, dt, seed, wstd=0.05, xstd=1.0):
     return to_dev(x), wq, s, b
 
 
-def _check(x, wq, s, b, y, bits, gs, dt, mode=0, **kw):
+def _check(x, wq, s, b, y, bits, gs, dt, mode=0, w_in_t=True, **kw):
     N = wq.shape[0]
     sc = dev_u8(s) if mode == 1 else dev_u16(s)
     bi = None if b is None else dev_u16(b)
-    yr, den = oracle.qmm(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt)
+    yr, den = oracle.qmm(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt, w_in_t=w_in_t)
     return check_matmul(dev_u16(y), yr, den, dt, **kw)
 
 
@@ -37,7 +41,8 @@ def _check_sampled(x, wq, s, b, y, bits, gs, dt, n_samples=512, seed=0, mode=0, 
     ns = np.concatenate([[0, N - 1, 0, N - 1], rng.integers(0, N, n_samples)])
     sc = dev_u8(s) if mode == 1 else dev_u16(s)
     bi = None if b is None else dev_u16(b)
-    yr, den = oracle.qmm_sampled(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt, ms, ns)
+    yr, den = oracle.qmm_sampled(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt, ms, ns,
+                                 w_in_t=True)
     ys = dev_u16(y)[ms, ns]
     return check_matmul(ys, yr, den, dt, **kw)
 
@@ -163,7 +168,7 @@ def test_qmm_matches_qmv_small_m():
     y2 = api.aq_qmv(x, wq, s, b, 4, 64)
     torch.cuda.synchronize()
     _check(x, wq, s, b, y1, 4, 64, 1)
-    _check(x, wq, s, b, y2, 4, 64, 1)
+    _check(x, wq, s, b, y2, 4, 64, 1, w_in_t=False)    # qmv keeps w_hat in fp32
 
 
 def test_qmm_empty():

@@ -354,6 +354,28 @@ def test_qmm_matches_unfused_numpy(bits, dt):
     assert np.array_equal(ys, y[[0, 4, 2], [0, 23, 11]])
 
 
+@pytest.mark.parametrize("dt", [F16, BF16])
+def test_qmm_w_in_t_uses_dequantize_output(dt):
+    """The T-tile reference equals numpy's product with aq_dequantize's values
+    (w_hat rounded once to T), and differs from the exact one by at most the
+    T rounding of w_hat."""
+    rng = np.random.default_rng(11 + dt)
+    M, N, K, gs, bits = 3, 20, 192, 64, 3
+    w = f64_to_u16(rng.standard_normal((N, K)) * 0.1, dt)
+    x = f64_to_u16(rng.standard_normal((M, K)), dt)
+    wq, s, b = oracle.quantize(w, bits, gs, dt)
+    yt, dent = oracle.qmm(x, wq, s, b, N, bits, gs, AFFINE, dt, w_in_t=True)
+    _, wt = oracle.dequantize(wq, s, b, N, K, bits, gs, AFFINE, dt)
+    X = u16_to_f64(x, dt)
+    WT = u16_to_f64(wt, dt)
+    assert np.allclose(yt, X @ WT.T, rtol=1e-12, atol=1e-12)
+    ye, den = oracle.qmm(x, wq, s, b, N, bits, gs, AFFINE, dt)
+    u = 2.0 ** (-11 if dt == F16 else -8)
+    assert np.all(np.abs(yt - ye) <= u * den * (1 + 1e-9))
+    ys, _ = oracle.qmm_sampled(x, wq, s, b, N, bits, gs, AFFINE, dt, [1, 2], [3, 19], w_in_t=True)
+    assert np.array_equal(ys, yt[[1, 2], [3, 19]])
+
+
 def test_qmm_8bit_unit_scale_is_integer_gemm():
     """bits=8, scale 1, bias 0 reduces to an integer GEMM."""
     rng = np.random.default_rng(3)
