@@ -1,15 +1,21 @@
 """Benchmark of the quantized matmul hot path on B200.
 
-Workload (one step): the decode sweep of a 16-layer Llama-3.2-1B-shaped stack
-of distinct bf16 weights quantized 4-bit, group 64 (q/o 2048x2048, k/v
-512x2048, gate/up 8192x2048, down 2048x8192; 547 MB of packed weights,
-scales and biases, more than 4x the 126 MB L2, so no L2 flush is needed and
-every step streams the weights from HBM).  For each M in (1, 2, 4, 8, 16) the
-step runs y = x . dequant(W)^T for every projection of every layer through
-aq_qmv.  The step is captured once in a CUDA graph and replayed.
+Headline workload (one step): the decode sweep of a 16-layer
+Llama-3.2-1B-shaped stack of distinct bf16 weights quantized 4-bit, group 64
+(q/o 2048x2048, k/v 512x2048, gate/up 8192x2048, down 2048x8192; 547 MB of
+packed weights, scales and biases, more than 4x the 126 MB L2, so no L2
+flush is needed and every step streams the weights from HBM).  For each M in
+(1, 2, 4, 8, 16) the step runs y = x . dequant(W)^T for every projection of
+every layer through aq_qmv.  The step is captured once in a CUDA graph and
+replayed.
 
 Metric: qmv weight-stream GB/s = (packed weights + scales + biases + x + y
 bytes of all calls) / device time of the step, whole job (all ranks).
+Beside it (not part of the step): the sweep's M = 32, 64 rows through
+aq_qmm, and the tensor-core side of the metric in TFLOP/s (2 M N K / time):
+the chained fp16 qmm (x[1024,1024] through W1 [4096,1024] and W2
+[1024,4096], ten times), FP4 weights at M = 4096, and the conv2d implicit
+GEMM.
 
 --impl reference times the CPU oracle on a bounded sample of the same
 workload (one layer at M = 1 per step) on the host cores.
@@ -32,6 +38,7 @@ sys.path.insert(0, ROOT)
 
 LAYERS = 16
 QMV_M = (1, 2, 4, 8, 16)
+QMM_M = (32, 64)
 BITS, GS = 4, 64
 METRIC = "qmv weight-stream GB/s (M<=16), % of B200 HBM roofline"
 WORKLOAD = ("decode sweep: 16-layer Llama-3.2-1B-shaped stack (q/o 2048x2048, k/v 512x2048, "
@@ -45,6 +52,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-qmm", action="store_true", help="skip the TFLOP/s side lines")
     return ap.parse_args()
 
 
@@ -52,19 +60,20 @@ def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return p["hbm_gbs"], p["bf16_tflops"], "measured"
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
     except Exception:
-        return 6650.0, 1590.0, "fallback"
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def proj_bytes(n, k, M):
+    """Algorithmic bytes of one projection call: packed weights, scales,
+    biases (bf16), x and y (bf16)."""
+    return n * k * BITS // 8 + 2 * 2 * n * (k // GS) + 2 * M * k + 2 * M * n
 
 
 def layer_bytes(M):
-    """Algorithmic bytes of one layer at M rows: packed weights, scales,
-    biases, x and y (bf16)."""
     from group_wise_affine_quant_b200.inputs import LLAMA_1B_PROJ
-    tot = 0
-    for _, n, k in LLAMA_1B_PROJ:
-        tot += n * k * BITS // 8 + 2 * 2 * n * (k // GS) + 2 * M * k + 2 * M * n
-    return tot
+    return sum(proj_bytes(n, k, M) for _, n, k in LLAMA_1B_PROJ)
 
 
 class ClockSampler:
@@ -90,7 +99,7 @@ class ClockSampler:
                     self.samples.append([v.strip() for v in out.split(",")])
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            self._stop.wait(0.1)
 
     def __enter__(self):
         self._t = threading.Thread(target=self._run, daemon=True)
@@ -104,8 +113,9 @@ class ClockSampler:
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        num = lambda v: v.replace(".", "", 1).isdigit()
+        sm = [float(s[0]) for s in self.samples if num(s[0])]
+        mx = [float(s[1]) for s in self.samples if num(s[1])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for s in self.samples for i in range(4)
                           if len(s) > 4 + i and s[4 + i].lower() == "active"})
@@ -151,19 +161,40 @@ def traffic_for(kernel, workload):
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)[kernel]
-        src = os.path.join(ROOT, rec["source"])
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if h != rec["source_sha256_16"] or rec["workload"] != workload:
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            h.update(open(os.path.join(ROOT, src), "rb").read())
+        if h.hexdigest()[:16] != rec["sources_sha256_16"] or rec["workload"] != workload:
             return None
         return rec["dram_bytes_per_launch"]
     except Exception:
         return None
 
 
-def cpu_baseline(seconds_hint=10.0):
+def graph_time_ms(torch, stream, fn, reps, warm=3):
+    """Device time per call of fn, captured `reps` times in one CUDA graph."""
+    with torch.cuda.stream(stream):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                fn()
+        for _ in range(warm):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / reps
+
+
+def cpu_baseline():
     """The oracle as it stands, on the host cores, over a bounded sample: one
     layer of the stack at M = 1, 2, 4, 8, 16 (the same inputs recipe)."""
-    import numpy as np
     import oracle
     from group_wise_affine_quant_b200 import inputs
     ws = inputs.decode_layer(seed=0)
@@ -177,13 +208,13 @@ def cpu_baseline(seconds_hint=10.0):
             oracle.qmm(x, wq, s, b, n, BITS, GS, 0, 1)
             tot_t += time.perf_counter() - t0
         tot_bytes += layer_bytes(M)
-    return {"value": tot_bytes / tot_t / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+    return {"value": round(tot_bytes / tot_t / 1e9, 3), "unit": "GB/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
             "sample": "one layer of the stack (7 projections) at M = 1,2,4,8,16, %.1f s" % tot_t}
 
 
 def run_reference(args):
-    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
@@ -215,6 +246,57 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+def qmm_lines(torch, api, inputs, dev, stream, tf_peak, tf_sust):
+    """TFLOP/s of the tensor-core workloads (not part of the timed step)."""
+    out = {}
+    # chained fp16 qmm, 4-bit g64: 20 products per chain
+    x, w1, w2 = inputs.chained()
+    q1 = api.aq_quantize(w1.to(dev), 4, 64)
+    q2 = api.aq_quantize(w2.to(dev), 4, 64)
+    xd = x.to(dev)
+    h = torch.empty((1024, 4096), dtype=torch.float16, device=dev)
+    o = torch.empty((1024, 1024), dtype=torch.float16, device=dev)
+
+    def chain():
+        cur = xd
+        for _ in range(10):
+            api.aq_qmm(cur, *q1, 4, 64, out=h)
+            api.aq_qmm(h, *q2, 4, 64, out=o)
+            cur = o
+    t = graph_time_ms(torch, stream, chain, 5)
+    fl = 20 * 2 * 1024 * 4096 * 1024
+    out["chained_fp16_4bit"] = {"tflops": round(fl / (t * 1e-3) / 1e12, 1), "ms_per_chain": round(t, 4)}
+    # FP4, M = 4096, E8M0 (finite) scales, bf16
+    codes, scales = inputs.fp4(4096, 4096, 32, seed=7)
+    xf = inputs.fp4_x(4096, 4096).to(dev)
+    wc, sc = codes.to(dev), scales.to(dev)
+    yf = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
+    t = graph_time_ms(torch, stream, lambda: api.aq_qmm(xf, wc, sc, None, 4, 32, out=yf), 10)
+    fl = 2 * 4096 ** 3
+    fp4 = {"tflops": round(fl / (t * 1e-3) / 1e12, 1), "ms": round(t, 4)}
+    out["fp4_e8m0_M4096"] = fp4
+    # affine 4-bit, M = N = K = 4096, bf16 (same shape as FP4)
+    wa = api.aq_quantize(inputs.normal((4096, 4096), 0.02, 1, inputs.gen(8)).to(dev), 4, 64)
+    t = graph_time_ms(torch, stream, lambda: api.aq_qmm(xf, *wa, 4, 64, out=yf), 10)
+    aff = {"tflops": round(fl / (t * 1e-3) / 1e12, 1), "ms": round(t, 4)}
+    out["affine4_M4096"] = aff
+    # conv2d, groups 1, 4-bit
+    xc, wcv = inputs.conv(1)
+    w2 = inputs.flatten_pad_conv_weight(wcv, 64)
+    qc = api.aq_quantize(w2.to(dev), 4, 64)
+    xcd = xc.to(dev)
+    yc = torch.empty((2, 64, 64, 320), dtype=torch.bfloat16, device=dev)
+    t = graph_time_ms(torch, stream, lambda: api.aq_qconv2d_nhwc(
+        xcd, *qc, 320, 3, 3, (1, 1), (1, 1), 1, 4, 64, out=yc), 10)
+    fl = 2 * 8192 * 320 * 2880
+    out["conv2d_g1_4bit"] = {"tflops": round(fl / (t * 1e-3) / 1e12, 1), "ms": round(t, 4)}
+    roof = {"bound": "tensor", "achieved": aff["tflops"], "peak": tf_peak, "unit": "TFLOP/s",
+            "frac": round(aff["tflops"] / tf_peak, 4), "peak_kind": "measured burst bf16",
+            "kernel": "qmm_tc_kernel (aq_qmm, 4-bit affine, M=N=K=4096)",
+            "traffic": traffic_for("qmm_tc_kernel", "affine4-M4096")}
+    return out, roof
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -225,34 +307,32 @@ def main():
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    hbm, tf, peak_kind = peaks()
+    hbm, tf, tf_sust, peak_kind = peaks()
 
     # Quantize the stack once (on the device, through the library).
     layers = []
     for li in range(LAYERS):
         ws = inputs.decode_layer(seed=100 + li)
-        q = {}
-        for name, w in ws.items():
-            q[name] = api.aq_quantize(w.to(dev), BITS, GS)
-        layers.append(q)
+        layers.append({name: api.aq_quantize(w.to(dev), BITS, GS) for name, w in ws.items()})
         del ws
     torch.cuda.synchronize()
     projs = inputs.LLAMA_1B_PROJ
-    xs = {(M, k): inputs.decode_x(M, k, seed=M).to(dev) for M in QMV_M for k in (2048, 8192)}
+    all_m = QMV_M + QMM_M
+    xs = {(M, k): inputs.decode_x(M, k, seed=M).to(dev) for M in all_m for k in (2048, 8192)}
     ys = {(M, name): torch.empty((M, n), dtype=torch.bfloat16, device=dev)
-          for M in QMV_M for name, n, _ in projs}
-    wsp = api.Workspace()
-    for M in QMV_M:                       # size the workspace before capture
-        for _, n, k in projs:
-            wsp.get(dev, api.aq_workspace_size(0, M, n, k, BITS, GS))
+          for M in all_m for name, n, _ in projs}
     launches_per_step = len(QMV_M) * LAYERS * len(projs)
+
+    def calls(M):
+        fn = api.aq_qmv if M <= 16 else api.aq_qmm
+        for q in layers:
+            for name, n, k in projs:
+                wq, s, b = q[name]
+                fn(xs[(M, k)], wq, s, b, BITS, GS, out=ys[(M, name)])
 
     def step():
         for M in QMV_M:
-            for q in layers:
-                for name, n, k in projs:
-                    wq, s, b = q[name]
-                    api.aq_qmv(xs[(M, k)], wq, s, b, BITS, GS, out=ys[(M, name)], workspace=wsp)
+            calls(M)
 
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
@@ -280,63 +360,54 @@ def main():
     step_bytes = LAYERS * sum(layer_bytes(M) for M in QMV_M)
     value = world * step_bytes / (ms * 1e-3) / 1e9
 
-    # Per-M view (each M's calls captured separately).
-    per_m = {}
-    with torch.cuda.stream(stream):
-        for M in QMV_M:
-            gm = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gm, stream=stream):
-                for q in layers:
-                    for name, n, k in projs:
-                        wq, s, b = q[name]
-                        api.aq_qmv(xs[(M, k)], wq, s, b, BITS, GS, out=ys[(M, name)], workspace=wsp)
-            for _ in range(3):
-                gm.replay()
-            a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(10):
-                gm.replay()
-            c.record(stream)
-            torch.cuda.synchronize()
-            t = a.elapsed_time(c) / 10
-            per_m[str(M)] = round(LAYERS * layer_bytes(M) / (t * 1e-3) / 1e9, 1)
-            del gm
+    # Per-M view: each M's 112 calls captured alone; per-kernel averages.
+    per_m, per_m_us = {}, {}
+    for M in all_m:
+        t = graph_time_ms(torch, stream, lambda: calls(M), 1)
+        per_m[str(M)] = round(LAYERS * layer_bytes(M) / (t * 1e-3) / 1e9, 1)
+        per_m_us[str(M)] = round(t * 1e3 / (LAYERS * len(projs)), 2)
 
     # End to end through the public API with host buffers: pinned x in,
     # every y out, around the same graph.
-    host_x = {key: v.cpu().pin_memory() for key, v in xs.items()}
-    host_y = {key: torch.empty(v.shape, dtype=v.dtype).pin_memory() for key, v in ys.items()}
+    host_x = {key: xs[key].cpu().pin_memory() for key in xs if key[0] in QMV_M}
+    host_y = {key: torch.empty(ys[key].shape, dtype=ys[key].dtype).pin_memory()
+              for key in ys if key[0] in QMV_M}
     h2d = sum(v.numel() * 2 for v in host_x.values())
     d2h = sum(v.numel() * 2 for v in host_y.values())
     with torch.cuda.stream(stream):
-        for _ in range(2):
-            for key in xs:
+        def e2e_step():
+            for key in host_x:
                 xs[key].copy_(host_x[key], non_blocking=True)
             g.replay()
-            for key in ys:
+            for key in host_y:
                 host_y[key].copy_(ys[key], non_blocking=True)
+        for _ in range(2):
+            e2e_step()
         torch.cuda.synchronize()
         barrier(world)
         a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(args.steps):
-            for key in xs:
-                xs[key].copy_(host_x[key], non_blocking=True)
-            g.replay()
-            for key in ys:
-                host_y[key].copy_(ys[key], non_blocking=True)
+            e2e_step()
         c.record(stream)
         torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a.elapsed_time(c) / args.steps, world)
-    e2e = {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+    e2e = {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    kernel_ms = ms / launches_per_step
-    achieved = (step_bytes / launches_per_step) / (kernel_ms * 1e-3) / 1e9
+    # Dominant kernel of the step: the kernel class with the largest share of
+    # the step (fp32 qmv for M <= 2, tensor-core qmm for M >= 4).
+    share = {"qmv_kernel (aq_qmv M<=2)": sum(per_m_us[str(M)] for M in QMV_M if M <= 2),
+             "qmm_tc_kernel (aq_qmv M>=4)": sum(per_m_us[str(M)] for M in QMV_M if M > 2)}
+    dom = max(share, key=share.get)
+    dom_m = [M for M in QMV_M if (M <= 2) == dom.startswith("qmv")]
+    dom_bytes = LAYERS * sum(layer_bytes(M) for M in dom_m)
+    dom_us = sum(per_m_us[str(M)] for M in dom_m) * LAYERS * len(projs)
+    achieved = dom_bytes / (dom_us * 1e-6) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-            "frac": round(achieved / hbm, 4), "peak_kind": peak_kind,
-            "kernel": "qmv_kernel (aq_qmv)",
-            "traffic": traffic_for("qmv_kernel", "decode-stack")}
+            "frac": round(achieved / hbm, 4), "peak_kind": peak_kind + " copy bandwidth",
+            "kernel": dom, "launch_share": {k: round(v / sum(share.values()), 3) for k, v in share.items()},
+            "traffic": traffic_for(dom.split()[0], "decode-stack")}
     line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -345,8 +416,12 @@ def main():
                        "group_size": GS, "parallelism": "replicas" if world > 1 else "single",
                        "l2": "weights 547 MB > 4x L2 per step; no flush needed",
                        "timing": "CUDA graph replay, CUDA events on the launching stream"},
-            "per_m_gbs": per_m, "roofline": roof, "clocks": clk.summary(), "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps}
+            "per_m_gbs": per_m, "per_call_us": per_m_us, "roofline": roof,
+            "clocks": clk.summary(), "e2e": e2e, "gpu_launches": launches_per_step * args.steps}
+    if not args.no_qmm:
+        qmm, roof_qmm = qmm_lines(torch, api, inputs, dev, stream, tf, tf_sust)
+        line["qmm_tflops"] = qmm
+        line["roofline_qmm"] = roof_qmm
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -26,6 +26,8 @@ aq_status cuda_status(cudaError_t e, const char* what) {
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
 const int64_t kMaxDim = (int64_t(1) << 31) - 1;
+// aq_qmv runs the fp32 weight-streaming kernel up to this many rows of x.
+const int64_t kQmvSimtMaxM = 2;
 
 // Format checks shared by every entry point.
 aq_status check_format(int bits, int gs, aq_mode mode, aq_dtype dt) {
@@ -131,13 +133,15 @@ aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void*
   if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
   if (N == 0) return AQ_OK;
   if (K == 0) return zero_output(y, M, N, stream);
-  const aq::QmvPlan p = aq::plan_qmv(M, N, K, bits, group_size, mode);
-  if (p.ws_bytes) {
-    if (!workspace || workspace_bytes < p.ws_bytes)
-      return fail(AQ_ERR_WORKSPACE, "aq_qmv needs %zu workspace bytes (got %zu%s)", p.ws_bytes,
-                  workspace_bytes, workspace ? "" : ", NULL");
-    if (!aligned(workspace, 256)) return fail(AQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  if (M > kQmvSimtMaxM) {
+    // From 3 rows of x on, the tensor-core kernel streams the weight faster
+    // than fp32 FMAs can consume it (each code costs M FMAs on CUDA cores).
+    const aq::QmmPlan p = aq::plan_qmm(M, N, K, bits, group_size, mode);
+    return cuda_status(aq::launch_qmm(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
+                                      mode, dtype, (cudaStream_t)stream),
+                       "aq_qmv launch");
   }
+  const aq::QmvPlan p = aq::plan_qmv(M, N, K, bits, group_size, mode);
   return cuda_status(aq::launch_qmv(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
                                     mode, dtype, workspace, (cudaStream_t)stream),
                      "aq_qmv launch");

@@ -1,4 +1,5 @@
-// qmv.cu — weight-streaming GEMV for few rows of x (M <= 16).
+// qmv.cu — fp32 weight-streaming GEMV for one or two rows of x (aq_qmv routes
+// 3..16 rows to the tensor-core kernel, which consumes codes faster there).
 //
 // Prior art: affine_packed_qmv_fast in "Add the 3bit packed qmm_t" (one
 // simdgroup streams a few weight rows, fp32 accumulation, simd_sum).  The
@@ -270,13 +271,8 @@ template <typename T, int BITS, bool FP4>
 cudaError_t by_mt(const QmvPlan& p, const void* x, const void* w_q, const void* scales,
                   const void* biases, void* y, int64_t M, int64_t N, int64_t K, int gs,
                   cudaStream_t st) {
-  switch (p.mt) {
-    case 1: return launch_one<T, BITS, 1, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
-    case 2: return launch_one<T, BITS, 2, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
-    case 4: return launch_one<T, BITS, 4, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
-    case 8: return launch_one<T, BITS, 8, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
-    default: return launch_one<T, BITS, 16, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
-  }
+  if (p.mt == 1) return launch_one<T, BITS, 1, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+  return launch_one<T, BITS, 2, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
 }
 
 template <typename T>
@@ -300,7 +296,7 @@ cudaError_t by_bits(const QmvPlan& p, const void* x, const void* w_q, const void
 QmvPlan plan_qmv(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
   (void)bits; (void)gs; (void)mode;
   QmvPlan p{};
-  p.mt = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
+  p.mt = M <= 1 ? 1 : 2;          // aq_qmv sends M > 2 to the tensor-core kernel
   const int64_t units = K / kUnit;
   // Shared memory per staged unit and row of x: 36 floats + 1 sum.
   const int64_t smem_cap = 160 * 1024;

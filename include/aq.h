@@ -110,7 +110,10 @@ AQ_API aq_status aq_dequantize(const void* w_q, const void* scales, const void* 
 /*
  * aq_qmv — y = x . w_hat^T for small M (1 <= M <= 16): the weight-streaming
  * path ("Add the 3bit packed qmm_t", affine_packed_qmv_fast, routed for few
- * rows of x).  x [M, K] T, y [M, N] T, fp32 accumulation.  K-slices are
+ * rows of x).  x [M, K] T, y [M, N] T, fp32 accumulation.  For M <= 2 an
+ * fp32 CUDA-core kernel with the scale and bias hoisted out of each group's
+ * dot product (w_hat never rounded); for M >= 3 the tensor-core kernel of
+ * aq_qmm, which reads the weight once for all rows of x.  K-slices are
  * reduced inside a thread block cluster, so no workspace is needed
  * (aq_workspace_size returns 0; workspace may be NULL and is not touched).
  * Returns AQ_ERR_INVALID_ARG for M outside 1..16.

@@ -1,5 +1,9 @@
 """GPU parity for aq_qmv against the oracle, within
-|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref)."""
+|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref).
+
+aq_qmv keeps w_hat in fp32 for M <= 2 (checked against the exact product) and
+hands M >= 3 to the tensor-core kernel, which multiplies T-valued weight tiles
+(checked against the product over w_hat rounded to T)."""
 import numpy as np
 import pytest
 import torch
@@ -26,7 +30,8 @@ def _check(x, wq, s, b, y, bits, gs, dt, mode=0, **kw):
     N = wq.shape[0]
     sc = dev_u8(s) if mode == 1 else dev_u16(s)
     bi = None if b is None else dev_u16(b)
-    yr, den = oracle.qmm(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt)
+    yr, den = oracle.qmm(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt,
+                         w_in_t=x.shape[0] > 2)
     return check_matmul(dev_u16(y), yr, den, dt, **kw)
 
 
