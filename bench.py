@@ -48,11 +48,13 @@ WORKLOAD = ("decode sweep: 16-layer Llama-3.2-1B-shaped stack (q/o 2048x2048, k/
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-qmm", action="store_true", help="skip the TFLOP/s side lines")
+    ap.add_argument("--only", default="all", choices=["all", "qmm"],
+                    help="qmm: run only the TFLOP/s workloads (for profiling)")
     return ap.parse_args()
 
 
@@ -77,7 +79,8 @@ def layer_bytes(M):
 
 
 class ClockSampler:
-    """Samples nvidia-smi during the timed region."""
+    """Samples SM clocks and throttle reasons with nvidia-smi's own loop
+    (-lms 50) while the timed region runs."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -86,29 +89,33 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.samples = []
-        self._stop = threading.Event()
-        self._t = None
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                out = subprocess.run(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                                      "--format=csv,noheader,nounits"], capture_output=True,
-                                     text=True, timeout=5).stdout.strip()
-                if out:
-                    self.samples.append([v.strip() for v in out.split(",")])
-            except Exception:
-                pass
-            self._stop.wait(0.1)
+        self._p = None
 
     def __enter__(self):
-        self._t = threading.Thread(target=self._run, daemon=True)
-        self._t.start()
+        try:
+            self._p = subprocess.Popen(["nvidia-smi", "-i", str(self.index),
+                                        "--query-gpu=" + self.FIELDS,
+                                        "--format=csv,noheader,nounits", "-lms", "50"],
+                                       stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)                      # let the first sample land
+        except Exception:
+            self._p = None
         return self
 
     def __exit__(self, *a):
-        self._stop.set()
-        self._t.join(timeout=10)
+        if self._p is None:
+            return
+        time.sleep(0.1)
+        self._p.terminate()
+        try:
+            out, _ = self._p.communicate(timeout=5)
+        except Exception:
+            self._p.kill()
+            out = ""
+        for ln in out.splitlines():
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) >= 8:
+                self.samples.append(f)
 
     def summary(self):
         if not self.samples:
@@ -308,6 +315,12 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     hbm, tf, tf_sust, peak_kind = peaks()
+    if args.only == "qmm":
+        stream = torch.cuda.Stream(dev)
+        qmm, roof_qmm = qmm_lines(torch, api, inputs, dev, stream, tf, tf_sust)
+        if rank == 0:
+            print(json.dumps({"qmm_tflops": qmm, "roofline_qmm": roof_qmm}))
+        return
 
     # Quantize the stack once (on the device, through the library).
     layers = []
