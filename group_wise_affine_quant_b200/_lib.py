@@ -32,6 +32,8 @@ SIGNATURES = {
     "aq_last_error": (ctypes.c_char_p, []),
     "aq_version": (_I, []),
     "aq_device_errors": (ctypes.c_uint, []),
+    "aq_set_weight_prefetch": (None, [_I]),
+    "aq_get_weight_prefetch": (_I, []),
 }
 
 _lib = None

@@ -13,8 +13,8 @@ from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, 
                    AQ_OP_QMV, AqError, check, lib)
 
 __all__ = ["aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmm", "aq_qconv2d_nhwc",
-           "aq_workspace_size", "aq_last_error", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4",
-           "Workspace"]
+           "aq_workspace_size", "aq_last_error", "aq_set_weight_prefetch",
+           "aq_get_weight_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
 
 _DT = {torch.float16: AQ_F16, torch.bfloat16: AQ_BF16}
 _TORCH_DT = {AQ_F16: torch.float16, AQ_BF16: torch.bfloat16}
@@ -40,11 +40,9 @@ def _mode(scales):
 
 
 class Workspace:
-    """Per-device zero-initialised scratch buffer, grown on demand.
-
-    The kernels leave their counters at zero after every call, so one buffer
-    serves all calls issued on one stream; calls on different streams need
-    different Workspace objects."""
+    """Per-device zero-initialised scratch buffer for the ABI's workspace
+    argument, grown on demand.  The current kernels report a workspace size of
+    0 (split-K reduces inside thread block clusters), so none is allocated."""
 
     def __init__(self):
         self._bufs = {}
@@ -60,6 +58,15 @@ class Workspace:
 
 
 _default_ws = Workspace()
+
+
+def aq_set_weight_prefetch(enable):
+    """Stream weights before waiting on the previous kernel (see include/aq.h)."""
+    lib().aq_set_weight_prefetch(1 if enable else 0)
+
+
+def aq_get_weight_prefetch():
+    return bool(lib().aq_get_weight_prefetch())
 
 
 def aq_last_error():

@@ -4,6 +4,8 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace {
@@ -70,9 +72,21 @@ aq_status check_weight(const void* w_q, const void* scales, const void* biases, 
 
 }  // namespace
 
+namespace {
+std::atomic<int> g_weight_prefetch{0};
+}
+
+int aq::weight_prefetch_enabled() { return g_weight_prefetch.load(std::memory_order_relaxed); }
+
 extern "C" {
 
 const char* aq_last_error(void) { return g_err; }
+
+void aq_set_weight_prefetch(int enable) {
+  g_weight_prefetch.store(enable ? 1 : 0, std::memory_order_relaxed);
+}
+
+int aq_get_weight_prefetch(void) { return aq::weight_prefetch_enabled(); }
 
 int aq_version(void) { return 100; }
 

@@ -122,5 +122,7 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
                          int sh, int sw, int ph, int pw, int groups, int bits, int gs, int dtype,
                          cudaStream_t st);
 cudaError_t read_device_error_qmm(unsigned* out);
+// aq_set_weight_prefetch's process-wide setting (0 or 1).
+int weight_prefetch_enabled();
 cudaError_t read_device_error_conv(unsigned* out);
 }  // namespace aq

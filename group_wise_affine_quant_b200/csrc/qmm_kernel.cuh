@@ -109,6 +109,7 @@ struct QmmArgs {
   // (i * kw + j) * Cg + c over the k_real = kh * kw * Cg real columns).
   int Cin, Cg, H, W, Ho, Wo, kh, kw, sh, sw, ph, pw, k_real;
   const void* x;        // conv gather path
+  int weights_early;    // load weights/scales before waiting on the previous kernel
 };
 
 struct QmmMaps {
@@ -469,8 +470,12 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Programmatic dependent launch: the next kernel in the stream may start
+  // its prologue now; it waits for this grid before touching its own inputs.
+  pdl_launch_dependents();
 
   if (warp == 0) {
+    pdl_wait();                                           // x may come from the previous kernel
     if constexpr (XMODE == 0) {
       // -------------------------------------------------- TMA producer (x)
       if (lane == 0) {
@@ -556,6 +561,9 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
       }
     }
   } else if (warp == kLoaderWarp) {
+    // Weights, scales and biases are read before the dependency wait only when
+    // the caller has declared that no preceding kernel writes them.
+    if (!a.weights_early) pdl_wait();
     if constexpr (FAST) {
       // ------------------- weight and scale chunks by TMA, in K order
       if (lane == 0) {
@@ -794,6 +802,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     }
 
     // ------------------------------------------------------- epilogue
+    pdl_wait();                                           // before y is written
     const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, 4000000000ull);
     tc_fence_after();
     const int q = warp & 3;                                 // TMEM lane quarter
@@ -826,6 +835,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
 
   // --------------------------------------------------------- split-K reduce
   if (a.splits > 1) {
+    pdl_wait();
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     if (!*abort_flag) {
@@ -924,13 +934,15 @@ cudaError_t launch_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, c
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = S::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = (unsigned)p.splits;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, maps, a);
 }
 

@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kThreads)
 qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
            const void* __restrict__ scales_v, const T* __restrict__ biases, T* __restrict__ y,
            int M, int64_t N, int64_t K, int gs_log2, int64_t Ks, int S, int lpr_log2, int RI,
-           int chunk_units) {
+           int chunk_units, int weights_early) {
   const int gs = 1 << gs_log2;
   extern __shared__ float4 smem4[];
   float* smem = reinterpret_cast<float*>(smem4);
@@ -100,14 +100,20 @@ qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
   const int64_t G = K >> gs_log2;
   const int64_t row_bytes = K * BITS / 8;
 
+  // Programmatic dependent launch: let the next kernel start its prologue.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // Prefetch this lane's first weight unit before staging x, so the HBM
-  // latency overlaps the staging.
+  // latency overlaps the staging (and, when the caller allows it, the end
+  // of the previous kernel: weights are then read before the dependency
+  // wait, x only after it).
+  if (!weights_early) asm volatile("griddepcontrol.wait;" ::: "memory");
   uint32_t wd[BITS];
   {
     const int64_t row = row_base + warp * rpw + seg;
     if (row < N && ul < nunits && ul < chunk_units)
       load_unit<BITS>(wq + row * row_bytes + k0 * BITS / 8 + (int64_t)ul * (4 * BITS), wd);
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   for (int c0 = 0; c0 < nunits; c0 += chunk_units) {
     const int cu = (nunits - c0 < chunk_units) ? (nunits - c0) : chunk_units;
@@ -255,16 +261,18 @@ cudaError_t launch_one(const QmvPlan& p, const void* x, const void* w_q, const v
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = (unsigned)p.splits;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, (const T*)x, (const uint8_t*)w_q, scales,
                             (const T*)biases, (T*)y, (int)M, N, K, ilog2_floor(gs), p.ks, p.splits,
-                            ilog2_floor(p.lpr), p.ri, p.chunk_units);
+                            ilog2_floor(p.lpr), p.ri, p.chunk_units, weight_prefetch_enabled());
 }
 
 template <typename T, int BITS, bool FP4>

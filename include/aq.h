@@ -173,6 +173,20 @@ AQ_API size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int b
  */
 AQ_API unsigned aq_device_errors(void);
 
+/*
+ * Weight prefetch across kernel boundaries (process-wide, default 0 = off).
+ * Every qmv / qmm / conv kernel is launched with programmatic dependent
+ * launch, so it may start while the previous kernel on its stream is still
+ * running; it always waits for that kernel before reading x or writing y.
+ * With prefetch on, it also streams w_q, scales and biases before that wait,
+ * which hides most of a small matmul's start-up behind the previous kernel.
+ * Turn it on only when no kernel launched just before a matmul on the same
+ * stream writes that matmul's weights (e.g. not directly after aq_quantize
+ * of the same weights without a synchronising operation in between).
+ */
+AQ_API void aq_set_weight_prefetch(int enable);
+AQ_API int aq_get_weight_prefetch(void);
+
 /* Message for the last non-AQ_OK status on the calling thread ("" if none). */
 AQ_API const char* aq_last_error(void);
 

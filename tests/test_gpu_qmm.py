@@ -171,6 +171,57 @@ def test_qmm_matches_qmv_small_m():
     _check(x, wq, s, b, y2, 4, 64, 1, w_in_t=False)    # qmv keeps w_hat in fp32
 
 
+@pytest.mark.parametrize("prefetch", [False, True])
+def test_dependent_chain_under_pdl(prefetch):
+    """Back-to-back dependent calls on one stream (each kernel may start
+    before the previous one ends): y feeds the next call's x and is
+    overwritten by a later call.  Results equal the same calls separated by
+    device synchronisation."""
+    bits, gs = 4, 64
+    g = inputs.gen(21)
+    ws = [api.aq_quantize(to_dev(inputs.normal((512, 512), 0.05, 1, g)), bits, gs) for _ in range(4)]
+    x = to_dev(inputs.normal((8, 512), 1.0, 1, g))
+    torch.cuda.synchronize()
+    ref = []
+    cur = x
+    for i in range(6):
+        fn = api.aq_qmv if i % 2 else api.aq_qmm
+        cur = fn(cur, *ws[i % 4], bits, gs)
+        torch.cuda.synchronize()
+        ref.append(cur.clone())
+    old = api.aq_get_weight_prefetch()
+    api.aq_set_weight_prefetch(prefetch)
+    try:
+        a = torch.empty_like(x)
+        b = torch.empty_like(x)
+        a.copy_(x)
+        outs = []
+        for i in range(6):
+            fn = api.aq_qmv if i % 2 else api.aq_qmm
+            dst = b if i % 2 == 0 else a
+            src = a if i % 2 == 0 else b
+            fn(src, *ws[i % 4], bits, gs, out=dst)
+            outs.append(dst)
+            if i in (1, 3, 5):
+                outs[-1] = dst.clone()
+        torch.cuda.synchronize()
+    finally:
+        api.aq_set_weight_prefetch(old)
+    for i in (1, 3, 5):
+        assert torch.equal(outs[i], ref[i]), i
+
+
+def test_quantize_then_matmul_default_order():
+    """Weights written by the kernel just before (prefetch off by default)."""
+    assert not api.aq_get_weight_prefetch()
+    w = to_dev(inputs.normal((256, 1024), 0.05, 1, inputs.gen(5)))
+    x = to_dev(inputs.normal((4, 1024), 1.0, 1, inputs.gen(6)))
+    q = api.aq_quantize(w, 4, 64)
+    y = api.aq_qmm(x, *q, 4, 64)
+    torch.cuda.synchronize()
+    _check(x, *q, y, 4, 64, 1)
+
+
 def test_qmm_empty():
     x = torch.zeros((0, 64), dtype=torch.float16, device=DEV)
     wq = torch.zeros((128, 32), dtype=torch.uint8, device=DEV)
