@@ -54,10 +54,10 @@ using namespace sm100;
 
 constexpr int kBK = 64;                  // K elements per stage (128 bytes of T)
 constexpr int kRowsW = 128;              // weight rows per tile (MMA M)
-constexpr int kThreads = 352;            // 11 warps
-constexpr int kProducerWarp0 = 2;        // warps 2..9: two groups of 4 dequantizer warps
-constexpr int kDqGroups = 2;             // group g takes K-stages i with i % 2 == g
-constexpr int kLoaderWarp = 10;          // streams packed codes, scales, biases
+constexpr int kDqGroups = 4;             // group g takes K-stages i with i % kDqGroups == g
+constexpr int kProducerWarp0 = 2;        // warps 2 .. 2 + 4 * kDqGroups - 1: dequantizer groups
+constexpr int kLoaderWarp = kProducerWarp0 + 4 * kDqGroups;   // packed codes, scales, biases
+constexpr int kThreads = 32 * (kLoaderWarp + 1);
 
 template <int BT, int BITS, bool FAST>
 struct QmmShape {
@@ -455,8 +455,8 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     }
     for (int s = 0; s < NL; ++s) {
       mbar_init(full_l(s), FAST ? 1 : 32);   // TMA arrive + tx, or every loader lane
-      // TMA path: every chunk spans >= 2 K-stages, so both dequantizer
-      // groups release it; cp.async path: one stage, one group.
+      // TMA path: every dequantizer group releases every chunk (after its
+      // data has landed); cp.async path: one stage, one group.
       mbar_init(empty_l(s), FAST ? 4 * kDqGroups : 4);
     }
     mbar_init(acc_full, 1);
@@ -744,6 +744,16 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         const int s_done =
             last ? nsc : ((((kt + kDqGroups) * kBK) >> a.gs_log2) / SGC) - sc0;
         if (w_done > w_freed || s_done > s_freed) {
+          // A chunk is released only after its data has landed (which proves
+          // the slot's previous chunk was released by every group), so each
+          // arrival counts toward the right phase even for chunks this group
+          // never reads.
+          bool okr = true;
+          for (; w_ready < w_done && okr; ++w_ready)
+            okr = mbar_wait(full_l(w_ready % WS), (w_ready / WS) & 1, abort_flag);
+          for (; s_ready < s_done && okr; ++s_ready)
+            okr = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
+          if (!okr) break;
           __syncwarp();
           if (lane == 0) {
             for (int c = w_freed; c < w_done; ++c) mbar_arrive(empty_l(c % WS));
