@@ -679,6 +679,40 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     const bool fp4_g16 = FP4 && a.gs_log2 == 4;
     int w_ready = 0, w_freed = 0;                          // TMA path: chunks waited / released
     int s_ready = 0, s_freed = 0;
+    // Release weight chunks below w_done and scale chunks below s_done, in
+    // the loader's K order (weight chunk first on a tie), waiting for each
+    // chunk's data to land just before releasing it.  Every group releases
+    // every chunk, so a chunk this group never reads is released too; the
+    // wait makes the arrival count toward the right phase of its slot, and
+    // the K order means the chunk waited for never sits behind a release this
+    // group still owes the loader.
+    auto release_upto = [&](int w_done, int s_done) -> bool {
+      bool okr = true;
+      while (okr && (w_freed < w_done || s_freed < s_done)) {
+        const int64_t kw = w_freed < w_done ? (int64_t)w_freed * 128 * 8 / BITS : INT64_MAX;
+        const int64_t ks = s_freed < s_done
+                               ? (int64_t)(sc0 + s_freed) * SGC * (1 << a.gs_log2) - (int64_t)kt0 * kBK
+                               : INT64_MAX;
+        if (kw <= ks) {
+          if (w_freed >= w_ready) {
+            okr = mbar_wait(full_l(w_freed % WS), (w_freed / WS) & 1, abort_flag);
+            w_ready = w_freed + 1;
+          }
+          __syncwarp();
+          if (okr && lane == 0) mbar_arrive(empty_l(w_freed % WS));
+          ++w_freed;
+        } else {
+          if (s_freed >= s_ready) {
+            okr = mbar_wait(full_l(WS + s_freed % SS), (s_freed / SS) & 1, abort_flag);
+            s_ready = s_freed + 1;
+          }
+          __syncwarp();
+          if (okr && lane == 0) mbar_arrive(empty_l(WS + s_freed % SS));
+          ++s_freed;
+        }
+      }
+      return okr;
+    };
     for (int i = grp; i < nkt; i += kDqGroups) {
       const int kt = kt0 + i;
       const bool tail = (kt + 1) * kBK > a.K;
@@ -743,25 +777,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         const int w_done = last ? nwc : (((i + kDqGroups) * S::kPB) >> 7);
         const int s_done =
             last ? nsc : ((((kt + kDqGroups) * kBK) >> a.gs_log2) / SGC) - sc0;
-        if (w_done > w_freed || s_done > s_freed) {
-          // A chunk is released only after its data has landed (which proves
-          // the slot's previous chunk was released by every group), so each
-          // arrival counts toward the right phase even for chunks this group
-          // never reads.
-          bool okr = true;
-          for (; w_ready < w_done && okr; ++w_ready)
-            okr = mbar_wait(full_l(w_ready % WS), (w_ready / WS) & 1, abort_flag);
-          for (; s_ready < s_done && okr; ++s_ready)
-            okr = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
-          if (!okr) break;
-          __syncwarp();
-          if (lane == 0) {
-            for (int c = w_freed; c < w_done; ++c) mbar_arrive(empty_l(c % WS));
-            for (int j = s_freed; j < s_done; ++j) mbar_arrive(empty_l(WS + j % SS));
-          }
-          w_freed = w_done > w_freed ? w_done : w_freed;
-          s_freed = s_done > s_freed ? s_done : s_freed;
-        }
+        if (!release_upto(w_done, s_done)) break;
       } else {
         const int ps = i % PST;
         if (!mbar_wait(full_l(ps), (i / PST) & 1, abort_flag)) break;
@@ -793,22 +809,8 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
       if (lane == 0) mbar_arrive(full_a(s));
     }
     if constexpr (FAST) {
-      // Chunks past this group's last stage are released too (both groups
-      // release every chunk), but only after their data has landed: the
-      // landing proves the slot's previous chunk was released by both
-      // groups, so this arrival counts toward the right phase.
-      bool ok = !*abort_flag;
-      for (; w_ready < nwc && ok; ++w_ready)
-        ok = mbar_wait(full_l(w_ready % WS), (w_ready / WS) & 1, abort_flag);
-      for (; s_ready < nsc && ok; ++s_ready)
-        ok = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
-      if (ok && (w_freed < nwc || s_freed < nsc)) {
-        __syncwarp();
-        if (lane == 0) {
-          for (int c = w_freed; c < nwc; ++c) mbar_arrive(empty_l(c % WS));
-          for (int j = s_freed; j < nsc; ++j) mbar_arrive(empty_l(WS + j % SS));
-        }
-      }
+      // Chunks past this group's last stage are released too.
+      if (!*abort_flag) release_upto(nwc, nsc);
     }
 
     // ------------------------------------------------------- epilogue
