@@ -54,10 +54,7 @@ using namespace sm100;
 
 constexpr int kBK = 64;                  // K elements per stage (128 bytes of T)
 constexpr int kRowsW = 128;              // weight rows per tile (MMA M)
-constexpr int kDqGroups = 4;             // group g takes K-stages i with i % kDqGroups == g
-constexpr int kProducerWarp0 = 2;        // warps 2 .. 2 + 4 * kDqGroups - 1: dequantizer groups
-constexpr int kLoaderWarp = kProducerWarp0 + 4 * kDqGroups;   // packed codes, scales, biases
-constexpr int kThreads = 32 * (kLoaderWarp + 1);
+constexpr int kProducerWarp0 = 2;        // warps 2 .. : dequantizer groups of 4 warps
 
 template <int BT, int BITS, bool FAST>
 struct QmmShape {
@@ -82,6 +79,14 @@ struct QmmShape {
   static constexpr int kOpBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
   static constexpr int kDataBytes = kOpBytes + kLoadBytes;
   static constexpr int kTmemCols = BT < 32 ? 32 : BT;
+  // Dequantizer groups: group g takes K-stages i with i % kGroups == g.  A
+  // group's consecutive stages are kGroups apart and its operand-slot wait
+  // is a phase-parity wait, which is unambiguous only while the slot's
+  // previous phase is already complete: that needs kGroups <= kStages.
+  static constexpr int kGroups = kStages < 4 ? kStages : 4;
+  static constexpr int kLoaderWarp = kProducerWarp0 + 4 * kGroups;
+  static constexpr int kThreads = 32 * (kLoaderWarp + 1);
+  static_assert(kGroups <= kStages, "parity waits need kGroups <= kStages");
   static constexpr int kBars = 3 * kStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
   static constexpr int kSmem = 1024 + kDataBytes + 512;             // align slack, barriers
   static_assert(kBars * 8 + 16 <= 512, "barrier area");
@@ -401,9 +406,12 @@ __device__ __forceinline__ uint32_t wchunk_off(int o, int r) {
 // 16-channel atom column of a K-stage, 32-byte swizzle); 2 = conv pixels
 // gathered with cp.async (16-byte granules, zero-filled outside the image).
 template <typename T, int BITS, bool FP4, int BT, bool FAST, int XMODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(QmmShape<BT, BITS, FAST>::kThreads, 1)
 qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   using S = QmmShape<BT, BITS, FAST>;
+  constexpr int kDqGroups = S::kGroups;
+  constexpr int kLoaderWarp = S::kLoaderWarp;
+  constexpr int kThreads = S::kThreads;
   constexpr int ST = S::kStages;
   constexpr int PST = S::kPStages;
   constexpr int WS = S::kWSlots;
@@ -943,7 +951,7 @@ cudaError_t launch_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, c
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.n_tiles, (unsigned)p.m_tiles, (unsigned)p.splits);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(S::kThreads, 1, 1);
   cfg.dynamicSmemBytes = S::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
