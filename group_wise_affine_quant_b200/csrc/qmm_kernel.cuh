@@ -859,16 +859,27 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     if (!*abort_flag) {
-      const float* red = reinterpret_cast<const float*>(ring);
-      for (int i = threadIdx.x; i < BT * kRowsW; i += kThreads) {
-        if (i % a.splits != split) continue;
-        const int j = i / kRowsW, rr = i - j * kRowsW;
+      // Rank `split` finishes a contiguous slice of the [BT][128] tile:
+      // 16-byte loads of every rank's parked partials, added in rank order.
+      const float4* red4 = reinterpret_cast<const float4*>(ring);
+      constexpr int kE4 = BT * kRowsW / 4;
+      const int per = (kE4 + a.splits - 1) / a.splits;
+      const int f0 = split * per, f1 = min(kE4, f0 + per);
+      for (int f = f0 + (int)threadIdx.x; f < f1; f += kThreads) {
+        float4 acc = cluster.map_shared_rank(red4, 0)[f];
+        for (int q = 1; q < a.splits; ++q) {
+          const float4 v = cluster.map_shared_rank(red4, q)[f];
+          acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        const int e = 4 * f;
+        const int j = e / kRowsW, rr = e - j * kRowsW;     // 4 consecutive weight rows
         const int m = m0 + j;
-        const int64_t orow = n0 + rr;
-        if (m >= a.M || nl0 + rr >= a.n_limit) continue;
-        float sum = 0.0f;
-        for (int q = 0; q < a.splits; ++q) sum += cluster.map_shared_rank(red, q)[i];
-        reinterpret_cast<T*>(a.y)[(int64_t)m * a.ldy + orow] = TT<T>::from_f(sum);
+        if (m >= a.M) continue;
+        T* yrow = reinterpret_cast<T*>(a.y) + (int64_t)m * a.ldy + n0 + rr;
+        const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          if (nl0 + rr + t < a.n_limit) yrow[t] = TT<T>::from_f(vals[t]);
       }
     }
     cluster.sync();

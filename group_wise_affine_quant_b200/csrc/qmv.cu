@@ -93,7 +93,7 @@ qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
   const int xs_stride = chunk_units * kUnitStride;
   float* xs = smem;                                         // [MT][xs_stride]
   float* bs = xs + MT * xs_stride;                          // [MT][chunk_units]
-  float* red = bs + MT * chunk_units;                       // [MT][rows_blk]
+  float* red = bs + ((MT * chunk_units + 3) & ~3);          // [MT][rows_blk], 16-byte aligned
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = lane >> lpr_log2, ul = lane & (lpr - 1);
@@ -222,14 +222,30 @@ qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
   // one so that no CTA exits while another still reads its shared memory.
   cg::cluster_group cluster = cg::this_cluster();
   if (S > 1) cluster.sync(); else __syncthreads();
-  for (int i = threadIdx.x; i < MT * rows_blk; i += kThreads) {
-    if (i % S != rank) continue;
-    const int m = i / rows_blk, rloc = i - m * rows_blk;
-    const int64_t row = row_base + rloc;
-    if (m >= M || row >= N) continue;
-    float sum = 0.0f;
-    for (int q = 0; q < S; ++q) sum += (S > 1 ? cluster.map_shared_rank(red, q) : red)[i];
-    y[(int64_t)m * N + row] = TT<T>::from_f(sum);
+  {
+    // Rank `rank` finishes a contiguous slice of the [MT][rows_blk] sums with
+    // 16-byte loads of every slice's partials (rows_blk is a multiple of 8),
+    // added in slice order.
+    const float4* red4 = reinterpret_cast<const float4*>(red);
+    const int e4 = MT * rows_blk / 4;
+    const int per = (e4 + S - 1) / S;
+    const int f0 = rank * per, f1 = min(e4, f0 + per);
+    for (int f = f0 + (int)threadIdx.x; f < f1; f += kThreads) {
+      float4 acc = (S > 1 ? cluster.map_shared_rank(red4, 0) : red4)[f];
+      for (int q = 1; q < S; ++q) {
+        const float4 v = cluster.map_shared_rank(red4, q)[f];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      const int e = 4 * f;
+      const int m = e / rows_blk, rloc = e - m * rows_blk;
+      if (m >= M) continue;
+      const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int64_t row = row_base + rloc + t;
+        if (row < N) y[(int64_t)m * N + row] = TT<T>::from_f(vals[t]);
+      }
+    }
   }
   if (S > 1) cluster.sync();
 }
@@ -338,8 +354,8 @@ QmvPlan plan_qmv(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
   }
   p.row_blocks = (N + (int64_t)p.rows_cta * p.ri - 1) / ((int64_t)p.rows_cta * p.ri);
   if (p.row_blocks < 1) p.row_blocks = 1;
-  p.smem = (size_t)p.mt * ((size_t)p.chunk_units * kUnitStride + p.chunk_units +
-                           (size_t)p.rows_cta * p.ri) * sizeof(float);
+  p.smem = ((size_t)p.mt * p.chunk_units * kUnitStride + (((size_t)p.mt * p.chunk_units + 3) & ~(size_t)3) +
+            (size_t)p.mt * p.rows_cta * p.ri) * sizeof(float);
   p.ws_bytes = 0;
   return p;
 }
