@@ -58,21 +58,26 @@ constexpr int kProducerWarp0 = 2;        // warps 2 .. : dequantizer groups of 4
 
 template <int BT, int BITS, bool FAST>
 struct QmmShape {
-  static constexpr int kStages = BT >= 256 ? 3 : 4;                 // operand stages
+  // Small token tiles (BT <= 32, the weight-streaming regime) use a light
+  // CTA (2 dequantizer groups, about 95 KB of shared memory) so that two
+  // CTAs fit on an SM: the next kernel of a stream can then start streaming
+  // its weights while this one finishes.  Larger tiles use a deeper pipeline.
+  static constexpr bool kLight = BT <= 32;
+  static constexpr int kStages = kLight ? 3 : BT >= 256 ? 3 : 4;   // operand stages
   static constexpr int kABytes = kRowsW * kBK * 2;                   // 16 KB
   static constexpr int kBBytes = BT * kBK * 2;                       // BT * 128
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kPB = 8 * BITS;                               // packed bytes / row / stage
   // cp.async path: one slot per stage, rows at a bank-spreading pitch.
-  static constexpr int kPStages = BT >= 256 ? 4 : BT >= 128 ? 6 : BT >= 64 ? 8 : BT >= 32 ? 10 : 12;
+  static constexpr int kPStages = kLight ? 4 : BT >= 256 ? 4 : BT >= 128 ? 6 : 8;
   static constexpr int kRP = (kPB % 32 == 0) ? kPB + 16 : kPB;
   static constexpr int kPSlot = kRowsW * kRP + kRowsW * 16;
   // TMA path: weight chunks of 128 rows x 128 bytes (128-byte swizzle) and
   // scale chunks of 128 rows x 16 bytes (scales, then biases).
   static constexpr int kWChunk = kRowsW * 128;                       // 16 KB
-  static constexpr int kWSlots = BT >= 256 ? 2 : BT >= 128 ? 3 : 4;
+  static constexpr int kWSlots = kLight ? 2 : BT >= 256 ? 2 : BT >= 128 ? 3 : 4;
   static constexpr int kSChunk = kRowsW * 16 * 2;                    // 4 KB
-  static constexpr int kSSlots = 4;
+  static constexpr int kSSlots = kLight ? 2 : 4;
   static constexpr int kLoadBytes = FAST ? kWSlots * kWChunk + kSSlots * kSChunk : kPStages * kPSlot;
   static constexpr int kRedBytes = BT * kRowsW * 4;                  // split-K parking
   static constexpr int kRingBytes = kStages * kStageBytes;
@@ -83,12 +88,12 @@ struct QmmShape {
   // group's consecutive stages are kGroups apart and its operand-slot wait
   // is a phase-parity wait, which is unambiguous only while the slot's
   // previous phase is already complete: that needs kGroups <= kStages.
-  static constexpr int kGroups = kStages < 4 ? kStages : 4;
+  static constexpr int kGroups = kLight ? 2 : (kStages < 4 ? kStages : 4);
   static constexpr int kLoaderWarp = kProducerWarp0 + 4 * kGroups;
   static constexpr int kThreads = 32 * (kLoaderWarp + 1);
-  static_assert(kGroups <= kStages, "parity waits need kGroups <= kStages");
   static constexpr int kBars = 3 * kStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
   static constexpr int kSmem = 1024 + kDataBytes + 512;             // align slack, barriers
+  static_assert(kGroups <= kStages, "parity waits need kGroups <= kStages");
   static_assert(kBars * 8 + 16 <= 512, "barrier area");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -406,7 +411,8 @@ __device__ __forceinline__ uint32_t wchunk_off(int o, int r) {
 // 16-channel atom column of a K-stage, 32-byte swizzle); 2 = conv pixels
 // gathered with cp.async (16-byte granules, zero-filled outside the image).
 template <typename T, int BITS, bool FP4, int BT, bool FAST, int XMODE>
-__global__ void __launch_bounds__(QmmShape<BT, BITS, FAST>::kThreads, 1)
+__global__ void __launch_bounds__(QmmShape<BT, BITS, FAST>::kThreads,
+                                  QmmShape<BT, BITS, FAST>::kLight ? 2 : 1)
 qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   using S = QmmShape<BT, BITS, FAST>;
   constexpr int kDqGroups = S::kGroups;
