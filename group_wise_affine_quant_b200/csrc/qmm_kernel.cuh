@@ -63,10 +63,14 @@ struct QmmShape {
   // CTAs fit on an SM: the next kernel of a stream can then start streaming
   // its weights while this one finishes.  Larger tiles use a deeper pipeline.
   static constexpr bool kLight = BT <= 32;
-  static constexpr int kStages = kLight ? 3 : BT >= 256 ? 3 : 4;   // operand stages
+  // Operand rings: kStages slots of dequantized A (the dequantizers refill
+  // them from shared memory, no memory latency to hide) and kBStages slots of
+  // x tiles (TMA from L2/HBM; one more slot at BT = 256, where the MMA stage
+  // is shortest relative to a TMA round trip).
+  static constexpr int kStages = kLight ? 3 : BT >= 256 ? 3 : 4;
+  static constexpr int kBStages = BT >= 256 ? 4 : kStages;
   static constexpr int kABytes = kRowsW * kBK * 2;                   // 16 KB
   static constexpr int kBBytes = BT * kBK * 2;                       // BT * 128
-  static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kPB = 8 * BITS;                               // packed bytes / row / stage
   // cp.async path: one slot per stage, rows at a bank-spreading pitch.
   static constexpr int kPStages = kLight ? 4 : BT >= 256 ? 4 : BT >= 128 ? 6 : 8;
@@ -80,7 +84,7 @@ struct QmmShape {
   static constexpr int kSSlots = kLight ? 2 : 4;
   static constexpr int kLoadBytes = FAST ? kWSlots * kWChunk + kSSlots * kSChunk : kPStages * kPSlot;
   static constexpr int kRedBytes = BT * kRowsW * 4;                  // split-K parking
-  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kRingBytes = kStages * kABytes + kBStages * kBBytes;
   static constexpr int kOpBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
   static constexpr int kDataBytes = kOpBytes + kLoadBytes;
   static constexpr int kTmemCols = BT < 32 ? 32 : BT;
@@ -91,7 +95,7 @@ struct QmmShape {
   static constexpr int kGroups = kLight ? 2 : (kStages < 4 ? kStages : 4);
   static constexpr int kLoaderWarp = kProducerWarp0 + 4 * kGroups;
   static constexpr int kThreads = 32 * (kLoaderWarp + 1);
-  static constexpr int kBars = 3 * kStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
+  static constexpr int kBars = 2 * kStages + 2 * kBStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
   static constexpr int kSmem = 1024 + kDataBytes + 512;             // align slack, barriers
   static_assert(kGroups <= kStages, "parity waits need kGroups <= kStages");
   static_assert(kBars * 8 + 16 <= 512, "barrier area");
@@ -418,20 +422,23 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   constexpr int kDqGroups = S::kGroups;
   constexpr int kLoaderWarp = S::kLoaderWarp;
   constexpr int kThreads = S::kThreads;
-  constexpr int ST = S::kStages;
+  constexpr int ST = S::kStages;                          // A slots
+  constexpr int SB = S::kBStages;                         // B slots
   constexpr int PST = S::kPStages;
   constexpr int WS = S::kWSlots;
   constexpr int SS = S::kSSlots;
   constexpr int SGC = FP4 ? 16 : 8;                       // groups per scale chunk (16 bytes)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* ring = smem;                                   // [ST] x (A 16 KB | B BT*128)
+  uint8_t* ring = smem;                                   // operand rings (and split-K parking)
+  uint8_t* ring_a = smem;                                 // [ST] A 16 KB
+  uint8_t* ring_b = smem + ST * S::kABytes;               // [SB] B BT*128
   uint8_t* pring = smem + S::kOpBytes;                    // loader area
   uint8_t* wring = pring;                                 // TMA path: [WS] weight chunks
   uint8_t* sring = pring + WS * S::kWChunk;               // TMA path: [SS] scale chunks
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kDataBytes);
   constexpr int NL = FAST ? WS + SS : PST;                // loader slots
-  // bars: full_a[ST], full_b[ST], empty[ST], full_l[NL], empty_l[NL], acc_full
+  // bars: full_a[ST], empty_a[ST], full_b[SB], empty_b[SB], full_l[NL], empty_l[NL], acc_full
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -447,11 +454,12 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   const int G = a.K >> a.gs_log2;
 
   auto full_a = [&](int s) { return smem_u32(bars + s); };
-  auto full_b = [&](int s) { return smem_u32(bars + ST + s); };
-  auto empty = [&](int s) { return smem_u32(bars + 2 * ST + s); };
-  auto full_l = [&](int s) { return smem_u32(bars + 3 * ST + s); };
-  auto empty_l = [&](int s) { return smem_u32(bars + 3 * ST + NL + s); };
-  const uint32_t acc_full = smem_u32(bars + 3 * ST + 2 * NL);
+  auto empty_a = [&](int s) { return smem_u32(bars + ST + s); };
+  auto full_b = [&](int s) { return smem_u32(bars + 2 * ST + s); };
+  auto empty_b = [&](int s) { return smem_u32(bars + 2 * ST + SB + s); };
+  auto full_l = [&](int s) { return smem_u32(bars + 2 * ST + 2 * SB + s); };
+  auto empty_l = [&](int s) { return smem_u32(bars + 2 * ST + 2 * SB + NL + s); };
+  const uint32_t acc_full = smem_u32(bars + 2 * ST + 2 * SB + 2 * NL);
 
   // TMA path bookkeeping: weight chunk c covers bytes [wb0 + 128 c, +128) of
   // every row, scale chunk j covers groups [SGC j, SGC (j + 1)).
@@ -464,8 +472,11 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(full_a(s), 4);          // one arrive per dequantizer warp
+      mbar_init(empty_a(s), 1);         // MMA commit
+    }
+    for (int s = 0; s < SB; ++s) {
       mbar_init(full_b(s), XMODE == 2 ? 32 : 1);   // TMA arrive + tx, or every gather lane
-      mbar_init(empty(s), 1);           // MMA commit
+      mbar_init(empty_b(s), 1);         // MMA commit
     }
     for (int s = 0; s < NL; ++s) {
       mbar_init(full_l(s), FAST ? 1 : 32);   // TMA arrive + tx, or every loader lane
@@ -494,11 +505,11 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
       // -------------------------------------------------- TMA producer (x)
       if (lane == 0) {
         for (int i = 0; i < nkt; ++i) {
-          const int s = i % ST;
-          const uint32_t par = ((i / ST) & 1) ^ 1;
-          if (!mbar_wait(empty(s), par, abort_flag)) break;
+          const int s = i % SB;
+          const uint32_t par = ((i / SB) & 1) ^ 1;
+          if (!mbar_wait(empty_b(s), par, abort_flag)) break;
           mbar_arrive_expect_tx(full_b(s), S::kBBytes);
-          tma_load_2d(smem_u32(ring + s * S::kStageBytes + S::kABytes), &maps.x, full_b(s),
+          tma_load_2d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full_b(s),
                       (kt0 + i) * kBK, m0);
         }
       }
@@ -511,11 +522,11 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         const int ho0 = rem / a.Wo, wo0 = rem - (rem / a.Wo) * a.Wo;
         const int taps = a.kh * a.kw;
         for (int i = 0; i < nkt; ++i) {
-          const int s = i % ST;
-          const uint32_t par = ((i / ST) & 1) ^ 1;
-          if (!mbar_wait(empty(s), par, abort_flag)) break;
+          const int s = i % SB;
+          const uint32_t par = ((i / SB) & 1) ^ 1;
+          if (!mbar_wait(empty_b(s), par, abort_flag)) break;
           mbar_arrive_expect_tx(full_b(s), S::kBBytes);
-          const uint32_t dst = smem_u32(ring + s * S::kStageBytes + S::kABytes);
+          const uint32_t dst = smem_u32(ring_b + s * S::kBBytes);
 #pragma unroll
           for (int at = 0; at < 4; ++at) {
             const int kk = (kt0 + i) * kBK + 16 * at;
@@ -533,15 +544,15 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
       }
     } else {
       // ------------------ conv pixels: cp.async gather of 16-byte granules
-      constexpr int kLagB = ST - 1;
+      constexpr int kLagB = SB - 1;
       const int taps = a.kh * a.kw;
       const int hw = a.Ho * a.Wo;
       int published = 0;
       for (int i = 0; i < nkt; ++i) {
-        const int s = i % ST;
-        const uint32_t par = ((i / ST) & 1) ^ 1;
-        if (!mbar_wait(empty(s), par, abort_flag)) break;
-        const uint32_t dst = smem_u32(ring + s * S::kStageBytes + S::kABytes);
+        const int s = i % SB;
+        const uint32_t par = ((i / SB) & 1) ^ 1;
+        if (!mbar_wait(empty_b(s), par, abort_flag)) break;
+        const uint32_t dst = smem_u32(ring_b + s * S::kBBytes);
         for (int idx = lane; idx < BT * 8; idx += 32) {
           const int j = idx >> 3, q = idx & 7;           // pixel row, granule of 8 channels
           const int kk = (kt0 + i) * kBK + 8 * q;
@@ -565,13 +576,13 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         cp_async_commit();
         if (i - kLagB >= 0) {
           cp_async_wait_group<kLagB>();
-          mbar_arrive(full_b((i - kLagB) % ST));
+          mbar_arrive(full_b((i - kLagB) % SB));
           published = i - kLagB + 1;
         }
       }
       cp_async_wait_all();
       if (!*abort_flag) {
-        for (int i = published; i < nkt; ++i) mbar_arrive(full_b(i % ST));
+        for (int i = published; i < nkt; ++i) mbar_arrive(full_b(i % SB));
       }
     }
   } else if (warp == kLoaderWarp) {
@@ -665,20 +676,21 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(std::is_same<T, __nv_bfloat16>::value, kRowsW, BT);
       for (int i = 0; i < nkt; ++i) {
-        const int s = i % ST;
-        const uint32_t par = (i / ST) & 1;
-        if (!(mbar_wait(full_a(s), par, abort_flag) && mbar_wait(full_b(s), par, abort_flag)))
+        const int s = i % ST, sb = i % SB;
+        if (!(mbar_wait(full_a(s), (i / ST) & 1, abort_flag) &&
+              mbar_wait(full_b(sb), (i / SB) & 1, abort_flag)))
           break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(ring + s * S::kStageBytes);
-        const uint32_t b_addr = a_addr + S::kABytes;
+        const uint32_t a_addr = smem_u32(ring_a + s * S::kABytes);
+        const uint32_t b_addr = smem_u32(ring_b + sb * S::kBBytes);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           const uint64_t bdesc = XMODE == 0 ? sdesc_sw128(b_addr + k * 32)
                                             : sdesc_sw32(b_addr + k * (BT * 32));
           mma_f16(tmem, sdesc_sw128(a_addr + k * 32), bdesc, idesc, (i > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit(empty(s));
+        mma_commit(empty_a(s));
+        mma_commit(empty_b(sb));
       }
       // Signals the epilogue once every issued MMA has completed (also on
       // abort, so nothing is in flight when TMEM is freed).
@@ -809,8 +821,8 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         if (lane == 0) mbar_arrive(empty_l(ps));
       }
       const int s = i % ST;
-      if (!mbar_wait(empty(s), ((i / ST) & 1) ^ 1, abort_flag)) break;
-      uint8_t* a_row = ring + s * S::kStageBytes + r * 128;
+      if (!mbar_wait(empty_a(s), ((i / ST) & 1) ^ 1, abort_flag)) break;
+      uint8_t* a_row = ring_a + s * S::kABytes + r * 128;
       if (row_ok) {
         dequant_stage<T, BITS, FP4>(pk, sb, fp4_g16, a_row, r, tail);
       } else {
