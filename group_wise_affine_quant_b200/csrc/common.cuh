@@ -112,6 +112,9 @@ struct QmmPlan {
   int k_tiles;     // K / 64 rounded up
   int k_tiles_split;
   int splits;      // K-slices, one cluster per output tile
+  int64_t tiles_main;     // tiles launched with `splits` slices (the rest: tail)
+  int tail_splits;        // K-slices of each remaining tile
+  int tail_k_tiles_split;
 };
 QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode);
 cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const void* scales,

@@ -48,13 +48,8 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
   p.bt = bt;
   p.n_tiles = (int64_t)ntg * groups;
   p.m_tiles = (M + bt - 1) / bt;
-  int splits = 1;
-  const int64_t tiles = p.n_tiles * p.m_tiles;
-  while (splits < 8 && tiles * splits * 2 <= sms && k_tiles / (splits * 2) >= 2) splits *= 2;
-  p.k_tiles_split = (int)((k_tiles + splits - 1) / splits);
-  if (bits & 1) p.k_tiles_split += p.k_tiles_split & 1;
-  p.splits = (int)((k_tiles + p.k_tiles_split - 1) / p.k_tiles_split);
   p.k_tiles = (int)k_tiles;
+  plan_splits(p, bits, sms);
 
   QmmMaps maps;
   memset(&maps, 0, sizeof(maps));

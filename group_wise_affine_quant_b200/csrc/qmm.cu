@@ -24,17 +24,9 @@ QmmPlan plan_qmm(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
   p.bt = bt;
   p.n_tiles = n_tiles;
   p.m_tiles = (M + bt - 1) / bt;
-  // Split K over up to 8 CTAs of a cluster while the tiles underfill the GPU.
-  int splits = 1;
-  const int64_t tiles = p.n_tiles * p.m_tiles;
-  // Light CTAs (bt <= 32) fit two per SM.
-  const int64_t slots = bt <= 32 ? 2 * sms : sms;
-  while (splits < 8 && tiles * splits * 2 <= slots && k_tiles / (splits * 2) >= 2) splits *= 2;
-  p.k_tiles_split = (int)((k_tiles + splits - 1) / splits);
-  // a K-slice must start on a 16-byte boundary of the packed rows
-  if (bits & 1) p.k_tiles_split += p.k_tiles_split & 1;
-  p.splits = (int)((k_tiles + p.k_tiles_split - 1) / p.k_tiles_split);
   p.k_tiles = (int)k_tiles;
+  // Light CTAs (bt <= 32) fit two per SM.
+  plan_splits(p, bits, bt <= 32 ? 2 * sms : sms);
   return p;
 }
 

@@ -114,11 +114,14 @@ struct QmmArgs {
   int splits;
   int vec;              // widest cp.async (16, 8 or 4 bytes) the packed rows allow
   int64_t row_bytes;
-  // Output columns: tile column block blockIdx.x covers weight rows
-  // g * n_limit + [nt * 128, nt * 128 + 128) with g = blockIdx.x / ntg and
-  // nt = blockIdx.x % ntg; rows at or past n_limit (within the block's group)
-  // are zero.  y[m, g * n_limit + row] at stride ldy.  Dense: one group.
+  // Output tiles are numbered t = tile0 + blockIdx.x; tile t covers x rows
+  // [(t / nt_all) * BT, +BT) and column block c = t % nt_all, which holds
+  // weight rows g * n_limit + [nt * 128, nt * 128 + 128) with g = c / ntg and
+  // nt = c % ntg; rows at or past n_limit (within the block's group) are
+  // zero.  y[m, g * n_limit + row] at stride ldy.  Dense: one group.
   int ldy, n_limit, ntg;
+  int nt_all;           // column blocks over all groups (ntg * groups)
+  int tile0;            // first tile of this launch
   // Implicit-GEMM conv geometry (x is NHWC [Bn, H, W, Cin]; K index =
   // (i * kw + j) * Cg + c over the k_real = kh * kw * Cg real columns).
   int Cin, Cg, H, W, Ho, Wo, kh, kw, sh, sw, ph, pw, k_real;
@@ -443,10 +446,12 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cgrp = blockIdx.x / a.ntg;                    // conv group (0 when dense)
-  const int nl0 = (blockIdx.x - cgrp * a.ntg) * kRowsW;   // first row within the group
+  const int tile = a.tile0 + (int)blockIdx.x;
+  const int cblk = tile % a.nt_all;                       // column block
+  const int cgrp = cblk / a.ntg;                          // conv group (0 when dense)
+  const int nl0 = (cblk - cgrp * a.ntg) * kRowsW;         // first row within the group
   const int n0 = cgrp * a.n_limit + nl0;                  // first weight row
-  const int m0 = blockIdx.y * BT;
+  const int m0 = (tile / a.nt_all) * BT;
   const int split = blockIdx.z;
   const int kt0 = split * a.k_tiles_split;
   const int kt1 = min(a.k_tiles, kt0 + a.k_tiles_split);
@@ -978,21 +983,43 @@ cudaError_t launch_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, c
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_done[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.n_tiles, (unsigned)p.m_tiles, (unsigned)p.splits);
-  cfg.blockDim = dim3(S::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = S::kSmem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = (unsigned)p.splits;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, maps, a);
+  // Part 0: tiles [0, tiles_main) with p.splits K-slices each; part 1 (the
+  // partial last wave, when the plan splits it): the remaining tiles with
+  // p.tail_splits slices each, so they spread over the idle SMs.
+  const int64_t tiles = p.n_tiles * p.m_tiles;
+  for (int part = 0; part < 2; ++part) {
+    QmmArgs ap = a;
+    ap.nt_all = (int)p.n_tiles;
+    int64_t count = tiles;
+    if (part == 0) {
+      count = p.tiles_main;
+      ap.tile0 = 0;
+    } else {
+      count = tiles - p.tiles_main;
+      if (count <= 0) break;
+      ap.tile0 = (int)p.tiles_main;
+      ap.splits = p.tail_splits;
+      ap.k_tiles_split = p.tail_k_tiles_split;
+    }
+    if (count <= 0) continue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)count, 1, (unsigned)ap.splits);
+    cfg.blockDim = dim3(S::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = S::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = (unsigned)ap.splits;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, kern, maps, ap);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <typename T, int BITS, bool FP4, bool FAST, int XMODE>
@@ -1055,6 +1082,40 @@ inline cudaError_t weight_maps(QmmMaps& maps, QmmArgs& a, const void* w_q, const
   if (mode != AQ_MODE_FP4)
     e = make_map(&maps.b, biases, st_t, esz, rows, G, 16 / esz, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE);
   return e;
+}
+
+// K-slice plan for p's tiles (n_tiles, m_tiles, k_tiles set) on `slots`
+// resident CTAs.  Tiles that underfill the GPU split K over a cluster of up
+// to 8; otherwise a last wave that is at most half full is launched apart,
+// its tiles split in 2 or 4, so that it takes a fraction of a tile time on
+// the SMs the full waves leave idle.  A K-slice starts on a 16-byte boundary
+// of the packed rows (an even number of k-tiles for odd bit widths).
+inline int slice_tiles(int64_t k_tiles, int splits, int bits) {
+  int kts = (int)((k_tiles + splits - 1) / splits);
+  if (bits & 1) kts += kts & 1;
+  return kts;
+}
+
+inline void plan_splits(QmmPlan& p, int bits, int64_t slots) {
+  const int64_t tiles = p.n_tiles * p.m_tiles;
+  int splits = 1;
+  while (splits < 8 && tiles * splits * 2 <= slots && p.k_tiles / (splits * 2) >= 2) splits *= 2;
+  p.k_tiles_split = slice_tiles(p.k_tiles, splits, bits);
+  p.splits = (p.k_tiles + p.k_tiles_split - 1) / p.k_tiles_split;
+  p.tiles_main = tiles;
+  p.tail_splits = 1;
+  p.tail_k_tiles_split = p.k_tiles_split;
+  if (p.splits != 1 || tiles <= slots) return;
+  const int64_t rem = tiles % slots;
+  int ts = 1;
+  while (ts < 4 && rem > 0 && rem * ts * 2 <= slots && p.k_tiles / (ts * 2) >= 4) ts *= 2;
+  if (ts == 1) return;
+  const int kts = slice_tiles(p.k_tiles, ts, bits);
+  ts = (p.k_tiles + kts - 1) / kts;
+  if (ts < 2) return;
+  p.tiles_main = tiles - rem;
+  p.tail_splits = ts;
+  p.tail_k_tiles_split = kts;
 }
 
 inline int ilog2i(int v) {

@@ -98,6 +98,28 @@ def test_qmm_split_k_cluster(M, N, K):
     _check(x, wq, s, b, y1, 4, 32, 0)
 
 
+@pytest.mark.parametrize("M,N,K,bits", [
+    (1024, 5120, 1024, 4),       # 160 tiles of 256 x 128: last 12 tiles in 4 K-slices
+    (1024, 5120, 1088, 3),       # odd width, 17 k-tiles: slices of an even k-tile count
+    (16, 44288, 1024, 4),        # light tiles, 346 of them: last 50 in 2 K-slices
+])
+def test_qmm_split_last_wave(M, N, K, bits):
+    """More tiles than resident CTAs with a last wave at most half full: the
+    remaining tiles launch apart with K split over a cluster."""
+    x, wq, s, b = _case(M, N, K, bits, 64, 1, seed=N + K + bits, wstd=0.02)
+    y1 = api.aq_qmm(x, wq, s, b, bits, 64)
+    y2 = api.aq_qmm(x, wq, s, b, bits, 64)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    rng = np.random.default_rng(bits)
+    tail_rows = np.arange(N - 128 * 13, N)          # columns of the tail tiles
+    ms = np.concatenate([[0, M - 1], rng.integers(0, M, 800), rng.integers(max(0, M - 256), M, 400)])
+    ns = np.concatenate([[0, N - 1], rng.integers(0, N, 800), rng.choice(tail_rows, 400)])
+    yr, den = oracle.qmm_sampled(dev_u16(x), dev_u8(wq), dev_u16(s), dev_u16(b), N, bits, 64, 0,
+                                 1, ms, ns, w_in_t=True)
+    check_matmul(dev_u16(y1)[ms, ns], yr, den, 1)
+
+
 @pytest.mark.parametrize("bits", [2, 3, 5, 6])
 def test_qmm_narrow_rows(bits):
     """K % 64 == 32: row strides that are not 16-byte multiples."""
