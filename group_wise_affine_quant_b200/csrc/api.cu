@@ -148,8 +148,12 @@ aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void*
   if (N == 0) return AQ_OK;
   if (K == 0) return zero_output(y, M, N, stream);
   if (M > kQmvSimtMaxM) {
-    // From 3 rows of x on, the tensor-core kernel streams the weight faster
+    // From 3 rows of x on, the tensor-core kernels stream the weight faster
     // than fp32 FMAs can consume it (each code costs M FMAs on CUDA cores).
+    if (aq::qmv_tc_applies(M, N, K, bits, group_size, mode, scales, biases))
+      return cuda_status(aq::launch_qmv_tc(x, w_q, scales, biases, y, M, N, K, bits, group_size,
+                                           mode, dtype, (cudaStream_t)stream),
+                         "aq_qmv launch");
     const aq::QmmPlan p = aq::plan_qmm(M, N, K, bits, group_size, mode);
     return cuda_status(aq::launch_qmm(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
                                       mode, dtype, (cudaStream_t)stream),
@@ -182,7 +186,9 @@ unsigned aq_device_errors(void) {
   unsigned v = 0, w = 0;
   if (aq::read_device_error_qmm(&v) != cudaSuccess) return 0xFFFFFFFFu;
   if (aq::read_device_error_conv(&w) != cudaSuccess) return 0xFFFFFFFFu;
-  return v | w;
+  unsigned t = 0;
+  if (aq::read_device_error_qmv_tc(&t) != cudaSuccess) return 0xFFFFFFFFu;
+  return v | w | t;
 }
 
 aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* scales,

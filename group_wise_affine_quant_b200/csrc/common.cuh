@@ -125,6 +125,14 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
                          int sh, int sw, int ph, int pw, int groups, int bits, int gs, int dtype,
                          cudaStream_t st);
 cudaError_t read_device_error_qmm(unsigned* out);
+// Tensor-core decode path for 1 <= M <= 16 (qmv_tc.cu): applies when the
+// packed rows and the scale rows are 16-byte multiples (TMA chunks).
+bool qmv_tc_applies(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode,
+                    const void* scales, const void* biases);
+cudaError_t launch_qmv_tc(const void* x, const void* w_q, const void* scales, const void* biases,
+                          void* y, int64_t M, int64_t N, int64_t K, int bits, int gs, int mode,
+                          int dtype, cudaStream_t st);
+cudaError_t read_device_error_qmv_tc(unsigned* out);
 // aq_set_weight_prefetch's process-wide setting (0 or 1).
 int weight_prefetch_enabled();
 cudaError_t read_device_error_conv(unsigned* out);
