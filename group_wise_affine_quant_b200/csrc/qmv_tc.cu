@@ -39,7 +39,6 @@ struct DecShape {
   // A stage is 128 K-columns (two 64-column k-tiles).  Dequantized weight
   // stages live in TMEM: 64 columns each (two 16-bit values per lane and
   // column); the accumulator takes columns 0-15.
-  static constexpr int kKS = 2 * kBK;
   static constexpr int kAStages = 3;
   static constexpr int kACol0 = 32;
   static constexpr int kTmemCols = 256;
@@ -53,13 +52,14 @@ struct DecShape {
   static constexpr int kWOff = 0;
   static constexpr int kXOff = kWOff + kWSlots * kWChunk;
   static constexpr int kSOff = kXOff + kXStages * kXBytes;
-  static constexpr int kDataBytes = kSOff + kSSlots * kSChunk;
-  // full/empty pairs for the four rings, then acc_full, red_full, go
-  static constexpr int kBars = 2 * (kAStages + kWSlots + kXStages + kSSlots) + 3;
+  // split-K: the partials this slice receives for the rows it owns, from
+  // every other slice: (slices - 1) x ceil(128 / slices) rows x M fp32
+  static constexpr int kRecvOff = kSOff + kSSlots * kSChunk;
+  static constexpr int kRecvBytes = 8 * 1024;
+  static constexpr int kDataBytes = kRecvOff + kRecvBytes;
+  // full/empty pairs for the four rings, then acc_full, recv_full
+  static constexpr int kBars = 2 * (kAStages + kWSlots + kXStages + kSSlots) + 2;
   static constexpr int kSmem = 1024 + kDataBytes + 512;
-  // split-K partials parked in the leader: (slices - 1) x 128 rows x 16 fp32
-  static constexpr int kMaxRedBytes = 7 * kRowsW * 16 * 4;
-  static_assert(kMaxRedBytes <= kDataBytes, "partials overlay the rings");
   static_assert(kBars * 8 + 16 <= 512, "barrier area");
   static_assert(kACol0 + 64 * kAStages <= kTmemCols, "TMEM columns");
 };
@@ -142,7 +142,7 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
   uint8_t* wring = smem + S::kWOff;
   uint8_t* xring = smem + S::kXOff;
   uint8_t* sring = smem + S::kSOff;
-  float* red = reinterpret_cast<float*>(smem);            // leader: [splits-1][128][mp]
+  float* recv = reinterpret_cast<float*>(smem + S::kRecvOff);  // [splits-1][rows owned][mp]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kDataBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -157,8 +157,7 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
   auto full_s = [&](int s) { return bar(2 * (AS + WS + XS) + s); };
   auto empty_s = [&](int s) { return bar(2 * (AS + WS + XS) + SS + s); };
   const uint32_t acc_full = bar(2 * (AS + WS + XS + SS));
-  const uint32_t red_full = acc_full + 8;
-  const uint32_t go = acc_full + 16;
+  const uint32_t recv_full = acc_full + 8;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kRowsW;
@@ -168,6 +167,10 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
   const int nkt = kt1 - kt0;                              // >= 1 (host plan)
   const int nst = (nkt + 1) >> 1;                         // 128-column stages
   const bool clustered = a.splits > 1;
+  // split-K: slice `split` owns rows [split * rpo, +rpo) of the tile and
+  // receives those rows' partials from every other slice
+  const int rpo = (kRowsW + a.splits - 1) / a.splits;
+  const int own0 = min(kRowsW, split * rpo), own1 = min(kRowsW, own0 + rpo);
   // weight chunk c covers bytes [wb0 + 128 c, +128) of every row; scale chunk
   // j covers groups [SGC (sc0 + j), +SGC)
   const int wb0 = kt0 * kPB;                              // 16-byte aligned (host plan)
@@ -203,18 +206,17 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
   };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < AS; ++s) { mbar_init(full_a(s), S::kDqWarps); mbar_init(empty_a(s), 1); }
+    for (int s = 0; s < AS; ++s) { mbar_init(full_a(s), 4); mbar_init(empty_a(s), 1); }
     for (int s = 0; s < WS; ++s) { mbar_init(full_w(s), 1); mbar_init(empty_w(s), S::kDqWarps); }
     for (int s = 0; s < XS; ++s) { mbar_init(full_x(s), 1); mbar_init(empty_x(s), 1); }
     for (int s = 0; s < SS; ++s) { mbar_init(full_s(s), 1); mbar_init(empty_s(s), S::kDqWarps); }
     mbar_init(acc_full, 1);
-    mbar_init(red_full, 1);
-    mbar_init(go, 1);
+    mbar_init(recv_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // the leader expects every other slice's partial before it reduces
-    if (clustered && split == 0)
-      mbar_arrive_expect_tx(red_full, (uint32_t)((a.splits - 1) * kRowsW * a.mp * 4));
+    // every other slice sends the owned rows' partials before this one adds
+    if (clustered)
+      mbar_arrive_expect_tx(recv_full, (uint32_t)((a.splits - 1) * (own1 - own0) * a.mp * 4));
     prefetch_tensormap(&maps.w);
     prefetch_tensormap(&maps.s);
     if constexpr (!FP4) prefetch_tensormap(&maps.b);
@@ -275,17 +277,46 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
     }
   } else {
     // ------------------------------------------------------- dequantizers
-    const int d = warp - S::kWarpDq0;                     // 0 .. 7
-    const int h = d >> 2;                                 // k-tile of the stage
+    // Two groups of four warps take alternate stages; a thread owns one
+    // weight row (its TMEM lane) and both k-tiles of the stage.
+    const int gq = (warp - S::kWarpDq0) >> 2;            // dequantizer group
     const int q = warp & 3;                               // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;                          // weight row in the tile = TMEM lane
     const bool fp4_g16 = FP4 && a.gs_log2 == 4;
     int w_ready = 0, w_freed = 0, s_ready = 0, s_freed = 0;
+    // Release weight chunks below w_done and scale chunks below s_done in
+    // the loader's K order (weight chunk first on a tie), waiting for each
+    // chunk's data first: every group releases every chunk, and the wait
+    // keeps this group's arrivals on the slot's current phase.
+    auto release_upto = [&](int w_done, int s_done) -> bool {
+      bool okr = true;
+      while (okr && (w_freed < w_done || s_freed < s_done)) {
+        const int64_t kw = w_freed < w_done ? (int64_t)w_freed * 128 * 8 / BITS : INT64_MAX;
+        const int64_t ks = s_freed < s_done
+                               ? (int64_t)(sc0 + s_freed) * SGC * (1 << a.gs_log2) - (int64_t)kt0 * kBK
+                               : INT64_MAX;
+        if (kw <= ks) {
+          if (w_freed >= w_ready) {
+            okr = mbar_wait(full_w(w_freed % WS), (w_freed / WS) & 1, abort_flag);
+            w_ready = w_freed + 1;
+          }
+          __syncwarp();
+          if (okr && lane == 0) mbar_arrive(empty_w(w_freed % WS));
+          ++w_freed;
+        } else {
+          if (s_freed >= s_ready) {
+            okr = mbar_wait(full_s(s_freed % SS), (s_freed / SS) & 1, abort_flag);
+            s_ready = s_freed + 1;
+          }
+          __syncwarp();
+          if (okr && lane == 0) mbar_arrive(empty_s(s_freed % SS));
+          ++s_freed;
+        }
+      }
+      return okr;
+    };
     bool ok = true;
-    for (int j = 0; j < nst && ok; ++j) {
-      const int kt = kt0 + 2 * j + h;                     // this warp's k-tile
-      const bool valid = 2 * j + h < nkt;
-      const bool tail = (kt + 1) * kBK > a.K;
+    for (int j = gq; j < nst && ok; j += 2) {
       const int st_end = min(2 * j + 2, nkt) * kPB;       // stage bytes end (slice-relative)
       const int c_hi = (st_end - 1) >> 7;                 // last chunk the stage touches
       for (; w_ready <= c_hi && ok; ++w_ready)
@@ -295,119 +326,113 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
         ok = mbar_wait(full_s(s_ready % SS), (s_ready / SS) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);                    // warp-uniform before the collectives
       if (!ok) break;
-      Packed<BITS> pk;
-      StageSB sb;
-      if (valid) {
-        load_row<BITS, WS>(pk, wring, (2 * j + h) * kPB, r);
-        const uint8_t* sslot = sring + ((s_ready - 1) % SS) * S::kSChunk;
-        const int g0 = (kt * kBK) >> a.gs_log2;
-        const int g1 = tail ? g0 : ((kt * kBK + 32) >> a.gs_log2);
-        if constexpr (FP4) {
-          const uint8_t* sp = sslot + r * 16;
-          const int gs = 1 << a.gs_log2;
-          auto sc = [&](int g) { return splat(TT<T>::from_f(fp4_scale_t<T>(sp[g % SGC], gs))); };
-          if (fp4_g16) {
-            sb.s[0] = sc(g0); sb.s[1] = sc(g0 + 1);
-            sb.b[0] = tail ? sb.s[0] : sc(g0 + 2);
-            sb.b[1] = tail ? sb.s[0] : sc(g0 + 3);
-          } else {
-            sb.s[0] = sc(g0); sb.s[1] = sc(g1); sb.b[0] = sb.b[1] = 0u;
-          }
-        } else {
-          const uint16_t* sp = reinterpret_cast<const uint16_t*>(sslot + r * 16);
-          const uint16_t* bp = reinterpret_cast<const uint16_t*>(sslot + kRowsW * 16 + r * 16);
-          const uint32_t s0 = sp[g0 % SGC], s1 = sp[g1 % SGC];
-          const uint32_t b0 = bp[g0 % SGC], b1 = bp[g1 % SGC];
-          sb.s[0] = s0 | (s0 << 16); sb.s[1] = s1 | (s1 << 16);
-          sb.b[0] = b0 | (b0 << 16); sb.b[1] = b1 | (b1 << 16);
-        }
-      }
-      // release the chunks no later stage reads (all of them after the last)
-      const bool last = j + 1 == nst;
+      const uint8_t* sslot = sring + ((s_ready - 1) % SS) * S::kSChunk;
+      // chunks that end with this stage are released once read (a slot is
+      // refilled only after all eight warps have released it)
+      const bool last = j + 2 >= nst;
       const int w_done = last ? nwc : (((2 * j + 2) * kPB) >> 7);
       const int s_done = last ? nsc : (((((kt0 + 2 * j + 2) * kBK) >> a.gs_log2) / SGC) - sc0);
-      __syncwarp();
-      for (; w_freed < w_done; ++w_freed) {
-        if (w_freed >= w_ready) {                         // a chunk no stage read
-          ok = ok && mbar_wait(full_w(w_freed % WS), (w_freed / WS) & 1, abort_flag);
-          w_ready = w_freed + 1;
-        }
-        if (lane == 0) mbar_arrive(empty_w(w_freed % WS));
-      }
-      for (; s_freed < s_done; ++s_freed) {
-        if (s_freed >= s_ready) {
-          ok = ok && mbar_wait(full_s(s_freed % SS), (s_freed / SS) & 1, abort_flag);
-          s_ready = s_freed + 1;
-        }
-        if (lane == 0) mbar_arrive(empty_s(s_freed % SS));
-      }
       const int s = j % AS;
       ok = __all_sync(0xffffffffu, ok && mbar_wait(empty_a(s), ((j / AS) & 1) ^ 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t o[32];
-      if (valid) {
-        dequant_row<T, BITS, FP4>(pk, sb, fp4_g16, tail, o);
-      } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) o[c] = 0u;
+      for (int h = 0; h < 2; ++h) {
+        const int kt = kt0 + 2 * j + h;
+        const bool tail = (kt + 1) * kBK > a.K;
+        uint32_t o[32];
+        if (2 * j + h < nkt) {
+          Packed<BITS> pk;
+          StageSB sb;
+          load_row<BITS, WS>(pk, wring, (2 * j + h) * kPB, r);
+          const int g0 = (kt * kBK) >> a.gs_log2;
+          const int g1 = tail ? g0 : ((kt * kBK + 32) >> a.gs_log2);
+          if constexpr (FP4) {
+            const uint8_t* sp = sslot + r * 16;
+            const int gs = 1 << a.gs_log2;
+            auto sc = [&](int g) { return splat(TT<T>::from_f(fp4_scale_t<T>(sp[g % SGC], gs))); };
+            if (fp4_g16) {
+              sb.s[0] = sc(g0); sb.s[1] = sc(g0 + 1);
+              sb.b[0] = tail ? sb.s[0] : sc(g0 + 2);
+              sb.b[1] = tail ? sb.s[0] : sc(g0 + 3);
+            } else {
+              sb.s[0] = sc(g0); sb.s[1] = sc(g1); sb.b[0] = sb.b[1] = 0u;
+            }
+          } else {
+            const uint16_t* sp = reinterpret_cast<const uint16_t*>(sslot + r * 16);
+            const uint16_t* bp = reinterpret_cast<const uint16_t*>(sslot + kRowsW * 16 + r * 16);
+            const uint32_t s0 = sp[g0 % SGC], s1 = sp[g1 % SGC];
+            const uint32_t b0 = bp[g0 % SGC], b1 = bp[g1 % SGC];
+            sb.s[0] = s0 | (s0 << 16); sb.s[1] = s1 | (s1 << 16);
+            sb.b[0] = b0 | (b0 << 16); sb.b[1] = b1 | (b1 << 16);
+          }
+          dequant_row<T, BITS, FP4>(pk, sb, fp4_g16, tail, o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        tmem_st_32(tmem + ((uint32_t)(q * 32) << 16) + S::kACol0 + 64 * s + 32 * h, o);
       }
-      tmem_st_32(tmem + ((uint32_t)(q * 32) << 16) + S::kACol0 + 64 * s + 32 * h, o);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(full_a(s));
+      // after the hand-over: a release may wait for chunks that the other
+      // group's next stage frees, which needs this stage's MMAs to run
+      ok = release_upto(w_done, s_done);
     }
+    // chunks past this group's last stage are released too
+    if (!*abort_flag) release_upto(nwc, nsc);
 
     // ------------------------------------------------------- epilogue
-    if (d < 4) {
-      const int rr = r;
+    if (gq == 0) {
       const bool acc_ok = mbar_wait(acc_full, 0, abort_flag, 4000000000ull);
       tc_fence_after();
       uint32_t v[16];
       tmem_ld_16(tmem + ((uint32_t)(q * 32) << 16), v);
       tmem_ld_wait();
-      const bool row_ok = n0 + rr < a.N;
-      if (acc_ok && !*abort_flag) {
-        if (clustered && split != 0) {
-          // wait for the leader's go, then push this slice's partial
-          cluster_wait();
-          if (mbar_wait_cluster(go, 0, abort_flag)) {
-            const uint32_t base = smem_u32(red + ((split - 1) * kRowsW + rr) * a.mp);
-            const uint32_t rbase = mapa_shared(base, 0);
-            const uint32_t rbar = mapa_shared(red_full, 0);
+      const bool live = acc_ok && !*abort_flag;
+      const int owner = clustered ? r / rpo : split;
+      if (clustered) cluster_wait();                      // every slice's barriers are initialised
+      if (live && owner != split) {
+        // send this row's partial to the slice that owns it
+        const int slot = split < owner ? split : split - 1;
+        const uint32_t dst = smem_u32(recv + (slot * rpo + (r - owner * rpo)) * a.mp);
+        const uint32_t rdst = mapa_shared(dst, (uint32_t)owner);
+        const uint32_t rbar = mapa_shared(recv_full, (uint32_t)owner);
 #pragma unroll
-            for (int t = 0; t < 16; t += 4)
-              if (t < a.mp) st_async_v4(rbase + 4 * t, v[t], v[t + 1], v[t + 2], v[t + 3], rbar);
-          }
-        } else {
-          float acc[16];
+        for (int t = 0; t < 16; t += 4)
+          if (t < a.mp) st_async_v4(rdst + 4 * t, v[t], v[t + 1], v[t + 2], v[t + 3], rbar);
+      }
+      // every lane of the warp has sent before any lane waits: a waiting
+      // lane must not hold back a sibling whose partial another slice awaits
+      __syncwarp();
+      if (live && owner == split) {
+        // an owned row: add every slice's partial in slice order
+        float acc[16];
 #pragma unroll
-          for (int t = 0; t < 16; ++t) acc[t] = __uint_as_float(v[t]);
-          bool have = true;
-          if (clustered) {
-            // leader: release the other slices, then add their partials in
-            // rank order once every byte has landed
-            cluster_wait();
-            __syncwarp();
-            if (rr < a.splits - 1) mbar_arrive_remote(mapa_shared(go, rr + 1));
-            have = mbar_wait_cluster(red_full, 0, abort_flag, 4000000000ull);
-            if (have) {
-              for (int j = 0; j < a.splits - 1; ++j) {
-                const float* pr = red + (j * kRowsW + rr) * a.mp;
+        for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+        bool have = true;
+        if (clustered) have = mbar_wait_cluster(recv_full, 0, abort_flag, 4000000000ull);
+        if (have) {
+          for (int k = 0; k < a.splits; ++k) {
+            if (k == split) {
 #pragma unroll
-                for (int t = 0; t < 16; t += 4) {
-                  if (t < a.mp) {
-                    const float4 p4 = *reinterpret_cast<const float4*>(pr + t);
-                    acc[t] += p4.x; acc[t + 1] += p4.y; acc[t + 2] += p4.z; acc[t + 3] += p4.w;
-                  }
+              for (int t = 0; t < 16; ++t) acc[t] += __uint_as_float(v[t]);
+            } else {
+              const float* pr = recv + ((k < split ? k : k - 1) * rpo + (r - own0)) * a.mp;
+#pragma unroll
+              for (int t = 0; t < 16; t += 4) {
+                if (t < a.mp) {
+                  const float4 p4 = *reinterpret_cast<const float4*>(pr + t);
+                  acc[t] += p4.x; acc[t + 1] += p4.y; acc[t + 2] += p4.z; acc[t + 3] += p4.w;
                 }
               }
             }
           }
           pdl_wait();                                     // before y is written
-          if (have && row_ok) {
-            T* yp = reinterpret_cast<T*>(a.y) + n0 + rr;
+          if (n0 + r < a.N) {
+            T* yp = reinterpret_cast<T*>(a.y) + n0 + r;
 #pragma unroll
             for (int t = 0; t < 16; ++t)
               if (t < a.M) yp[(int64_t)t * a.N] = TT<T>::from_f(acc[t]);
