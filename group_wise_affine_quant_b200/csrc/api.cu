@@ -147,13 +147,16 @@ aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void*
   if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
   if (N == 0) return AQ_OK;
   if (K == 0) return zero_output(y, M, N, stream);
+  // The tensor-core decode kernel dequantizes each code once for all rows of
+  // x and costs fewer instructions per code than fp32 FMAs even for one row;
+  // it takes every shape whose packed rows and scale rows are 16-byte
+  // multiples.  Other shapes: the fp32 kernel for one or two rows, the
+  // general tensor-core kernel beyond.
+  if (aq::qmv_tc_applies(M, N, K, bits, group_size, mode, scales, biases))
+    return cuda_status(aq::launch_qmv_tc(x, w_q, scales, biases, y, M, N, K, bits, group_size,
+                                         mode, dtype, (cudaStream_t)stream),
+                       "aq_qmv launch");
   if (M > kQmvSimtMaxM) {
-    // From 3 rows of x on, the tensor-core kernels stream the weight faster
-    // than fp32 FMAs can consume it (each code costs M FMAs on CUDA cores).
-    if (aq::qmv_tc_applies(M, N, K, bits, group_size, mode, scales, biases))
-      return cuda_status(aq::launch_qmv_tc(x, w_q, scales, biases, y, M, N, K, bits, group_size,
-                                           mode, dtype, (cudaStream_t)stream),
-                         "aq_qmv launch");
     const aq::QmmPlan p = aq::plan_qmm(M, N, K, bits, group_size, mode);
     return cuda_status(aq::launch_qmm(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
                                       mode, dtype, (cudaStream_t)stream),

@@ -110,12 +110,16 @@ AQ_API aq_status aq_dequantize(const void* w_q, const void* scales, const void* 
 /*
  * aq_qmv — y = x . w_hat^T for small M (1 <= M <= 16): the weight-streaming
  * path ("Add the 3bit packed qmm_t", affine_packed_qmv_fast, routed for few
- * rows of x).  x [M, K] T, y [M, N] T, fp32 accumulation.  For M <= 2 an
- * fp32 CUDA-core kernel with the scale and bias hoisted out of each group's
- * dot product (w_hat never rounded); for M >= 3 the tensor-core kernel of
- * aq_qmm, which reads the weight once for all rows of x.  K-slices are
- * reduced inside a thread block cluster, so no workspace is needed
- * (aq_workspace_size returns 0; workspace may be NULL and is not touched).
+ * rows of x).  x [M, K] T, y [M, N] T, fp32 accumulation.  When the
+ * packed rows (K * bits / 8 bytes) and the rows of scales (K / group_size
+ * elements) are 16-byte multiples and scales / biases are 16-byte aligned, a
+ * tensor-core decode kernel: each code is dequantized once into T (the value
+ * aq_dequantize writes) in tensor memory and multiplied with all rows of x.
+ * Other shapes: for M <= 2 an fp32 CUDA-core kernel with the scale and bias
+ * hoisted out of each group's dot product (w_hat never rounded), for M >= 3
+ * the tensor-core kernel of aq_qmm.  K-slices are reduced inside a thread
+ * block cluster, so no workspace is needed (aq_workspace_size returns 0;
+ * workspace may be NULL and is not touched).
  * Returns AQ_ERR_INVALID_ARG for M outside 1..16.
  */
 AQ_API aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void* biases,

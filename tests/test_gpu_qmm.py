@@ -190,7 +190,7 @@ def test_qmm_matches_qmv_small_m():
     y2 = api.aq_qmv(x, wq, s, b, 4, 64)
     torch.cuda.synchronize()
     _check(x, wq, s, b, y1, 4, 64, 1)
-    _check(x, wq, s, b, y2, 4, 64, 1, w_in_t=False)    # qmv keeps w_hat in fp32
+    _check(x, wq, s, b, y2, 4, 64, 1)
 
 
 @pytest.mark.parametrize("prefetch", [False, True])

@@ -1,9 +1,10 @@
 """GPU parity for aq_qmv against the oracle, within
 |y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref).
 
-aq_qmv keeps w_hat in fp32 for M <= 2 (checked against the exact product) and
-hands M >= 3 to the tensor-core kernel, which multiplies T-valued weight tiles
-(checked against the product over w_hat rounded to T)."""
+aq_qmv's tensor-core kernels multiply weight tiles rounded to T (checked
+against the product over w_hat rounded to T); its fp32 kernel, used for M <= 2
+on shapes the tensor-core decode kernel does not take, keeps w_hat in fp32
+(checked against the exact product)."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +12,7 @@ import torch
 import oracle
 from group_wise_affine_quant_b200 import api, inputs
 from tests.gpu_util import DEV, TDT, dev_u16, dev_u8, to_dev
-from tests.util import check_matmul
+from tests.util import check_matmul, qmv_w_in_t
 
 pytestmark = pytest.mark.gpu
 
@@ -30,8 +31,9 @@ def _check(x, wq, s, b, y, bits, gs, dt, mode=0, **kw):
     N = wq.shape[0]
     sc = dev_u8(s) if mode == 1 else dev_u16(s)
     bi = None if b is None else dev_u16(b)
+    M, K = x.shape
     yr, den = oracle.qmm(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt,
-                         w_in_t=x.shape[0] > 2)
+                         w_in_t=qmv_w_in_t(M, K, bits, gs, mode))
     return check_matmul(dev_u16(y), yr, den, dt, **kw)
 
 
@@ -58,11 +60,14 @@ def test_qmv_ragged_and_split_k(bits, K):
     _check(x, wq, s, b, y, bits, gs, 1)
 
 
-@pytest.mark.parametrize("M", [1, 16])
-def test_qmv_split_k_twice_in_a_row(M):
-    """Long K splits over a cluster of CTAs; two calls give identical results."""
+@pytest.mark.parametrize("M", [1, 2, 16])
+@pytest.mark.parametrize("K", [8192, 8192 + 64])
+def test_qmv_split_k_twice_in_a_row(M, K):
+    """Long K splits over a cluster of CTAs; two calls give identical results
+    (K = 8256 gives rows of scales that are not 16-byte multiples: the fp32
+    kernel for M <= 2)."""
     bits, gs, dt = 4, 64, 1
-    x, wq, s, b = _case(M, 512, 8192, bits, gs, dt, seed=5)
+    x, wq, s, b = _case(M, 512, K, bits, gs, dt, seed=5)
     y1 = api.aq_qmv(x, wq, s, b, bits, gs)
     y2 = api.aq_qmv(x, wq, s, b, bits, gs)
     torch.cuda.synchronize()
@@ -71,10 +76,12 @@ def test_qmv_split_k_twice_in_a_row(M):
 
 
 @pytest.mark.parametrize("M", [1, 3, 16])
-def test_qmv_very_long_k_chunked(M):
-    """K beyond one shared-memory chunk per slice (x staged in chunks)."""
+@pytest.mark.parametrize("K", [65536, 65536 + 128])
+def test_qmv_very_long_k_chunked(M, K):
+    """Very long K: 64 stages per slice on the tensor-core decode kernel
+    (K = 65536), x staged in chunks on the other kernels (K = 65664)."""
     bits, gs, dt = 4, 128, 0
-    x, wq, s, b = _case(M, 40, 65536 + 128, bits, gs, dt, seed=9, wstd=0.01)
+    x, wq, s, b = _case(M, 40, K, bits, gs, dt, seed=9, wstd=0.01)
     y = api.aq_qmv(x, wq, s, b, bits, gs)
     torch.cuda.synchronize()
     _check(x, wq, s, b, y, bits, gs, dt)

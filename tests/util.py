@@ -87,3 +87,13 @@ def check_matmul(y_t_u16, y_ref, den, dt, rel=REL_TOL, what="y", overflow_any_no
             % (what, len(bad), ok.size, rel, i, y[i], y_ref[i], den[i]))
     err = np.abs(np.where(fin, y, 0) - y_ref) / np.maximum(tol, 1e-300)
     return float(np.max(np.where(fin, err, 0)))
+
+
+def qmv_w_in_t(M, K, bits, gs, mode=0):
+    """Which w_hat aq_qmv multiplies: the tensor-core decode kernel (taken
+    whenever the packed rows and the rows of scales are 16-byte multiples)
+    and the tensor-core fallback for M >= 3 multiply weight tiles rounded to
+    T; only the fp32 kernel (M <= 2, other shapes) keeps w_hat in fp32."""
+    esz = 1 if mode == 1 else 2
+    tc = (K * bits // 8) % 16 == 0 and (K // gs * esz) % 16 == 0
+    return tc or M > 2
