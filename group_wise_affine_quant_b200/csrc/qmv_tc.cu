@@ -391,6 +391,9 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
       uint32_t v[16];
       tmem_ld_16(tmem + ((uint32_t)(q * 32) << 16), v);
       tmem_ld_wait();
+      // the accumulator is in registers: the MMA warp may free TMEM now
+      tc_fence_before();
+      named_barrier_arrive(1, 32 * 5);
       const bool live = acc_ok && !*abort_flag;
       const int owner = clustered ? r / rpo : split;
       if (clustered) cluster_wait();                      // every slice's barriers are initialised
@@ -415,7 +418,9 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
         bool have = true;
         if (clustered) have = mbar_wait_cluster(recv_full, 0, abort_flag, 4000000000ull);
         if (have) {
-          for (int k = 0; k < a.splits; ++k) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if (k >= a.splits) break;
             if (k == split) {
 #pragma unroll
               for (int t = 0; t < 16; ++t) acc[t] += __uint_as_float(v[t]);
@@ -442,13 +447,15 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
     }
   }
 
-  tc_fence_before();
-  __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) atomicOr(&g_aq_device_error, 1u);
   if (warp == S::kWarpMma) {
+    // every tcgen05 operation has completed (acc_full) and the epilogue warps
+    // have read the accumulator
+    named_barrier_sync(1, 32 * 5);
     tc_fence_after();
     tmem_dealloc(tmem, S::kTmemCols);
   }
+  __syncwarp();
+  if (lane == 0 && *abort_flag) atomicOr(&g_aq_device_error, 1u);
 }
 
 template <typename T, int BITS, bool FP4>

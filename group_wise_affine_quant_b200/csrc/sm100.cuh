@@ -96,6 +96,16 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
+// ------------------------------------------------------------ named barriers
+// Barrier `id` (1..15) over `count` threads (a multiple of 32); arrive does
+// not wait.  Non-aligned forms: the threads of a warp may come separately.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t count) {
+  asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------------ thread block cluster
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
