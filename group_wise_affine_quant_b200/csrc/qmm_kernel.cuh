@@ -63,13 +63,14 @@ struct QmmShape {
   // CTAs fit on an SM: the next kernel of a stream can then start streaming
   // its weights while this one finishes.  Larger tiles use a deeper pipeline.
   static constexpr bool kLight = BT <= 32;
-  // Operand rings: kStages slots of dequantized A (the dequantizers refill
-  // them from shared memory, no memory latency to hide) and kBStages slots of
-  // x tiles (TMA from L2/HBM; one more slot at BT = 256, where the MMA stage
-  // is shortest relative to a TMA round trip).
-  static constexpr int kStages = kLight ? 3 : BT >= 256 ? 3 : 4;
-  static constexpr int kBStages = BT >= 256 ? 4 : kStages;
-  static constexpr int kABytes = kRowsW * kBK * 2;                   // 16 KB
+  // Operand rings: kStages slots of dequantized A in tensor memory (the
+  // dequantizers refill them from shared memory, no memory latency to hide;
+  // the MMA reads A from TMEM, which keeps the A tile out of the shared-memory
+  // bandwidth) and kBStages slots of x tiles in shared memory (TMA from
+  // L2/HBM; one more slot at BT = 256, where the MMA stage is shortest
+  // relative to a TMA round trip).
+  static constexpr int kStages = kLight ? 3 : 4;
+  static constexpr int kBStages = 4;
   static constexpr int kBBytes = BT * kBK * 2;                       // BT * 128
   static constexpr int kPB = 8 * BITS;                               // packed bytes / row / stage
   // cp.async path: one slot per stage, rows at a bank-spreading pitch.
@@ -84,10 +85,15 @@ struct QmmShape {
   static constexpr int kSSlots = kLight ? 2 : 4;
   static constexpr int kLoadBytes = FAST ? kWSlots * kWChunk + kSSlots * kSChunk : kPStages * kPSlot;
   static constexpr int kRedBytes = BT * kRowsW * 4;                  // split-K parking
-  static constexpr int kRingBytes = kStages * kABytes + kBStages * kBBytes;
+  static constexpr int kRingBytes = kBStages * kBBytes;
   static constexpr int kOpBytes = kRingBytes > kRedBytes ? kRingBytes : kRedBytes;
   static constexpr int kDataBytes = kOpBytes + kLoadBytes;
-  static constexpr int kTmemCols = BT < 32 ? 32 : BT;
+  // TMEM: the fp32 accumulator in columns [0, kACol0), then kStages A
+  // stages of 32 columns (64 16-bit values per lane).
+  static constexpr int kACol0 = BT < 32 ? 32 : BT;
+  static constexpr int kTmemNeed = kACol0 + 32 * kStages;
+  static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
+                                   : kTmemNeed <= 256 ? 256 : 512;
   // Dequantizer groups: group g takes K-stages i with i % kGroups == g.  A
   // group's consecutive stages are kGroups apart and its operand-slot wait
   // is a phase-parity wait, which is unambiguous only while the slot's
@@ -364,16 +370,15 @@ __device__ __forceinline__ StageSB sb_from_words(const uint4 wv, const QmmArgs& 
   return r;
 }
 
+// Dequantize one weight row of a K-stage (64 codes) into 32 words (T pairs
+// in K order), the layout of an A operand in tensor memory: lane = row, two
+// 16-bit values per column.  With `tail` the upper 32 columns are zero.
 template <typename T, int BITS, bool FP4>
-__device__ __forceinline__ void dequant_stage(const Packed<BITS>& p, const StageSB& sb, bool fp4_g16,
-                                              uint8_t* a_row, int r, bool tail) {
-  // chunk c of 8 elements lands at 16-byte slot c ^ (r & 7) of the row
-  const int sw = r & 7;
-  auto put = [&](int c, uint4 v) {
-    *reinterpret_cast<uint4*>(a_row + ((c ^ sw) << 4)) = v;
-  };
+__device__ __forceinline__ void dequant_row(const Packed<BITS>& p, const StageSB& sb, bool fp4_g16,
+                                            bool tail, uint32_t (&o)[32]) {
+  auto put = [&](int c, uint4 v) { o[4 * c] = v.x; o[4 * c + 1] = v.y; o[4 * c + 2] = v.z; o[4 * c + 3] = v.w; };
   if constexpr (FP4) {
-    // quarters of 16 elements: scales s0 s1 (g16: b0 b1 hold quarters 2, 3)
+    // quarters of 16 elements: scales s0 s1 (group 16: b0 b1 hold quarters 2, 3)
     const uint32_t q0 = sb.s[0];
     const uint32_t q1 = fp4_g16 ? sb.s[1] : sb.s[0];
     const uint32_t q2 = fp4_g16 ? sb.b[0] : sb.s[1];
@@ -382,27 +387,23 @@ __device__ __forceinline__ void dequant_stage(const Packed<BITS>& p, const Stage
     put(1, dequant_chunk<T, BITS, FP4, 1>(p, q0, 0u));
     put(2, dequant_chunk<T, BITS, FP4, 2>(p, q1, 0u));
     put(3, dequant_chunk<T, BITS, FP4, 3>(p, q1, 0u));
-    if (!tail) {
-      put(4, dequant_chunk<T, BITS, FP4, 4>(p, q2, 0u));
-      put(5, dequant_chunk<T, BITS, FP4, 5>(p, q2, 0u));
-      put(6, dequant_chunk<T, BITS, FP4, 6>(p, q3, 0u));
-      put(7, dequant_chunk<T, BITS, FP4, 7>(p, q3, 0u));
-    }
+    put(4, dequant_chunk<T, BITS, FP4, 4>(p, q2, 0u));
+    put(5, dequant_chunk<T, BITS, FP4, 5>(p, q2, 0u));
+    put(6, dequant_chunk<T, BITS, FP4, 6>(p, q3, 0u));
+    put(7, dequant_chunk<T, BITS, FP4, 7>(p, q3, 0u));
   } else {
     put(0, dequant_chunk<T, BITS, FP4, 0>(p, sb.s[0], sb.b[0]));
     put(1, dequant_chunk<T, BITS, FP4, 1>(p, sb.s[0], sb.b[0]));
     put(2, dequant_chunk<T, BITS, FP4, 2>(p, sb.s[0], sb.b[0]));
     put(3, dequant_chunk<T, BITS, FP4, 3>(p, sb.s[0], sb.b[0]));
-    if (!tail) {
-      put(4, dequant_chunk<T, BITS, FP4, 4>(p, sb.s[1], sb.b[1]));
-      put(5, dequant_chunk<T, BITS, FP4, 5>(p, sb.s[1], sb.b[1]));
-      put(6, dequant_chunk<T, BITS, FP4, 6>(p, sb.s[1], sb.b[1]));
-      put(7, dequant_chunk<T, BITS, FP4, 7>(p, sb.s[1], sb.b[1]));
-    }
+    put(4, dequant_chunk<T, BITS, FP4, 4>(p, sb.s[1], sb.b[1]));
+    put(5, dequant_chunk<T, BITS, FP4, 5>(p, sb.s[1], sb.b[1]));
+    put(6, dequant_chunk<T, BITS, FP4, 6>(p, sb.s[1], sb.b[1]));
+    put(7, dequant_chunk<T, BITS, FP4, 7>(p, sb.s[1], sb.b[1]));
   }
   if (tail) {
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    put(4, z); put(5, z); put(6, z); put(7, z);
+#pragma unroll
+    for (int c = 16; c < 32; ++c) o[c] = 0u;
   }
 }
 
@@ -434,8 +435,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = smem;                                   // operand rings (and split-K parking)
-  uint8_t* ring_a = smem;                                 // [ST] A 16 KB
-  uint8_t* ring_b = smem + ST * S::kABytes;               // [SB] B BT*128
+  uint8_t* ring_b = smem;                                 // [SB] B BT*128
   uint8_t* pring = smem + S::kOpBytes;                    // loader area
   uint8_t* wring = pring;                                 // TMA path: [WS] weight chunks
   uint8_t* sring = pring + WS * S::kWChunk;               // TMA path: [SS] scale chunks
@@ -686,13 +686,13 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
               mbar_wait(full_b(sb), (i / SB) & 1, abort_flag)))
           break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(ring_a + s * S::kABytes);
+        const uint32_t a_col = tmem + S::kACol0 + 32 * s;
         const uint32_t b_addr = smem_u32(ring_b + sb * S::kBBytes);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           const uint64_t bdesc = XMODE == 0 ? sdesc_sw128(b_addr + k * 32)
                                             : sdesc_sw32(b_addr + k * (BT * 32));
-          mma_f16(tmem, sdesc_sw128(a_addr + k * 32), bdesc, idesc, (i > 0 || k > 0) ? 1u : 0u);
+          mma_f16_tmem_a(tmem, a_col + 8 * k, bdesc, idesc, (i > 0 || k > 0) ? 1u : 0u);
         }
         mma_commit(empty_a(s));
         mma_commit(empty_b(sb));
@@ -704,7 +704,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   } else {
     // ------------------------------------------- dequantizers (warps 2..5)
     const int grp = (warp - kProducerWarp0) >> 2;          // dequantizer group
-    const int r = ((warp - kProducerWarp0) & 3) * 32 + lane; // weight row in the tile
+    const int r = (warp & 3) * 32 + lane;                  // weight row in the tile = TMEM lane
     const int64_t row = n0 + r;
     const bool row_ok = nl0 + r < a.n_limit;
     const bool fp4_g16 = FP4 && a.gs_log2 == 4;
@@ -826,16 +826,18 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         if (lane == 0) mbar_arrive(empty_l(ps));
       }
       const int s = i % ST;
-      if (!mbar_wait(empty_a(s), ((i / ST) & 1) ^ 1, abort_flag)) break;
-      uint8_t* a_row = ring_a + s * S::kABytes + r * 128;
+      if (!__all_sync(0xffffffffu, mbar_wait(empty_a(s), ((i / ST) & 1) ^ 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t o[32];
       if (row_ok) {
-        dequant_stage<T, BITS, FP4>(pk, sb, fp4_g16, a_row, r, tail);
+        dequant_row<T, BITS, FP4>(pk, sb, fp4_g16, tail, o);
       } else {
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a_row + (c << 4)) = z;
+        for (int c = 0; c < 32; ++c) o[c] = 0u;
       }
-      fence_proxy_async_smem();
+      tmem_st_32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + S::kACol0 + 32 * s, o);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(full_a(s));
     }

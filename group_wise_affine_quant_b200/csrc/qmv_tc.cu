@@ -95,40 +95,6 @@ __device__ __forceinline__ void load_row(Packed<BITS>& p, const uint8_t* wring, 
   }
 }
 
-// Dequantize one k-tile row (64 codes) into 32 words (T pairs in K order);
-// with `tail` the upper 32 columns are zero.  sb as for the smem dequantizer.
-template <typename T, int BITS, bool FP4>
-__device__ __forceinline__ void dequant_row(const Packed<BITS>& p, const StageSB& sb, bool fp4_g16,
-                                            bool tail, uint32_t (&o)[32]) {
-  auto put = [&](int c, uint4 v) { o[4 * c] = v.x; o[4 * c + 1] = v.y; o[4 * c + 2] = v.z; o[4 * c + 3] = v.w; };
-  if constexpr (FP4) {
-    const uint32_t q0 = sb.s[0];
-    const uint32_t q1 = fp4_g16 ? sb.s[1] : sb.s[0];
-    const uint32_t q2 = fp4_g16 ? sb.b[0] : sb.s[1];
-    const uint32_t q3 = fp4_g16 ? sb.b[1] : sb.s[1];
-    put(0, dequant_chunk<T, BITS, FP4, 0>(p, q0, 0u));
-    put(1, dequant_chunk<T, BITS, FP4, 1>(p, q0, 0u));
-    put(2, dequant_chunk<T, BITS, FP4, 2>(p, q1, 0u));
-    put(3, dequant_chunk<T, BITS, FP4, 3>(p, q1, 0u));
-    put(4, dequant_chunk<T, BITS, FP4, 4>(p, q2, 0u));
-    put(5, dequant_chunk<T, BITS, FP4, 5>(p, q2, 0u));
-    put(6, dequant_chunk<T, BITS, FP4, 6>(p, q3, 0u));
-    put(7, dequant_chunk<T, BITS, FP4, 7>(p, q3, 0u));
-  } else {
-    put(0, dequant_chunk<T, BITS, FP4, 0>(p, sb.s[0], sb.b[0]));
-    put(1, dequant_chunk<T, BITS, FP4, 1>(p, sb.s[0], sb.b[0]));
-    put(2, dequant_chunk<T, BITS, FP4, 2>(p, sb.s[0], sb.b[0]));
-    put(3, dequant_chunk<T, BITS, FP4, 3>(p, sb.s[0], sb.b[0]));
-    put(4, dequant_chunk<T, BITS, FP4, 4>(p, sb.s[1], sb.b[1]));
-    put(5, dequant_chunk<T, BITS, FP4, 5>(p, sb.s[1], sb.b[1]));
-    put(6, dequant_chunk<T, BITS, FP4, 6>(p, sb.s[1], sb.b[1]));
-    put(7, dequant_chunk<T, BITS, FP4, 7>(p, sb.s[1], sb.b[1]));
-  }
-  if (tail) {
-#pragma unroll
-    for (int c = 16; c < 32; ++c) o[c] = 0u;
-  }
-}
 
 template <typename T, int BITS, bool FP4>
 __global__ void __launch_bounds__(DecShape::kThreads, 2)
