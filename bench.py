@@ -53,8 +53,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-qmm", action="store_true", help="skip the TFLOP/s side lines")
-    ap.add_argument("--only", default="all", choices=["all", "qmm"],
-                    help="qmm: run only the TFLOP/s workloads (for profiling)")
+    ap.add_argument("--only", default="all", choices=["all", "qmm", "qmm-affine"],
+                    help="qmm: run only the TFLOP/s workloads; qmm-affine: only the 4-bit "
+                         "affine M = N = K = 4096 product (for profiling)")
     return ap.parse_args()
 
 
@@ -253,9 +254,16 @@ def run_reference(args):
     print(json.dumps(line))
 
 
-def qmm_lines(torch, api, inputs, dev, stream, tf_peak, tf_sust):
+def qmm_lines(torch, api, inputs, dev, stream, tf_peak, tf_sust, affine_only=False):
     """TFLOP/s of the tensor-core workloads (not part of the timed step)."""
     out = {}
+    if affine_only:
+        xf = inputs.fp4_x(4096, 4096).to(dev)
+        yf = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
+        wa = api.aq_quantize(inputs.normal((4096, 4096), 0.02, 1, inputs.gen(8)).to(dev), 4, 64)
+        t = graph_time_ms(torch, stream, lambda: api.aq_qmm(xf, *wa, 4, 64, out=yf), 10)
+        out["affine4_M4096"] = {"tflops": round(2 * 4096 ** 3 / (t * 1e-3) / 1e12, 1), "ms": round(t, 4)}
+        return out, None
     # chained fp16 qmm, 4-bit g64: 20 products per chain
     x, w1, w2 = inputs.chained()
     q1 = api.aq_quantize(w1.to(dev), 4, 64)
@@ -315,9 +323,10 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     hbm, tf, tf_sust, peak_kind = peaks()
-    if args.only == "qmm":
+    if args.only in ("qmm", "qmm-affine"):
         stream = torch.cuda.Stream(dev)
-        qmm, roof_qmm = qmm_lines(torch, api, inputs, dev, stream, tf, tf_sust)
+        qmm, roof_qmm = qmm_lines(torch, api, inputs, dev, stream, tf, tf_sust,
+                                  affine_only=args.only == "qmm-affine")
         if rank == 0:
             print(json.dumps({"qmm_tflops": qmm, "roofline_qmm": roof_qmm}))
         return
