@@ -34,6 +34,8 @@ SIGNATURES = {
     "aq_device_errors": (ctypes.c_uint, []),
     "aq_set_weight_prefetch": (None, [_I]),
     "aq_get_weight_prefetch": (_I, []),
+    "aq_set_input_prefetch": (None, [_I]),
+    "aq_get_input_prefetch": (_I, []),
 }
 
 _lib = None

@@ -14,7 +14,7 @@ from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, 
 
 __all__ = ["aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmm", "aq_qconv2d_nhwc",
            "aq_workspace_size", "aq_last_error", "aq_set_weight_prefetch",
-           "aq_get_weight_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
+           "aq_get_weight_prefetch", "aq_set_input_prefetch", "aq_get_input_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
 
 _DT = {torch.float16: AQ_F16, torch.bfloat16: AQ_BF16}
 _TORCH_DT = {AQ_F16: torch.float16, AQ_BF16: torch.bfloat16}
@@ -67,6 +67,15 @@ def aq_set_weight_prefetch(enable):
 
 def aq_get_weight_prefetch():
     return bool(lib().aq_get_weight_prefetch())
+
+
+def aq_set_input_prefetch(enable):
+    """Read x before waiting on the previous kernel (see include/aq.h)."""
+    lib().aq_set_input_prefetch(1 if enable else 0)
+
+
+def aq_get_input_prefetch():
+    return bool(lib().aq_get_input_prefetch())
 
 
 def aq_last_error():

@@ -74,9 +74,11 @@ aq_status check_weight(const void* w_q, const void* scales, const void* biases, 
 
 namespace {
 std::atomic<int> g_weight_prefetch{0};
+std::atomic<int> g_input_prefetch{0};
 }
 
 int aq::weight_prefetch_enabled() { return g_weight_prefetch.load(std::memory_order_relaxed); }
+int aq::input_prefetch_enabled() { return g_input_prefetch.load(std::memory_order_relaxed); }
 
 extern "C" {
 
@@ -87,6 +89,12 @@ void aq_set_weight_prefetch(int enable) {
 }
 
 int aq_get_weight_prefetch(void) { return aq::weight_prefetch_enabled(); }
+
+void aq_set_input_prefetch(int enable) {
+  g_input_prefetch.store(enable ? 1 : 0, std::memory_order_relaxed);
+}
+
+int aq_get_input_prefetch(void) { return aq::input_prefetch_enabled(); }
 
 int aq_version(void) { return 100; }
 

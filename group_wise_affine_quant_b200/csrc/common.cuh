@@ -135,5 +135,7 @@ cudaError_t launch_qmv_tc(const void* x, const void* w_q, const void* scales, co
 cudaError_t read_device_error_qmv_tc(unsigned* out);
 // aq_set_weight_prefetch's process-wide setting (0 or 1).
 int weight_prefetch_enabled();
+// aq_set_input_prefetch's process-wide setting (0 or 1).
+int input_prefetch_enabled();
 cudaError_t read_device_error_conv(unsigned* out);
 }  // namespace aq

@@ -73,6 +73,7 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
   a.K = Kp;
   a.gs_log2 = ilog2i(gs);
   a.weights_early = weight_prefetch_enabled();
+  a.x_early = input_prefetch_enabled();
   a.k_tiles = p.k_tiles;
   a.k_tiles_split = p.k_tiles_split;
   a.splits = p.splits;

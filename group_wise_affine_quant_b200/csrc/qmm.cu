@@ -51,6 +51,7 @@ cudaError_t launch_qmm(const QmmPlan& p, const void* x, const void* w_q, const v
   a.K = (int)K;
   a.gs_log2 = ilog2i(gs);
   a.weights_early = weight_prefetch_enabled();
+  a.x_early = input_prefetch_enabled();
   a.k_tiles = p.k_tiles;
   a.k_tiles_split = p.k_tiles_split;
   a.splits = p.splits;

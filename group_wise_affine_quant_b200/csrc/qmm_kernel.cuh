@@ -133,6 +133,7 @@ struct QmmArgs {
   int Cin, Cg, H, W, Ho, Wo, kh, kw, sh, sw, ph, pw, k_real;
   const void* x;        // conv gather path
   int weights_early;    // load weights/scales before waiting on the previous kernel
+  int x_early;          // read x before waiting on the previous kernel
 };
 
 struct QmmMaps {
@@ -505,7 +506,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   pdl_launch_dependents();
 
   if (warp == 0) {
-    pdl_wait();                                           // x may come from the previous kernel
+    if (!a.x_early) pdl_wait();                           // x may come from the previous kernel
     if constexpr (XMODE == 0) {
       // -------------------------------------------------- TMA producer (x)
       if (lane == 0) {

@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kThreads)
 qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
            const void* __restrict__ scales_v, const T* __restrict__ biases, T* __restrict__ y,
            int M, int64_t N, int64_t K, int gs_log2, int64_t Ks, int S, int lpr_log2, int RI,
-           int chunk_units, int weights_early) {
+           int chunk_units, int weights_early, int x_early) {
   const int gs = 1 << gs_log2;
   extern __shared__ float4 smem4[];
   float* smem = reinterpret_cast<float*>(smem4);
@@ -113,7 +113,7 @@ qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
     if (row < N && ul < nunits && ul < chunk_units)
       load_unit<BITS>(wq + row * row_bytes + k0 * BITS / 8 + (int64_t)ul * (4 * BITS), wd);
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (!x_early) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   for (int c0 = 0; c0 < nunits; c0 += chunk_units) {
     const int cu = (nunits - c0 < chunk_units) ? (nunits - c0) : chunk_units;
@@ -222,6 +222,7 @@ qmv_kernel(const T* __restrict__ x, const uint8_t* __restrict__ wq,
   // one so that no CTA exits while another still reads its shared memory.
   cg::cluster_group cluster = cg::this_cluster();
   if (S > 1) cluster.sync(); else __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");     // before y is written
   {
     // Rank `rank` finishes a contiguous slice of the [MT][rows_blk] sums with
     // 16-byte loads of every slice's partials (rows_blk is a multiple of 8),
@@ -288,7 +289,8 @@ cudaError_t launch_one(const QmvPlan& p, const void* x, const void* w_q, const v
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, (const T*)x, (const uint8_t*)w_q, scales,
                             (const T*)biases, (T*)y, (int)M, N, K, ilog2_floor(gs), p.ks, p.splits,
-                            ilog2_floor(p.lpr), p.ri, p.chunk_units, weight_prefetch_enabled());
+                            ilog2_floor(p.lpr), p.ri, p.chunk_units, weight_prefetch_enabled(),
+                            input_prefetch_enabled());
 }
 
 template <typename T, int BITS, bool FP4>

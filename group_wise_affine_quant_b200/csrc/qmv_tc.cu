@@ -73,6 +73,7 @@ struct DecArgs {
   int splits;
   int mp;               // M rounded up to 4 (partial columns pushed per row)
   int weights_early;
+  int x_early;           // read x before waiting on the previous kernel
 };
 
 // This thread's weight row for one k-tile (64 codes, 8 * BITS bytes at
@@ -204,7 +205,7 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
     if (lane == 0) load_chunks(false);
   } else if (warp == S::kWarpX) {
     // -------------------------------------------------------- x tiles by TMA
-    pdl_wait();                                           // x may come from the previous kernel
+    if (!a.x_early) pdl_wait();                           // x may come from the previous kernel
     if (lane == 0) {
       for (int j = 0; j < nst; ++j) {
         const int s = j % XS;
@@ -505,6 +506,7 @@ cudaError_t launch_qmv_tc(const void* x, const void* w_q, const void* scales, co
   a.splits = splits;
   a.mp = (int)((M + 3) / 4 * 4);
   a.weights_early = weight_prefetch_enabled();
+  a.x_early = input_prefetch_enabled();
   QmmMaps maps;
   memset(&maps, 0, sizeof(maps));
   const CUtensorMapDataType tt =

@@ -191,6 +191,19 @@ AQ_API unsigned aq_device_errors(void);
 AQ_API void aq_set_weight_prefetch(int enable);
 AQ_API int aq_get_weight_prefetch(void);
 
+/*
+ * Input prefetch (process-wide, default 0 = off).  With it on, a matmul that
+ * starts while the previous kernel on its stream is still running also
+ * reads x before waiting for that kernel; it still waits before writing y,
+ * so y is ordered after everything earlier on the stream.  Turn it on only
+ * when no kernel that may still be running when a matmul starts writes that
+ * matmul's x: for instance calls whose x were all written before the first
+ * of them was launched (projections that share an input, experts of one
+ * batch, a sweep over fixed activations).
+ */
+AQ_API void aq_set_input_prefetch(int enable);
+AQ_API int aq_get_input_prefetch(void);
+
 /* Message for the last non-AQ_OK status on the calling thread ("" if none). */
 AQ_API const char* aq_last_error(void);
 

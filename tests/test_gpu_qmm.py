@@ -233,6 +233,36 @@ def test_dependent_chain_under_pdl(prefetch):
         assert torch.equal(outs[i], ref[i]), i
 
 
+def test_independent_calls_under_input_prefetch():
+    """Calls whose x were all written before the first launch, each into its
+    own y, with weight and input prefetch on (each kernel may read its
+    weights and x while the previous one runs): results equal the same calls
+    separated by device synchronisation."""
+    bits, gs = 4, 64
+    g = inputs.gen(33)
+    ws = [api.aq_quantize(to_dev(inputs.normal((n, 1024), 0.05, 1, g)), bits, gs)
+          for n in (512, 128, 2048, 384)]
+    xs = [to_dev(inputs.normal((m, 1024), 1.0, 1, g)) for m in (1, 4, 16, 40)]
+    torch.cuda.synchronize()
+    calls = [(api.aq_qmv if x.shape[0] <= 16 else api.aq_qmm, x, w) for x in xs for w in ws]
+    ref = []
+    for fn, x, w in calls:
+        ref.append(fn(x, *w, bits, gs))
+        torch.cuda.synchronize()
+    old_w, old_x = api.aq_get_weight_prefetch(), api.aq_get_input_prefetch()
+    api.aq_set_weight_prefetch(True)
+    api.aq_set_input_prefetch(True)
+    try:
+        outs = [fn(x, *w, bits, gs) for fn, x, w in calls]
+        torch.cuda.synchronize()
+    finally:
+        api.aq_set_weight_prefetch(old_w)
+        api.aq_set_input_prefetch(old_x)
+    for i, (a, b) in enumerate(zip(outs, ref)):
+        assert torch.equal(a, b), i
+    assert api.lib().aq_device_errors() == 0
+
+
 def test_quantize_then_matmul_default_order():
     """Weights written by the kernel just before (prefetch off by default)."""
     assert not api.aq_get_weight_prefetch()
