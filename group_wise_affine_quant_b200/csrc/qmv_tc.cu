@@ -385,21 +385,30 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
         bool have = true;
         if (clustered) have = mbar_wait_cluster(recv_full, 0, abort_flag, 4000000000ull);
         if (have) {
+          // all partials of this row first (independent loads), then the
+          // sum in slice order with this slice's own partial at its place
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            if (k >= a.splits) break;
-            if (k == split) {
+          for (int t = 0; t < 16; t += 4) {
+            if (t < a.mp) {
+              float4 p[7];
 #pragma unroll
-              for (int t = 0; t < 16; ++t) acc[t] += __uint_as_float(v[t]);
-            } else {
-              const float* pr = recv + ((k < split ? k : k - 1) * rpo + (r - own0)) * a.mp;
+              for (int k = 0; k < 7; ++k)
+                p[k] = k < a.splits - 1
+                           ? *reinterpret_cast<const float4*>(recv + (k * rpo + (r - own0)) * a.mp + t)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+              // slices 0 .. split-1 (receive slots 0 .. split-1), this slice,
+              // then slices split+1 .. (receive slots split ..)
+              auto add = [&](float4 q4) {
+                acc[t] += q4.x; acc[t + 1] += q4.y; acc[t + 2] += q4.z; acc[t + 3] += q4.w;
+              };
 #pragma unroll
-              for (int t = 0; t < 16; t += 4) {
-                if (t < a.mp) {
-                  const float4 p4 = *reinterpret_cast<const float4*>(pr + t);
-                  acc[t] += p4.x; acc[t + 1] += p4.y; acc[t + 2] += p4.z; acc[t + 3] += p4.w;
-                }
-              }
+              for (int k = 0; k < 7; ++k)
+                if (k < split) add(p[k]);
+              add(make_float4(__uint_as_float(v[t]), __uint_as_float(v[t + 1]),
+                              __uint_as_float(v[t + 2]), __uint_as_float(v[t + 3])));
+#pragma unroll
+              for (int k = 0; k < 7; ++k)
+                if (k >= split && k < a.splits - 1) add(p[k]);
             }
           }
           pdl_wait();                                     // before y is written
