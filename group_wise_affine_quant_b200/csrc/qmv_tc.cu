@@ -158,15 +158,18 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
         const int slot = lc % WS;
         if (prologue ? lc >= WS : !mbar_wait(empty_w(slot), ((lc / WS) & 1) ^ 1, abort_flag)) return;
         mbar_arrive_expect_tx(full_w(slot), S::kWChunk);
-        tma_load_2d(smem_u32(wring + slot * S::kWChunk), &maps.w, full_w(slot), wb0 + 128 * lc, n0);
+        tma_load_2d_hint(smem_u32(wring + slot * S::kWChunk), &maps.w, full_w(slot), wb0 + 128 * lc, n0,
+                         l2_policy_evict_first());
         ++lc;
       } else {
         const int slot = lj % SS;
         if (prologue ? lj >= SS : !mbar_wait(empty_s(slot), ((lj / SS) & 1) ^ 1, abort_flag)) return;
         const uint32_t dst = smem_u32(sring + slot * S::kSChunk);
         mbar_arrive_expect_tx(full_s(slot), FP4 ? kRowsW * 16 : 2 * kRowsW * 16);
-        tma_load_2d(dst, &maps.s, full_s(slot), (sc0 + lj) * SGC, n0);
-        if constexpr (!FP4) tma_load_2d(dst + kRowsW * 16, &maps.b, full_s(slot), (sc0 + lj) * SGC, n0);
+        tma_load_2d_hint(dst, &maps.s, full_s(slot), (sc0 + lj) * SGC, n0, l2_policy_evict_first());
+        if constexpr (!FP4)
+          tma_load_2d_hint(dst + kRowsW * 16, &maps.b, full_s(slot), (sc0 + lj) * SGC, n0,
+                           l2_policy_evict_first());
         ++lj;
       }
     }
@@ -213,8 +216,10 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
         if (!mbar_wait(empty_x(s), ((j / XS) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(full_x(s), two ? S::kXBytes : S::kXAtom);
         const uint32_t dst = smem_u32(xring + s * S::kXBytes);
-        tma_load_2d(dst, &maps.x, full_x(s), (kt0 + 2 * j) * kBK, 0);
-        if (two) tma_load_2d(dst + S::kXAtom, &maps.x, full_x(s), (kt0 + 2 * j + 1) * kBK, 0);
+        tma_load_2d_hint(dst, &maps.x, full_x(s), (kt0 + 2 * j) * kBK, 0, l2_policy_evict_last());
+        if (two)
+          tma_load_2d_hint(dst + S::kXAtom, &maps.x, full_x(s), (kt0 + 2 * j + 1) * kBK, 0,
+                           l2_policy_evict_last());
       }
     }
   } else if (warp == S::kWarpMma) {
