@@ -289,10 +289,31 @@ __device__ __forceinline__ uint32_t code_pair(const Packed<BITS>& p) {
   }
 }
 
-template <typename T, int C, int J>
-__device__ __forceinline__ uint32_t fp4_pair(const Packed<4>& p) {
-  constexpr int k0 = 8 * C + 2 * J;
-  return Pair<T>::from_f2(e2m1_to_float(code_at<4, k0>(p.w)), e2m1_to_float(code_at<4, k0 + 1>(p.w)));
+// E2M1 magnitudes (code & 7: 0, 0.5, 1, 1.5, 2, 3, 4, 6) as T, split into
+// high and low bytes so that one byte permute looks up four codes at once.
+template <typename T> struct Fp4Bytes;
+template <> struct Fp4Bytes<__nv_bfloat16> {
+  static constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u;   // 0x00 0x3F 0x3F 0x3F | 0x40 x4
+  static constexpr uint32_t kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;   // 0x00 0x00 0x80 0xC0 | 0x00 0x40 0x80 0xC0
+};
+template <> struct Fp4Bytes<__half> {
+  static constexpr uint32_t kHi0 = 0x3E3C3800u, kHi1 = 0x46444240u;   // 0x00 0x38 0x3C 0x3E | 0x40 0x42 0x44 0x46
+  static constexpr uint32_t kLo0 = 0u, kLo1 = 0u;
+};
+
+// The four E2M1 codes in the low 16 bits of h (code i in bits 4i..4i+3,
+// bit 3 the sign) as two T pairs in code order: exact values, no rounding.
+template <typename T>
+__device__ __forceinline__ void fp4_quad(uint32_t h, uint32_t& pa, uint32_t& pb) {
+  const uint32_t sel = h & 0x7777u;                     // magnitude index per code
+  const uint32_t sg = h & 0x8888u;                      // sign bits
+  uint32_t hi = __byte_perm(Fp4Bytes<T>::kHi0, Fp4Bytes<T>::kHi1, sel);
+  // sign of code i into bit 7 of byte i: bytes of (sg << 4) carry codes 0 and
+  // 2 at bit 7, bytes of sg carry codes 1 and 3 there
+  hi |= __byte_perm(sg << 4, sg, 0x5140) & 0x80808080u;
+  const uint32_t lo = __byte_perm(Fp4Bytes<T>::kLo0, Fp4Bytes<T>::kLo1, sel);
+  pa = __byte_perm(lo, hi, 0x5140);                     // (code 0, code 1)
+  pb = __byte_perm(lo, hi, 0x7362);                     // (code 2, code 3)
 }
 
 // Dequantize chunk C (8 elements) into 16 bytes.
@@ -300,10 +321,14 @@ template <typename T, int BITS, bool FP4, int C>
 __device__ __forceinline__ uint4 dequant_chunk(const Packed<BITS>& p, uint32_t s2, uint32_t b2) {
   uint4 o;
   if constexpr (FP4) {
-    o.x = Pair<T>::mul(fp4_pair<T, C, 0>(p), s2);
-    o.y = Pair<T>::mul(fp4_pair<T, C, 1>(p), s2);
-    o.z = Pair<T>::mul(fp4_pair<T, C, 2>(p), s2);
-    o.w = Pair<T>::mul(fp4_pair<T, C, 3>(p), s2);
+    // 8 codes of chunk C are word C (4-bit, low nibble first)
+    uint32_t q0, q1, q2, q3;
+    fp4_quad<T>(p.w[C], q0, q1);
+    fp4_quad<T>(p.w[C] >> 16, q2, q3);
+    o.x = Pair<T>::mul(q0, s2);
+    o.y = Pair<T>::mul(q1, s2);
+    o.z = Pair<T>::mul(q2, s2);
+    o.w = Pair<T>::mul(q3, s2);
   } else {
     o.x = Pair<T>::fma(code_pair<T, BITS, C, 0>(p), s2, b2);
     o.y = Pair<T>::fma(code_pair<T, BITS, C, 1>(p), s2, b2);
