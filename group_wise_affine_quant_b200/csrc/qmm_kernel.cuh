@@ -134,6 +134,7 @@ struct QmmArgs {
   const void* x;        // conv gather path
   int weights_early;    // load weights/scales before waiting on the previous kernel
   int x_early;          // read x before waiting on the previous kernel
+  int scale_copy;       // TMA path: scale rows are not 16-byte multiples, copy them
 };
 
 struct QmmMaps {
@@ -621,30 +622,75 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     // the caller has declared that no preceding kernel writes them.
     if (!a.weights_early) pdl_wait();
     if constexpr (FAST) {
-      // ------------------- weight and scale chunks by TMA, in K order
-      if (lane == 0) {
-        int c = 0, j = 0;
-        while (c < nwc || j < nsc) {
-          // K position (in codes, relative to kt0 * 64) where each chunk starts
-          const int64_t kw = c < nwc ? (int64_t)c * 128 * 8 / BITS : INT64_MAX;
-          const int64_t ks = j < nsc ? (int64_t)(sc0 + j) * SGC * (1 << a.gs_log2) - (int64_t)kt0 * kBK
-                                     : INT64_MAX;
-          if (kw <= ks) {
-            const int slot = c % WS;
-            if (!mbar_wait(empty_l(slot), ((c / WS) & 1) ^ 1, abort_flag)) break;
-            mbar_arrive_expect_tx(full_l(slot), S::kWChunk);
-            tma_load_2d(smem_u32(wring + slot * S::kWChunk), &maps.w, full_l(slot),
-                        (int)(wb0 + 128 * c), n0);
-            ++c;
-          } else {
-            const int slot = j % SS;
-            if (!mbar_wait(empty_l(WS + slot), ((j / SS) & 1) ^ 1, abort_flag)) break;
-            const uint32_t dst = smem_u32(sring + slot * S::kSChunk);
-            mbar_arrive_expect_tx(full_l(WS + slot), FP4 ? kRowsW * 16 : 2 * kRowsW * 16);
-            tma_load_2d(dst, &maps.s, full_l(WS + slot), (sc0 + j) * SGC, n0);
-            if constexpr (!FP4) tma_load_2d(dst + kRowsW * 16, &maps.b, full_l(WS + slot), (sc0 + j) * SGC, n0);
-            ++j;
+      // ------------------- weight and scale chunks in K order
+      // Weight chunks by TMA (lane 0).  Scale chunks by TMA too when the rows
+      // of scales are 16-byte multiples; otherwise the whole warp copies them
+      // with element loads into the same chunk layout (4 rows per lane) and
+      // lane 0 publishes the chunk with a release arrive.  Every branch is
+      // taken by the whole warp, so a failed wait leaves the loop together.
+      int c = 0, j = 0;
+      while (c < nwc || j < nsc) {
+        // K position (in codes, relative to kt0 * 64) where each chunk starts
+        const int64_t kw = c < nwc ? (int64_t)c * 128 * 8 / BITS : INT64_MAX;
+        const int64_t ks = j < nsc ? (int64_t)(sc0 + j) * SGC * (1 << a.gs_log2) - (int64_t)kt0 * kBK
+                                   : INT64_MAX;
+        if (kw <= ks) {
+          const int slot = c % WS;
+          bool ok = true;
+          if (lane == 0) {
+            ok = mbar_wait(empty_l(slot), ((c / WS) & 1) ^ 1, abort_flag);
+            if (ok) {
+              mbar_arrive_expect_tx(full_l(slot), S::kWChunk);
+              tma_load_2d(smem_u32(wring + slot * S::kWChunk), &maps.w, full_l(slot),
+                          (int)(wb0 + 128 * c), n0);
+            }
           }
+          if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+          ++c;
+        } else {
+          const int slot = j % SS;
+          if (a.scale_copy) {
+            if (!__all_sync(0xffffffffu, mbar_wait(empty_l(WS + slot), ((j / SS) & 1) ^ 1, abort_flag))) break;
+            uint8_t* dst = sring + slot * S::kSChunk;
+            const int g0 = (sc0 + j) * SGC;
+#pragma unroll
+            for (int jj = 0; jj < kRowsW / 32; ++jj) {
+              const int rr = lane + 32 * jj;
+              const int64_t row = n0 + rr;
+              const bool rok = nl0 + rr < a.n_limit && row < a.N;
+              if constexpr (FP4) {
+                const uint8_t* sp = reinterpret_cast<const uint8_t*>(a.scales) + row * G;
+#pragma unroll
+                for (int q = 0; q < SGC; ++q)
+                  dst[rr * 16 + q] = (rok && g0 + q < G) ? sp[g0 + q] : (uint8_t)0;
+              } else {
+                const uint16_t* sp = reinterpret_cast<const uint16_t*>(a.scales) + row * G;
+                const uint16_t* bp = reinterpret_cast<const uint16_t*>(a.biases) + row * G;
+#pragma unroll
+                for (int q = 0; q < SGC; ++q) {
+                  const bool in = rok && g0 + q < G;
+                  reinterpret_cast<uint16_t*>(dst + rr * 16)[q] = in ? sp[g0 + q] : (uint16_t)0;
+                  reinterpret_cast<uint16_t*>(dst + kRowsW * 16 + rr * 16)[q] = in ? bp[g0 + q] : (uint16_t)0;
+                }
+              }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full_l(WS + slot));
+          } else {
+            bool ok = true;
+            if (lane == 0) {
+              ok = mbar_wait(empty_l(WS + slot), ((j / SS) & 1) ^ 1, abort_flag);
+              if (ok) {
+                const uint32_t dst = smem_u32(sring + slot * S::kSChunk);
+                mbar_arrive_expect_tx(full_l(WS + slot), FP4 ? kRowsW * 16 : 2 * kRowsW * 16);
+                tma_load_2d(dst, &maps.s, full_l(WS + slot), (sc0 + j) * SGC, n0);
+                if constexpr (!FP4)
+                  tma_load_2d(dst + kRowsW * 16, &maps.b, full_l(WS + slot), (sc0 + j) * SGC, n0);
+              }
+            }
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+          }
+          ++j;
         }
       }
     } else {
@@ -1097,12 +1143,16 @@ inline cudaError_t weight_maps(QmmMaps& maps, QmmArgs& a, const void* w_q, const
           : (a.row_bytes % 8 == 0 && (8 * bits) % 8 == 0) ? 8 : 4;
   const int64_t G = K / gs;
   const int esz = mode == AQ_MODE_FP4 ? 1 : 2;
-  *fast = a.row_bytes % 16 == 0 && (G * esz) % 16 == 0 && ((uintptr_t)scales & 15) == 0 &&
-          (mode == AQ_MODE_FP4 || ((uintptr_t)biases & 15) == 0);
+  *fast = a.row_bytes % 16 == 0;
   if (!*fast) return cudaSuccess;
+  // scale rows that TMA cannot address (stride or base not 16-byte aligned)
+  // are copied by the loader warp instead
+  a.scale_copy = !((G * esz) % 16 == 0 && ((uintptr_t)scales & 15) == 0 &&
+                   (mode == AQ_MODE_FP4 || ((uintptr_t)biases & 15) == 0));
   cudaError_t e = make_map(&maps.w, w_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, a.row_bytes, 128,
                            kRowsW, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
+  if (a.scale_copy) return cudaSuccess;
   const CUtensorMapDataType st_t =
       mode == AQ_MODE_FP4 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
   e = make_map(&maps.s, scales, st_t, esz, rows, G, 16 / esz, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE);

@@ -532,7 +532,7 @@ cudaError_t launch_qmv_tc(const void* x, const void* w_q, const void* scales, co
   bool fast = false;
   e = weight_maps(maps, wa, w_q, scales, biases, N, K, bits, gs, mode, &fast);
   if (e != cudaSuccess) return e;
-  if (!fast) return cudaErrorInvalidValue;
+  if (!fast || wa.scale_copy) return cudaErrorInvalidValue;   // qmv_tc_applies excludes both
   return dtype == AQ_F16 ? dec_by_bits<__half>(maps, a, n_tiles, bits, mode, st)
                          : dec_by_bits<__nv_bfloat16>(maps, a, n_tiles, bits, mode, st);
 }
