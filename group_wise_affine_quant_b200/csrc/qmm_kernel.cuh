@@ -400,6 +400,34 @@ __device__ __forceinline__ StageSB sb_from_words(const uint4 wv, const QmmArgs& 
 // Dequantize one weight row of a K-stage (64 codes) into 32 words (T pairs
 // in K order), the layout of an A operand in tensor memory: lane = row, two
 // 16-bit values per column.  With `tail` the upper 32 columns are zero.
+// Raw scale / bias values of one row for K-stage kt, straight from global
+// memory (rows of scales that TMA cannot address): affine {s(g0), s(g1),
+// b(g0), b(g1)}; FP4 the scale bytes of the stage's groups (four at group
+// 16, two at group 32).  g1 is the group of the stage's second half.
+template <bool FP4>
+__device__ __forceinline__ void load_stage_scales(uint32_t (&raw)[4], const void* scales,
+                                                  const void* biases, int64_t row, int G, int kt,
+                                                  int gs_log2, int K, bool valid) {
+  raw[0] = raw[1] = raw[2] = raw[3] = 0u;
+  if (!valid) return;
+  const bool tail = (kt + 1) * 64 > K;
+  const int g0 = (kt * 64) >> gs_log2;
+  if constexpr (FP4) {
+    const uint8_t* sp = reinterpret_cast<const uint8_t*>(scales) + row * G;
+    if (gs_log2 == 4) {
+      raw[0] = sp[g0]; raw[1] = sp[g0 + 1];
+      if (!tail) { raw[2] = sp[g0 + 2]; raw[3] = sp[g0 + 3]; }
+    } else {
+      raw[0] = sp[g0]; raw[1] = tail ? raw[0] : sp[(kt * 64 + 32) >> gs_log2];
+    }
+  } else {
+    const int g1 = tail ? g0 : ((kt * 64 + 32) >> gs_log2);
+    const uint16_t* sp = reinterpret_cast<const uint16_t*>(scales) + row * G;
+    const uint16_t* bp = reinterpret_cast<const uint16_t*>(biases) + row * G;
+    raw[0] = sp[g0]; raw[1] = sp[g1]; raw[2] = bp[g0]; raw[3] = bp[g1];
+  }
+}
+
 template <typename T, int BITS, bool FP4>
 __device__ __forceinline__ void dequant_row(const Packed<BITS>& p, const StageSB& sb, bool fp4_g16,
                                             bool tail, uint32_t (&o)[32]) {
@@ -499,7 +527,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   const int nwc = (int)((nkt * S::kPB + 127) / 128);
   const int sc0 = ((kt0 * kBK) >> a.gs_log2) / SGC;
   const int sc1 = (((kt1 * kBK) - 1) >> a.gs_log2) / SGC;
-  const int nsc = sc1 - sc0 + 1;
+  const int nsc = a.scale_copy ? 0 : sc1 - sc0 + 1;    // scale chunks (none: read from global)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -623,11 +651,10 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     if (!a.weights_early) pdl_wait();
     if constexpr (FAST) {
       // ------------------- weight and scale chunks in K order
-      // Weight chunks by TMA (lane 0).  Scale chunks by TMA too when the rows
-      // of scales are 16-byte multiples; otherwise the whole warp copies them
-      // with element loads into the same chunk layout (4 rows per lane) and
-      // lane 0 publishes the chunk with a release arrive.  Every branch is
-      // taken by the whole warp, so a failed wait leaves the loop together.
+      // Weight and scale chunks by TMA (lane 0; the warp follows lane 0's
+      // wait result, so a failed wait leaves the loop together).  When the
+      // rows of scales are not 16-byte multiples there are no scale chunks:
+      // the dequantizers read their scales from global memory.
       int c = 0, j = 0;
       while (c < nwc || j < nsc) {
         // K position (in codes, relative to kt0 * 64) where each chunk starts
@@ -649,47 +676,18 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
           ++c;
         } else {
           const int slot = j % SS;
-          if (a.scale_copy) {
-            if (!__all_sync(0xffffffffu, mbar_wait(empty_l(WS + slot), ((j / SS) & 1) ^ 1, abort_flag))) break;
-            uint8_t* dst = sring + slot * S::kSChunk;
-            const int g0 = (sc0 + j) * SGC;
-#pragma unroll
-            for (int jj = 0; jj < kRowsW / 32; ++jj) {
-              const int rr = lane + 32 * jj;
-              const int64_t row = n0 + rr;
-              const bool rok = nl0 + rr < a.n_limit && row < a.N;
-              if constexpr (FP4) {
-                const uint8_t* sp = reinterpret_cast<const uint8_t*>(a.scales) + row * G;
-#pragma unroll
-                for (int q = 0; q < SGC; ++q)
-                  dst[rr * 16 + q] = (rok && g0 + q < G) ? sp[g0 + q] : (uint8_t)0;
-              } else {
-                const uint16_t* sp = reinterpret_cast<const uint16_t*>(a.scales) + row * G;
-                const uint16_t* bp = reinterpret_cast<const uint16_t*>(a.biases) + row * G;
-#pragma unroll
-                for (int q = 0; q < SGC; ++q) {
-                  const bool in = rok && g0 + q < G;
-                  reinterpret_cast<uint16_t*>(dst + rr * 16)[q] = in ? sp[g0 + q] : (uint16_t)0;
-                  reinterpret_cast<uint16_t*>(dst + kRowsW * 16 + rr * 16)[q] = in ? bp[g0 + q] : (uint16_t)0;
-                }
-              }
+          bool ok = true;
+          if (lane == 0) {
+            ok = mbar_wait(empty_l(WS + slot), ((j / SS) & 1) ^ 1, abort_flag);
+            if (ok) {
+              const uint32_t dst = smem_u32(sring + slot * S::kSChunk);
+              mbar_arrive_expect_tx(full_l(WS + slot), FP4 ? kRowsW * 16 : 2 * kRowsW * 16);
+              tma_load_2d(dst, &maps.s, full_l(WS + slot), (sc0 + j) * SGC, n0);
+              if constexpr (!FP4)
+                tma_load_2d(dst + kRowsW * 16, &maps.b, full_l(WS + slot), (sc0 + j) * SGC, n0);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full_l(WS + slot));
-          } else {
-            bool ok = true;
-            if (lane == 0) {
-              ok = mbar_wait(empty_l(WS + slot), ((j / SS) & 1) ^ 1, abort_flag);
-              if (ok) {
-                const uint32_t dst = smem_u32(sring + slot * S::kSChunk);
-                mbar_arrive_expect_tx(full_l(WS + slot), FP4 ? kRowsW * 16 : 2 * kRowsW * 16);
-                tma_load_2d(dst, &maps.s, full_l(WS + slot), (sc0 + j) * SGC, n0);
-                if constexpr (!FP4)
-                  tma_load_2d(dst + kRowsW * 16, &maps.b, full_l(WS + slot), (sc0 + j) * SGC, n0);
-              }
-            }
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
           }
+          if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
           ++j;
         }
       }
@@ -816,6 +814,12 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
       }
       return okr;
     };
+    // scales straight from global memory: this group's next stage is loaded
+    // one iteration ahead, so the load latency hides behind a stage
+    uint32_t sraw[4] = {0u, 0u, 0u, 0u};
+    if (FAST && a.scale_copy && grp < nkt)
+      load_stage_scales<FP4>(sraw, a.scales, a.biases, row, G, kt0 + grp, a.gs_log2, a.K,
+                             row_ok && row < a.N);
     for (int i = grp; i < nkt; i += kDqGroups) {
       const int kt = kt0 + i;
       const bool tail = (kt + 1) * kBK > a.K;
@@ -827,9 +831,11 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         bool ok = true;
         for (; w_ready <= c_hi && ok; ++w_ready)
           ok = mbar_wait(full_l(w_ready % WS), (w_ready / WS) & 1, abort_flag);
-        const int sj = (((kt * kBK) >> a.gs_log2) / SGC) - sc0;
-        for (; s_ready <= sj && ok; ++s_ready)
-          ok = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
+        if (!a.scale_copy) {
+          const int sj = (((kt * kBK) >> a.gs_log2) / SGC) - sc0;
+          for (; s_ready <= sj && ok; ++s_ready)
+            ok = mbar_wait(full_l(WS + s_ready % SS), (s_ready / SS) & 1, abort_flag);
+        }
         if (!ok) break;
         if constexpr (S::kPB % 16 == 0) {
 #pragma unroll
@@ -852,34 +858,52 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
 #pragma unroll
           for (int w = BITS; w < 2 * BITS; ++w) pk.w[w] = 0u;
         }
-        const uint8_t* sslot = sring + ((s_ready - 1) % SS) * S::kSChunk;
-        const int g0 = (kt * kBK) >> a.gs_log2;
-        const int g1 = tail ? g0 : ((kt * kBK + 32) >> a.gs_log2);
-        if constexpr (FP4) {
-          const uint8_t* sp = sslot + r * 16;
-          const int gs = 1 << a.gs_log2;
-          auto sc = [&](int g) { return splat(TT<T>::from_f(fp4_scale_t<T>(sp[g % SGC], gs))); };
-          if (fp4_g16) {
-            sb.s[0] = sc(g0); sb.s[1] = sc(g0 + 1);
-            sb.b[0] = tail ? sb.s[0] : sc(g0 + 2);
-            sb.b[1] = tail ? sb.s[0] : sc(g0 + 3);
+        uint32_t raw[4];
+        if (a.scale_copy) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) raw[u] = sraw[u];
+          if (i + kDqGroups < nkt)
+            load_stage_scales<FP4>(sraw, a.scales, a.biases, row, G, kt + kDqGroups, a.gs_log2, a.K,
+                                   row_ok && row < a.N);
+        } else {
+          const uint8_t* sslot = sring + ((s_ready - 1) % SS) * S::kSChunk;
+          const int g0 = (kt * kBK) >> a.gs_log2;
+          const int g1 = tail ? g0 : ((kt * kBK + 32) >> a.gs_log2);
+          if constexpr (FP4) {
+            const uint8_t* sp = sslot + r * 16;
+            if (fp4_g16) {
+              raw[0] = sp[g0 % SGC]; raw[1] = sp[(g0 + 1) % SGC];
+              raw[2] = sp[(g0 + 2) % SGC]; raw[3] = sp[(g0 + 3) % SGC];
+            } else {
+              raw[0] = sp[g0 % SGC]; raw[1] = sp[g1 % SGC]; raw[2] = raw[3] = 0u;
+            }
           } else {
-            sb.s[0] = sc(g0); sb.s[1] = sc(g1); sb.b[0] = sb.b[1] = 0u;
+            const uint16_t* sp = reinterpret_cast<const uint16_t*>(sslot + r * 16);
+            const uint16_t* bp = reinterpret_cast<const uint16_t*>(sslot + kRowsW * 16 + r * 16);
+            raw[0] = sp[g0 % SGC]; raw[1] = sp[g1 % SGC];
+            raw[2] = bp[g0 % SGC]; raw[3] = bp[g1 % SGC];
+          }
+        }
+        if constexpr (FP4) {
+          const int gs = 1 << a.gs_log2;
+          auto sc = [&](uint32_t v) { return splat(TT<T>::from_f(fp4_scale_t<T>(v, gs))); };
+          if (fp4_g16) {
+            sb.s[0] = sc(raw[0]); sb.s[1] = sc(raw[1]);
+            sb.b[0] = tail ? sb.s[0] : sc(raw[2]);
+            sb.b[1] = tail ? sb.s[0] : sc(raw[3]);
+          } else {
+            sb.s[0] = sc(raw[0]); sb.s[1] = sc(raw[1]); sb.b[0] = sb.b[1] = 0u;
           }
         } else {
-          const uint16_t* sp = reinterpret_cast<const uint16_t*>(sslot + r * 16);
-          const uint16_t* bp = reinterpret_cast<const uint16_t*>(sslot + kRowsW * 16 + r * 16);
-          const uint32_t s0 = sp[g0 % SGC], s1 = sp[g1 % SGC];
-          const uint32_t b0 = bp[g0 % SGC], b1 = bp[g1 % SGC];
-          sb.s[0] = s0 | (s0 << 16); sb.s[1] = s1 | (s1 << 16);
-          sb.b[0] = b0 | (b0 << 16); sb.b[1] = b1 | (b1 << 16);
+          sb.s[0] = raw[0] | (raw[0] << 16); sb.s[1] = raw[1] | (raw[1] << 16);
+          sb.b[0] = raw[2] | (raw[2] << 16); sb.b[1] = raw[3] | (raw[3] << 16);
         }
         // release the chunks this group is done with: those that end before
         // its next stage starts (all of them after its last stage)
         const bool last = i + kDqGroups >= nkt;
         const int w_done = last ? nwc : (((i + kDqGroups) * S::kPB) >> 7);
-        const int s_done =
-            last ? nsc : ((((kt + kDqGroups) * kBK) >> a.gs_log2) / SGC) - sc0;
+        const int s_done = a.scale_copy ? 0
+                           : last ? nsc : ((((kt + kDqGroups) * kBK) >> a.gs_log2) / SGC) - sc0;
         if (!release_upto(w_done, s_done)) break;
       } else {
         const int ps = i % PST;
