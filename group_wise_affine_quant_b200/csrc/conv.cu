@@ -10,6 +10,9 @@
 //     as one 4-D TMA box at the filter tap's (w, h) offset; out-of-bounds
 //     coordinates read zeros, which are the image padding, and K-columns past
 //     kh*kw*Cg read a box past the image (zeros).
+//   * When, besides, Cg is a multiple of 64, every 64-column K-stage is 64
+//     channels of a single tap, and the stage is one 64-channel box with the
+//     128-byte swizzle of the dense path (fewer, wider TMA requests).
 //   * Other shapes gather 16-byte granules (8 channels) with cp.async,
 //     zero-filling the padding.
 // Output channel block g of the conv group g is weight rows [g*Ng, (g+1)*Ng)
@@ -44,6 +47,10 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
     for (int cand = bt; cand >= 64; cand /= 2)
       if (rect(cand)) { bt = cand; xmode = 1; break; }
   }
+  // Every 64-column K-stage is 64 channels of one tap when Cg % 64 == 0: one
+  // 64-channel box per stage (weights on the TMA path, rows 16-byte multiples)
+  const bool w_rows16 = ((int64_t)Kp * bits / 8) % 16 == 0;
+  if (xmode == 1 && Cg % 64 == 0 && w_rows16) xmode = 3;
   QmmPlan p{};
   p.bt = bt;
   p.n_tiles = (int64_t)ntg * groups;
@@ -56,9 +63,9 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
   const CUtensorMapDataType tt =
       dtype == AQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cudaError_t e = cudaSuccess;
-  if (xmode == 1) {
+  if (xmode == 1 || xmode == 3) {
     const int bw = bt <= Wo ? bt : Wo;
-    e = make_map_nhwc(&maps.x, x, tt, Bn, H, W, Cin, bw, bt / bw);
+    e = make_map_nhwc(&maps.x, x, tt, Bn, H, W, Cin, bw, bt / bw, xmode == 3 ? 64 : 16);
     if (e != cudaSuccess) return e;
   }
   QmmArgs a;
@@ -86,7 +93,10 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
   e = weight_maps(maps, a, w_q, scales, biases, Cout, Kp, bits, gs, AQ_MODE_AFFINE, &fast);
   if (e != cudaSuccess) return e;
   const bool f16 = dtype == AQ_F16;
-  if (xmode == 1) {
+  if (xmode == 3 && fast)
+    return f16 ? by_bits_tc<__half, true, 3>(p, maps, a, bits, 0, st)
+               : by_bits_tc<__nv_bfloat16, true, 3>(p, maps, a, bits, 0, st);
+  if (xmode == 1 || xmode == 3) {
     if (fast) return f16 ? by_bits_tc<__half, true, 1>(p, maps, a, bits, 0, st)
                          : by_bits_tc<__nv_bfloat16, true, 1>(p, maps, a, bits, 0, st);
     return f16 ? by_bits_tc<__half, false, 1>(p, maps, a, bits, 0, st)

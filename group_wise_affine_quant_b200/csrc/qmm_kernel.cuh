@@ -470,7 +470,9 @@ __device__ __forceinline__ uint32_t wchunk_off(int o, int r) {
   return (uint32_t)(r * 128 + ((((o >> 4) & 7) ^ (r & 7)) << 4) + (o & 15));
 }
 
-// XMODE: 0 = dense x by 2-D TMA; 1 = conv pixels by 4-D TMA boxes (one per
+// XMODE: 0 = dense x by 2-D TMA; 3 = conv pixels by one 4-D TMA box of 64
+// channels per K-stage (Cg % 64 == 0, 128-byte swizzle); 1 = conv pixels by
+// 4-D TMA boxes (one per
 // 16-channel atom column of a K-stage, 32-byte swizzle); 2 = conv pixels
 // gathered with cp.async (16-byte granules, zero-filled outside the image).
 template <typename T, int BITS, bool FP4, int BT, bool FAST, int XMODE>
@@ -571,6 +573,33 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
           mbar_arrive_expect_tx(full_b(s), S::kBBytes);
           tma_load_2d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full_b(s),
                       (kt0 + i) * kBK, m0);
+        }
+      }
+    } else if constexpr (XMODE == 3) {
+      // ------------ conv pixels: one 4-D TMA box of 64 channels per K-stage
+      // (every stage is 64 channels of one filter tap when Cg % 64 == 0),
+      // 128-byte swizzle: the same B layout as the dense path
+      if (lane == 0) {
+        const int hw = a.Ho * a.Wo;
+        const int bimg = m0 / hw;
+        const int rem = m0 - bimg * hw;
+        const int ho0 = rem / a.Wo, wo0 = rem - (rem / a.Wo) * a.Wo;
+        const int taps = a.kh * a.kw;
+        for (int i = 0; i < nkt; ++i) {
+          const int s = i % SB;
+          const uint32_t par = ((i / SB) & 1) ^ 1;
+          if (!mbar_wait(empty_b(s), par, abort_flag)) break;
+          mbar_arrive_expect_tx(full_b(s), S::kBBytes);
+          const int kk = (kt0 + i) * kBK;
+          const int tap = kk / a.Cg, c = kk - (kk / a.Cg) * a.Cg;
+          int cx = cgrp * a.Cg + c, cw, ch;
+          if (tap < taps && kk < a.k_real) {
+            cw = wo0 - a.pw + tap % a.kw;
+            ch = ho0 - a.ph + tap / a.kw;
+          } else {
+            cx = 0; cw = 0; ch = a.H;                      // past the image: zero fill
+          }
+          tma_load_4d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full_b(s), cx, cw, ch, bimg);
         }
       }
     } else if constexpr (XMODE == 1) {
@@ -760,7 +789,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         const uint32_t b_addr = smem_u32(ring_b + sb * S::kBBytes);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
-          const uint64_t bdesc = XMODE == 0 ? sdesc_sw128(b_addr + k * 32)
+          const uint64_t bdesc = (XMODE == 0 || XMODE == 3) ? sdesc_sw128(b_addr + k * 32)
                                             : sdesc_sw32(b_addr + k * (BT * 32));
           mma_f16_tmem_a(tmem, a_col + 8 * k, bdesc, idesc, (i > 0 || k > 0) ? 1u : 0u);
         }
@@ -1052,18 +1081,20 @@ cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType typ
 }
 
 // 4-D tensor map over an NHWC activation [Bn, H, W, C] of 2-byte elements,
-// box {16 channels, bw, bh, 1}, 32-byte swizzle, zero fill out of bounds
-// (which supplies the convolution's padding).
+// box {cbox channels, bw, bh, 1}: 16 channels with 32-byte swizzle or 64
+// with 128-byte swizzle; zero fill out of bounds (which supplies the
+// convolution's padding).
 inline cudaError_t make_map_nhwc(CUtensorMap* map, const void* base, CUtensorMapDataType type,
-                                 int Bn, int H, int W, int C, int bw, int bh) {
+                                 int Bn, int H, int W, int C, int bw, int bh, int cbox) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)Bn};
   cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)H * W * C * 2};
-  cuuint32_t box[4] = {16, (cuuint32_t)bw, (cuuint32_t)bh, 1};
+  cuuint32_t box[4] = {(cuuint32_t)cbox, (cuuint32_t)bw, (cuuint32_t)bh, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, type, 4, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   cbox == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }

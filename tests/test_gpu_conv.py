@@ -39,6 +39,9 @@ def _check_full(xd, wq, s, b, y, Cout, k, stride, pad, groups, bits, gs, dt):
     (2, 9, 9, 16, 16, 3, 2, 1, 1),      # stride 2: gather path
     (1, 6, 5, 24, 48, 1, 1, 0, 3),      # 1x1, Cg = 8: gather path
     (1, 10, 10, 16, 200, 3, 1, 0, 1),   # no padding, several weight tiles
+    (1, 8, 8, 64, 64, 3, 1, 1, 1),      # Cg = 64: one 64-channel box per K-stage
+    (2, 8, 16, 128, 96, 3, 1, 1, 2),    # Cg = 64, two conv groups, two images
+    (1, 16, 8, 192, 80, 3, 1, 1, 1),    # Cg = 192, ragged weight tile
 ])
 @pytest.mark.parametrize("bits,gs,dt", [(4, 64, 1), (8, 32, 0), (3, 64, 1)])
 def test_conv_small(B, H, W, Cin, Cout, k, stride, pad, groups, bits, gs, dt):
