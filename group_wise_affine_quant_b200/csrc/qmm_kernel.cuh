@@ -63,14 +63,15 @@ struct QmmShape {
   // CTAs fit on an SM: the next kernel of a stream can then start streaming
   // its weights while this one finishes.  Larger tiles use a deeper pipeline.
   static constexpr bool kLight = BT <= 32;
-  // Operand rings: kStages slots of dequantized A in tensor memory (the
-  // dequantizers refill them from shared memory, no memory latency to hide;
-  // the MMA reads A from TMEM, which keeps the A tile out of the shared-memory
-  // bandwidth) and kBStages slots of x tiles in shared memory (TMA from
-  // L2/HBM; one more slot at BT = 256, where the MMA stage is shortest
-  // relative to a TMA round trip).
+  // Operand stages: K-stage i fills slot i % kStages of both rings, the
+  // dequantized A tile in tensor memory (the dequantizers refill it from
+  // shared memory; the MMA reads A from TMEM, which keeps the A tile out of
+  // the shared-memory bandwidth) and the x tile in shared memory (TMA from
+  // L2/HBM).  One "full" barrier per slot takes the dequantizers' arrivals
+  // and the x tile's, and one MMA commit frees both halves of the slot, so
+  // the MMA issuer waits once and commits once per stage.
   static constexpr int kStages = kLight ? 3 : 4;
-  static constexpr int kBStages = 4;
+  static constexpr int kBStages = kStages;
   static constexpr int kBBytes = BT * kBK * 2;                       // BT * 128
   static constexpr int kPB = 8 * BITS;                               // packed bytes / row / stage
   // cp.async path: one slot per stage, rows at a bank-spreading pitch.
@@ -101,7 +102,7 @@ struct QmmShape {
   static constexpr int kGroups = kLight ? 2 : (kStages < 4 ? kStages : 4);
   static constexpr int kLoaderWarp = kProducerWarp0 + 4 * kGroups;
   static constexpr int kThreads = 32 * (kLoaderWarp + 1);
-  static constexpr int kBars = 2 * kStages + 2 * kBStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
+  static constexpr int kBars = 2 * kStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
   static constexpr int kSmem = 1024 + kDataBytes + 512;             // align slack, barriers
   static_assert(kGroups <= kStages, "parity waits need kGroups <= kStages");
   static_assert(kBars * 8 + 16 <= 512, "barrier area");
@@ -483,8 +484,8 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   constexpr int kDqGroups = S::kGroups;
   constexpr int kLoaderWarp = S::kLoaderWarp;
   constexpr int kThreads = S::kThreads;
-  constexpr int ST = S::kStages;                          // A slots
-  constexpr int SB = S::kBStages;                         // B slots
+  constexpr int ST = S::kStages;                          // operand slots (A and B)
+  constexpr int SB = S::kBStages;                         // == ST
   constexpr int PST = S::kPStages;
   constexpr int WS = S::kWSlots;
   constexpr int SS = S::kSSlots;
@@ -498,7 +499,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   uint8_t* sring = pring + WS * S::kWChunk;               // TMA path: [SS] scale chunks
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kDataBytes);
   constexpr int NL = FAST ? WS + SS : PST;                // loader slots
-  // bars: full_a[ST], empty_a[ST], full_b[SB], empty_b[SB], full_l[NL], empty_l[NL], acc_full
+  // bars: full[ST], empty[ST], full_l[NL], empty_l[NL], acc_full
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -515,13 +516,12 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
   const int nkt = kt1 - kt0;                              // >= 1
   const int G = a.K >> a.gs_log2;
 
-  auto full_a = [&](int s) { return smem_u32(bars + s); };
-  auto empty_a = [&](int s) { return smem_u32(bars + ST + s); };
-  auto full_b = [&](int s) { return smem_u32(bars + 2 * ST + s); };
-  auto empty_b = [&](int s) { return smem_u32(bars + 2 * ST + SB + s); };
-  auto full_l = [&](int s) { return smem_u32(bars + 2 * ST + 2 * SB + s); };
-  auto empty_l = [&](int s) { return smem_u32(bars + 2 * ST + 2 * SB + NL + s); };
-  const uint32_t acc_full = smem_u32(bars + 2 * ST + 2 * SB + 2 * NL);
+  static_assert(SB == ST, "one barrier pair per operand slot");
+  auto full = [&](int s) { return smem_u32(bars + s); };
+  auto empty = [&](int s) { return smem_u32(bars + ST + s); };
+  auto full_l = [&](int s) { return smem_u32(bars + 2 * ST + s); };
+  auto empty_l = [&](int s) { return smem_u32(bars + 2 * ST + NL + s); };
+  const uint32_t acc_full = smem_u32(bars + 2 * ST + 2 * NL);
 
   // TMA path bookkeeping: weight chunk c covers bytes [wb0 + 128 c, +128) of
   // every row, scale chunk j covers groups [SGC j, SGC (j + 1)).
@@ -533,12 +533,10 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
-      mbar_init(full_a(s), 4);          // one arrive per dequantizer warp
-      mbar_init(empty_a(s), 1);         // MMA commit
-    }
-    for (int s = 0; s < SB; ++s) {
-      mbar_init(full_b(s), XMODE == 2 ? 32 : 1);   // TMA arrive + tx, or every gather lane
-      mbar_init(empty_b(s), 1);         // MMA commit
+      // one arrive per dequantizer warp, plus the x tile's: the TMA
+      // producer's arrive (with the tile's bytes as tx), or every gather lane
+      mbar_init(full(s), 4 + (XMODE == 2 ? 32 : 1));
+      mbar_init(empty(s), 1);           // MMA commit
     }
     for (int s = 0; s < NL; ++s) {
       mbar_init(full_l(s), FAST ? 1 : 32);   // TMA arrive + tx, or every loader lane
@@ -569,9 +567,9 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         for (int i = 0; i < nkt; ++i) {
           const int s = i % SB;
           const uint32_t par = ((i / SB) & 1) ^ 1;
-          if (!mbar_wait(empty_b(s), par, abort_flag)) break;
-          mbar_arrive_expect_tx(full_b(s), S::kBBytes);
-          tma_load_2d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full_b(s),
+          if (!mbar_wait(empty(s), par, abort_flag)) break;
+          mbar_arrive_expect_tx(full(s), S::kBBytes);
+          tma_load_2d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full(s),
                       (kt0 + i) * kBK, m0);
         }
       }
@@ -588,8 +586,8 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         for (int i = 0; i < nkt; ++i) {
           const int s = i % SB;
           const uint32_t par = ((i / SB) & 1) ^ 1;
-          if (!mbar_wait(empty_b(s), par, abort_flag)) break;
-          mbar_arrive_expect_tx(full_b(s), S::kBBytes);
+          if (!mbar_wait(empty(s), par, abort_flag)) break;
+          mbar_arrive_expect_tx(full(s), S::kBBytes);
           const int kk = (kt0 + i) * kBK;
           const int tap = kk / a.Cg, c = kk - (kk / a.Cg) * a.Cg;
           int cx = cgrp * a.Cg + c, cw, ch;
@@ -599,7 +597,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
           } else {
             cx = 0; cw = 0; ch = a.H;                      // past the image: zero fill
           }
-          tma_load_4d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full_b(s), cx, cw, ch, bimg);
+          tma_load_4d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full(s), cx, cw, ch, bimg);
         }
       }
     } else if constexpr (XMODE == 1) {
@@ -613,8 +611,8 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         for (int i = 0; i < nkt; ++i) {
           const int s = i % SB;
           const uint32_t par = ((i / SB) & 1) ^ 1;
-          if (!mbar_wait(empty_b(s), par, abort_flag)) break;
-          mbar_arrive_expect_tx(full_b(s), S::kBBytes);
+          if (!mbar_wait(empty(s), par, abort_flag)) break;
+          mbar_arrive_expect_tx(full(s), S::kBBytes);
           const uint32_t dst = smem_u32(ring_b + s * S::kBBytes);
 #pragma unroll
           for (int at = 0; at < 4; ++at) {
@@ -627,7 +625,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
             } else {
               cx = 0; cw = 0; ch = a.H;                    // past the image: zero fill
             }
-            tma_load_4d(dst + at * (BT * 32), &maps.x, full_b(s), cx, cw, ch, bimg);
+            tma_load_4d(dst + at * (BT * 32), &maps.x, full(s), cx, cw, ch, bimg);
           }
         }
       }
@@ -640,7 +638,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
       for (int i = 0; i < nkt; ++i) {
         const int s = i % SB;
         const uint32_t par = ((i / SB) & 1) ^ 1;
-        if (!mbar_wait(empty_b(s), par, abort_flag)) break;
+        if (!mbar_wait(empty(s), par, abort_flag)) break;
         const uint32_t dst = smem_u32(ring_b + s * S::kBBytes);
         for (int idx = lane; idx < BT * 8; idx += 32) {
           const int j = idx >> 3, q = idx & 7;           // pixel row, granule of 8 channels
@@ -665,13 +663,13 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         cp_async_commit();
         if (i - kLagB >= 0) {
           cp_async_wait_group<kLagB>();
-          mbar_arrive(full_b((i - kLagB) % SB));
+          mbar_arrive(full((i - kLagB) % SB));
           published = i - kLagB + 1;
         }
       }
       cp_async_wait_all();
       if (!*abort_flag) {
-        for (int i = published; i < nkt; ++i) mbar_arrive(full_b(i % SB));
+        for (int i = published; i < nkt; ++i) mbar_arrive(full(i % SB));
       }
     }
   } else if (warp == kLoaderWarp) {
@@ -777,29 +775,32 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(std::is_same<T, __nv_bfloat16>::value, kRowsW, BT);
-      for (int i = 0; i < nkt; ++i) {
-        const int s = i % ST, sb = i % SB;
-        if (!(mbar_wait(full_a(s), (i / ST) & 1, abort_flag) &&
-              mbar_wait(full_b(sb), (i / SB) & 1, abort_flag)))
-          break;
-        tc_fence_after();
-        const uint32_t a_col = tmem + S::kACol0 + 32 * s;
-        const uint32_t b_addr = smem_u32(ring_b + sb * S::kBBytes);
+    // The whole warp runs the loop (warp-uniform waits and descriptors); one
+    // elected lane issues the MMAs and the commits.  A single thread issuing
+    // the same sequence spends about twice as long per stage.
+    constexpr uint32_t idesc = idesc_f16(std::is_same<T, __nv_bfloat16>::value, kRowsW, BT);
+    for (int i = 0; i < nkt; ++i) {
+      const int s = i % ST;
+      if (!__all_sync(0xffffffffu, mbar_wait(full(s), (i / ST) & 1, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t a_col = tmem + S::kACol0 + 32 * s;
+      const uint32_t b_addr = smem_u32(ring_b + s * S::kBBytes);
+      if (elect_one()) {
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           const uint64_t bdesc = (XMODE == 0 || XMODE == 3) ? sdesc_sw128(b_addr + k * 32)
                                             : sdesc_sw32(b_addr + k * (BT * 32));
           mma_f16_tmem_a(tmem, a_col + 8 * k, bdesc, idesc, (i > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit(empty_a(s));
-        mma_commit(empty_b(sb));
+        mma_commit(empty(s));                    // frees the A and the x half of slot s
       }
-      // Signals the epilogue once every issued MMA has completed (also on
-      // abort, so nothing is in flight when TMEM is freed).
-      mma_commit(acc_full);
+      __syncwarp();
     }
+    // Signals the epilogue once every issued MMA has completed (also on
+    // abort, so nothing is in flight when TMEM is freed).  The elected lane
+    // is the issuing lane (the lowest lane of the full warp).
+    if (elect_one()) mma_commit(acc_full);
+    __syncwarp();
   } else {
     // ------------------------------------------- dequantizers (warps 2..5)
     const int grp = (warp - kProducerWarp0) >> 2;          // dequantizer group
@@ -951,7 +952,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         if (lane == 0) mbar_arrive(empty_l(ps));
       }
       const int s = i % ST;
-      if (!__all_sync(0xffffffffu, mbar_wait(empty_a(s), ((i / ST) & 1) ^ 1, abort_flag))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(empty(s), ((i / ST) & 1) ^ 1, abort_flag))) break;
       tc_fence_after();
       uint32_t o[32];
       if (row_ok) {
@@ -964,7 +965,7 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(full_a(s));
+      if (lane == 0) mbar_arrive(full(s));
     }
     if constexpr (FAST) {
       // Chunks past this group's last stage are released too.

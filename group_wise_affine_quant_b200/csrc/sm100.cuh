@@ -96,6 +96,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
+// One lane of the (converged, full) warp is elected; the others get false.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(pred));
+  return pred != 0;
+}
+
 // ------------------------------------------------------------ named barriers
 // Barrier `id` (1..15) over `count` threads (a multiple of 32); arrive does
 // not wait.  Non-aligned forms: the threads of a warp may come separately.
