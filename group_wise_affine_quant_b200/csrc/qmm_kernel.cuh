@@ -69,7 +69,8 @@ struct QmmShape {
   // the shared-memory bandwidth) and the x tile in shared memory (TMA from
   // L2/HBM).  One "full" barrier per slot takes the dequantizers' arrivals
   // and the x tile's, and one MMA commit frees both halves of the slot, so
-  // the MMA issuer waits once and commits once per stage.
+  // the MMA issuer waits once and commits once per stage.  (Deeper rings,
+  // 5 slots at BT = 256 and 8 below, measured a few percent slower.)
   static constexpr int kStages = kLight ? 3 : 4;
   static constexpr int kBStages = kStages;
   static constexpr int kBBytes = BT * kBK * 2;                       // BT * 128
@@ -561,71 +562,66 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
 
   if (warp == 0) {
     if (!a.x_early) pdl_wait();                           // x may come from the previous kernel
-    if constexpr (XMODE == 0) {
-      // -------------------------------------------------- TMA producer (x)
-      if (lane == 0) {
-        for (int i = 0; i < nkt; ++i) {
-          const int s = i % SB;
-          const uint32_t par = ((i / SB) & 1) ^ 1;
-          if (!mbar_wait(empty(s), par, abort_flag)) break;
-          mbar_arrive_expect_tx(full(s), S::kBBytes);
-          tma_load_2d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full(s),
-                      (kt0 + i) * kBK, m0);
-        }
-      }
-    } else if constexpr (XMODE == 3) {
-      // ------------ conv pixels: one 4-D TMA box of 64 channels per K-stage
-      // (every stage is 64 channels of one filter tap when Cg % 64 == 0),
-      // 128-byte swizzle: the same B layout as the dense path
-      if (lane == 0) {
+    if constexpr (XMODE != 2) {
+      // ------------------------------------------------- TMA producer (x)
+      // The whole warp runs the loop (warp-uniform waits and coordinates);
+      // one elected lane issues the copies.  Conv coordinates advance
+      // incrementally: (tap, c) is the filter tap and the channel within the
+      // conv group of the stage's first K column, (dy, dx) the tap's offset.
+      //   XMODE 0: x rows [m0, m0 + BT) x K columns [kk, kk + 64), 2-D box;
+      //   XMODE 3: one 64-channel 4-D box (Cg % 64 == 0: one tap per stage);
+      //   XMODE 1: four 16-channel 4-D boxes, one per atom column.
+      int bimg = 0, ho0 = 0, wo0 = 0, taps = 0, tap = 0, c = 0, dy = 0, dx = 0;
+      int kk = kt0 * kBK;
+      if constexpr (XMODE != 0) {
         const int hw = a.Ho * a.Wo;
-        const int bimg = m0 / hw;
+        bimg = m0 / hw;
         const int rem = m0 - bimg * hw;
-        const int ho0 = rem / a.Wo, wo0 = rem - (rem / a.Wo) * a.Wo;
-        const int taps = a.kh * a.kw;
-        for (int i = 0; i < nkt; ++i) {
-          const int s = i % SB;
-          const uint32_t par = ((i / SB) & 1) ^ 1;
-          if (!mbar_wait(empty(s), par, abort_flag)) break;
-          mbar_arrive_expect_tx(full(s), S::kBBytes);
-          const int kk = (kt0 + i) * kBK;
-          const int tap = kk / a.Cg, c = kk - (kk / a.Cg) * a.Cg;
-          int cx = cgrp * a.Cg + c, cw, ch;
-          if (tap < taps && kk < a.k_real) {
-            cw = wo0 - a.pw + tap % a.kw;
-            ch = ho0 - a.ph + tap / a.kw;
-          } else {
-            cx = 0; cw = 0; ch = a.H;                      // past the image: zero fill
-          }
-          tma_load_4d(smem_u32(ring_b + s * S::kBBytes), &maps.x, full(s), cx, cw, ch, bimg);
-        }
+        ho0 = rem / a.Wo;
+        wo0 = rem - ho0 * a.Wo;
+        taps = a.kh * a.kw;
+        tap = kk / a.Cg;
+        c = kk - tap * a.Cg;
+        dy = tap / a.kw;
+        dx = tap - dy * a.kw;
       }
-    } else if constexpr (XMODE == 1) {
-      // ------------------------ conv pixels: one 4-D TMA box per atom column
-      if (lane == 0) {
-        const int hw = a.Ho * a.Wo;
-        const int bimg = m0 / hw;
-        const int rem = m0 - bimg * hw;
-        const int ho0 = rem / a.Wo, wo0 = rem - (rem / a.Wo) * a.Wo;
-        const int taps = a.kh * a.kw;
-        for (int i = 0; i < nkt; ++i) {
-          const int s = i % SB;
-          const uint32_t par = ((i / SB) & 1) ^ 1;
-          if (!mbar_wait(empty(s), par, abort_flag)) break;
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i % SB;
+        const uint32_t par = ((i / SB) & 1) ^ 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(empty(s), par, abort_flag))) break;
+        if (elect_one()) {
           mbar_arrive_expect_tx(full(s), S::kBBytes);
           const uint32_t dst = smem_u32(ring_b + s * S::kBBytes);
+          if constexpr (XMODE == 0) {
+            tma_load_2d(dst, &maps.x, full(s), kk, m0);
+          } else if constexpr (XMODE == 3) {
+            const bool in = tap < taps && kk < a.k_real;   // else past the image: zero fill
+            tma_load_4d(dst, &maps.x, full(s), in ? cgrp * a.Cg + c : 0, in ? wo0 - a.pw + dx : 0,
+                        in ? ho0 - a.ph + dy : a.H, bimg);
+          } else {
+            int t2 = tap, c2 = c, dy2 = dy, dx2 = dx;
 #pragma unroll
-          for (int at = 0; at < 4; ++at) {
-            const int kk = (kt0 + i) * kBK + 16 * at;
-            const int tap = kk / a.Cg, c = kk - (kk / a.Cg) * a.Cg;
-            int cx = cgrp * a.Cg + c, cw, ch;
-            if (tap < taps && kk < a.k_real) {
-              cw = wo0 - a.pw + tap % a.kw;
-              ch = ho0 - a.ph + tap / a.kw;
-            } else {
-              cx = 0; cw = 0; ch = a.H;                    // past the image: zero fill
+            for (int at = 0; at < 4; ++at) {
+              const bool in = t2 < taps && kk + 16 * at < a.k_real;
+              tma_load_4d(dst + at * (BT * 32), &maps.x, full(s), in ? cgrp * a.Cg + c2 : 0,
+                          in ? wo0 - a.pw + dx2 : 0, in ? ho0 - a.ph + dy2 : a.H, bimg);
+              c2 += 16;                                    // Cg % 16 == 0: exact wrap
+              if (c2 >= a.Cg) {
+                c2 = 0;
+                ++t2;
+                if (++dx2 == a.kw) { dx2 = 0; ++dy2; }
+              }
             }
-            tma_load_4d(dst + at * (BT * 32), &maps.x, full(s), cx, cw, ch, bimg);
+          }
+        }
+        __syncwarp();
+        kk += kBK;
+        if constexpr (XMODE != 0) {
+          c += kBK;
+          while (c >= a.Cg) {
+            c -= a.Cg;
+            ++tap;
+            if (++dx == a.kw) { dx = 0; ++dy; }
           }
         }
       }
