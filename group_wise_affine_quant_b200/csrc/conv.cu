@@ -40,8 +40,12 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
     return (bt <= Wo) ? (Wo % bt == 0) : (bt % Wo == 0 && ((int64_t)Ho * Wo) % bt == 0 && bt / Wo <= 256);
   };
   const bool tma_ok = sh == 1 && sw == 1 && Cg % 16 == 0 && Cin % 8 == 0;
+  // The widest pixel tile: a K-stage's dequantization cost is the same at
+  // every tile width and feeds twice the MMA work at 256 pixels as at 128, so
+  // a single wave of wide tiles beats more waves (or K-split tiles) of
+  // narrow ones.  Narrower only when the whole image batch fits one.
   int bt = 256;
-  while (bt > 64 && (int64_t)ntg * groups * ((M + bt - 1) / bt) < sms) bt /= 2;
+  while (bt > 64 && M <= bt / 2) bt /= 2;
   int xmode = 2;
   if (tma_ok) {
     for (int cand = bt; cand >= 64; cand /= 2)

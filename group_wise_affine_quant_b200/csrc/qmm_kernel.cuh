@@ -81,8 +81,12 @@ struct QmmShape {
   static constexpr int kPSlot = kRowsW * kRP + kRowsW * 16;
   // TMA path: weight chunks of 128 rows x 128 bytes (128-byte swizzle) and
   // scale chunks of 128 rows x 16 bytes (scales, then biases).
+  // A chunk slot is refilled only after every group has passed the chunk,
+  // and the refill comes from HBM (a few microseconds): four slots cover 16
+  // K-stages of 4-bit codes (8 of 8-bit), so the refill lands before the
+  // first group reaches it.
   static constexpr int kWChunk = kRowsW * 128;                       // 16 KB
-  static constexpr int kWSlots = kLight ? 2 : BT >= 256 ? 2 : BT >= 128 ? 3 : 4;
+  static constexpr int kWSlots = kLight ? 2 : 4;
   static constexpr int kSChunk = kRowsW * 16 * 2;                    // 4 KB
   static constexpr int kSSlots = kLight ? 2 : 4;
   static constexpr int kLoadBytes = FAST ? kWSlots * kWChunk + kSSlots * kSChunk : kPStages * kPSlot;
