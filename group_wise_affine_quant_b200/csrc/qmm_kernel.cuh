@@ -110,6 +110,7 @@ struct QmmShape {
   static constexpr int kBars = 2 * kStages + 2 * (FAST ? kWSlots + kSSlots : kPStages) + 1;
   static constexpr int kSmem = 1024 + kDataBytes + 512;             // align slack, barriers
   static_assert(kGroups <= kStages, "parity waits need kGroups <= kStages");
+  static_assert(kOpBytes >= 4 * kGroups * 1024, "epilogue staging: 1 KB per dequantizer warp");
   static_assert(kBars * 8 + 16 <= 512, "barrier area");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -141,6 +142,7 @@ struct QmmArgs {
   int weights_early;    // load weights/scales before waiting on the previous kernel
   int x_early;          // read x before waiting on the previous kernel
   int scale_copy;       // TMA path: scale rows are not 16-byte multiples, copy them
+  int y_vec;            // y rows and the group's columns allow 16-byte stores (set at launch)
 };
 
 struct QmmMaps {
@@ -987,7 +989,27 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         uint32_t v[16];
         tmem_ld_16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
         tmem_ld_wait();
-        if (a.splits == 1) {
+        if (a.splits == 1 && a.y_vec) {
+          // Through this warp's 1 KB of the (now idle) operand ring: the 16
+          // columns x 32 rows go in as [column][row] T, and come out as
+          // 16-byte runs of 8 rows, which are contiguous in y.
+          T* stg = reinterpret_cast<T*>(ring) + (warp - kProducerWarp0) * 512;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) stg[j * 32 + lane] = TT<T>::from_f(__uint_as_float(v[j]));
+          __syncwarp();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j = 8 * h + (lane >> 2), part = lane & 3;
+            const int m = m0 + c0 + j;
+            const int nl = nl0 + q * 32 + 8 * part;         // first of the 8 rows, within the group
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + j * 32 + 8 * part);
+            // y_vec implies n_limit % 8 == 0: a run of 8 rows is whole or absent
+            if (m < a.M && nl < a.n_limit)
+              *reinterpret_cast<uint4*>(reinterpret_cast<T*>(a.y) + (int64_t)m * a.ldy +
+                                        (n0 + q * 32 + 8 * part)) = val;
+          }
+          __syncwarp();
+        } else if (a.splits == 1) {
           if (orow_ok) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -1028,9 +1050,20 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
         if (m >= a.M) continue;
         T* yrow = reinterpret_cast<T*>(a.y) + (int64_t)m * a.ldy + n0 + rr;
         const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+        if (a.y_vec && nl0 + rr + 4 <= a.n_limit) {
+          const T o0 = TT<T>::from_f(vals[0]), o1 = TT<T>::from_f(vals[1]);
+          const T o2 = TT<T>::from_f(vals[2]), o3 = TT<T>::from_f(vals[3]);
+          uint2 pk;
+          pk.x = (uint32_t)*reinterpret_cast<const uint16_t*>(&o0) |
+                 ((uint32_t)*reinterpret_cast<const uint16_t*>(&o1) << 16);
+          pk.y = (uint32_t)*reinterpret_cast<const uint16_t*>(&o2) |
+                 ((uint32_t)*reinterpret_cast<const uint16_t*>(&o3) << 16);
+          *reinterpret_cast<uint2*>(yrow) = pk;
+        } else {
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-          if (nl0 + rr + t < a.n_limit) yrow[t] = TT<T>::from_f(vals[t]);
+          for (int t = 0; t < 4; ++t)
+            if (nl0 + rr + t < a.n_limit) yrow[t] = TT<T>::from_f(vals[t]);
+        }
       }
     }
     cluster.sync();
@@ -1120,6 +1153,7 @@ cudaError_t launch_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, c
   for (int part = 0; part < 2; ++part) {
     QmmArgs ap = a;
     ap.nt_all = (int)p.n_tiles;
+    ap.y_vec = a.ldy % 8 == 0 && a.n_limit % 8 == 0 && ((uintptr_t)a.y & 15) == 0;
     int64_t count = tiles;
     if (part == 0) {
       count = p.tiles_main;
