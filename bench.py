@@ -181,6 +181,7 @@ def traffic_for(kernel, workload):
 
 def graph_time_ms(torch, stream, fn, reps, warm=3):
     """Device time per call of fn, captured `reps` times in one CUDA graph."""
+    torch.cuda.synchronize()              # inputs written on other streams are complete
     with torch.cuda.stream(stream):
         fn()
         torch.cuda.synchronize()
@@ -255,8 +256,12 @@ def run_reference(args):
 
 
 def qmm_lines(torch, api, inputs, dev, stream, tf_peak, tf_sust, affine_only=False):
-    """TFLOP/s of the tensor-core workloads (not part of the timed step)."""
+    """TFLOP/s of the tensor-core workloads (not part of the timed step).
+    Every weight here is quantized before its timed calls and no timed kernel
+    writes one, so the kernels may stream weights before their dependency wait
+    (the same setting as the decode step)."""
     out = {}
+    api.aq_set_weight_prefetch(True)
     if affine_only:
         xf = inputs.fp4_x(4096, 4096).to(dev)
         yf = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
