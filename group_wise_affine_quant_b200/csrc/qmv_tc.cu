@@ -224,17 +224,19 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
     }
   } else if (warp == S::kWarpMma) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(std::is_same<T, __nv_bfloat16>::value, kRowsW, 16);
-      for (int j = 0; j < nst; ++j) {
-        const int s = j % AS, sx = j % XS;
-        if (!(mbar_wait(full_a(s), (j / AS) & 1, abort_flag) &&
-              mbar_wait(full_x(sx), (j / XS) & 1, abort_flag)))
-          break;
-        tc_fence_after();
-        const uint32_t a_col = tmem + S::kACol0 + 64 * s;
-        const uint32_t b_addr = smem_u32(xring + sx * S::kXBytes);
-        const int halves = 2 * j + 1 < nkt ? 2 : 1;
+    // The whole warp runs the loop (warp-uniform waits and descriptors); an
+    // elected lane, the same one every stage, issues the MMAs and commits.
+    constexpr uint32_t idesc = idesc_f16(std::is_same<T, __nv_bfloat16>::value, kRowsW, 16);
+    for (int j = 0; j < nst; ++j) {
+      const int s = j % AS, sx = j % XS;
+      if (!__all_sync(0xffffffffu, mbar_wait(full_a(s), (j / AS) & 1, abort_flag) &&
+                                       mbar_wait(full_x(sx), (j / XS) & 1, abort_flag)))
+        break;
+      tc_fence_after();
+      const uint32_t a_col = tmem + S::kACol0 + 64 * s;
+      const uint32_t b_addr = smem_u32(xring + sx * S::kXBytes);
+      const int halves = 2 * j + 1 < nkt ? 2 : 1;
+      if (elect_one()) {
         for (int h = 0; h < halves; ++h) {
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
@@ -245,8 +247,10 @@ qmv_tc_kernel(const __grid_constant__ QmmMaps maps, const DecArgs a) {
         mma_commit(empty_a(s));
         mma_commit(empty_x(sx));
       }
-      mma_commit(acc_full);                               // also on abort: nothing left in flight
+      __syncwarp();
     }
+    if (elect_one()) mma_commit(acc_full);                // also on abort: nothing left in flight
+    __syncwarp();
   } else {
     // ------------------------------------------------------- dequantizers
     // Two groups of four warps take alternate stages; a thread owns one
