@@ -53,9 +53,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-qmm", action="store_true", help="skip the TFLOP/s side lines")
-    ap.add_argument("--only", default="all", choices=["all", "qmm", "qmm-affine"],
+    ap.add_argument("--only", default="all", choices=["all", "qmm", "qmm-affine", "conv"],
                     help="qmm: run only the TFLOP/s workloads; qmm-affine: only the 4-bit "
-                         "affine M = N = K = 4096 product (for profiling)")
+                         "affine M = N = K = 4096 product; conv: only the groups-1 4-bit conv "
+                         "(the last two for profiling)")
     return ap.parse_args()
 
 
@@ -255,13 +256,30 @@ def run_reference(args):
     print(json.dumps(line))
 
 
-def qmm_lines(torch, api, inputs, dev, stream, tf_peak, tf_sust, affine_only=False):
+def qmm_lines(torch, api, inputs, dev, stream, tf_peak, tf_sust, affine_only=False,
+              conv_only=False):
     """TFLOP/s of the tensor-core workloads (not part of the timed step).
     Every weight here is quantized before its timed calls and no timed kernel
     writes one, so the kernels may stream weights before their dependency wait
     (the same setting as the decode step)."""
     out = {}
     api.aq_set_weight_prefetch(True)
+
+    def conv_g1():
+        # conv2d, groups 1, 4-bit: batch 2, 64x64, 320 -> 320 channels, 3x3, pad 1
+        xc, wcv = inputs.conv(1)
+        w2 = inputs.flatten_pad_conv_weight(wcv, 64)
+        qc = api.aq_quantize(w2.to(dev), 4, 64)
+        xcd = xc.to(dev)
+        yc = torch.empty((2, 64, 64, 320), dtype=torch.bfloat16, device=dev)
+        t = graph_time_ms(torch, stream, lambda: api.aq_qconv2d_nhwc(
+            xcd, *qc, 320, 3, 3, (1, 1), (1, 1), 1, 4, 64, out=yc), 10)
+        fl = 2 * 8192 * 320 * 2880
+        out["conv2d_g1_4bit"] = {"tflops": round(fl / (t * 1e-3) / 1e12, 1), "ms": round(t, 4)}
+
+    if conv_only:
+        conv_g1()
+        return out, None
     if affine_only:
         xf = inputs.fp4_x(4096, 4096).to(dev)
         yf = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
@@ -300,16 +318,7 @@ def qmm_lines(torch, api, inputs, dev, stream, tf_peak, tf_sust, affine_only=Fal
     t = graph_time_ms(torch, stream, lambda: api.aq_qmm(xf, *wa, 4, 64, out=yf), 10)
     aff = {"tflops": round(fl / (t * 1e-3) / 1e12, 1), "ms": round(t, 4)}
     out["affine4_M4096"] = aff
-    # conv2d, groups 1, 4-bit
-    xc, wcv = inputs.conv(1)
-    w2 = inputs.flatten_pad_conv_weight(wcv, 64)
-    qc = api.aq_quantize(w2.to(dev), 4, 64)
-    xcd = xc.to(dev)
-    yc = torch.empty((2, 64, 64, 320), dtype=torch.bfloat16, device=dev)
-    t = graph_time_ms(torch, stream, lambda: api.aq_qconv2d_nhwc(
-        xcd, *qc, 320, 3, 3, (1, 1), (1, 1), 1, 4, 64, out=yc), 10)
-    fl = 2 * 8192 * 320 * 2880
-    out["conv2d_g1_4bit"] = {"tflops": round(fl / (t * 1e-3) / 1e12, 1), "ms": round(t, 4)}
+    conv_g1()
     roof = {"bound": "tensor", "achieved": aff["tflops"], "peak": tf_peak, "unit": "TFLOP/s",
             "frac": round(aff["tflops"] / tf_peak, 4), "peak_kind": "measured burst bf16",
             "kernel": "qmm_tc_kernel (aq_qmm, 4-bit affine, M=N=K=4096)",
@@ -328,10 +337,11 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     hbm, tf, tf_sust, peak_kind = peaks()
-    if args.only in ("qmm", "qmm-affine"):
+    if args.only in ("qmm", "qmm-affine", "conv"):
         stream = torch.cuda.Stream(dev)
         qmm, roof_qmm = qmm_lines(torch, api, inputs, dev, stream, tf, tf_sust,
-                                  affine_only=args.only == "qmm-affine")
+                                  affine_only=args.only == "qmm-affine",
+                                  conv_only=args.only == "conv")
         if rank == 0:
             print(json.dumps({"qmm_tflops": qmm, "roofline_qmm": roof_qmm}))
         return
