@@ -42,6 +42,8 @@ def _check_full(xd, wq, s, b, y, Cout, k, stride, pad, groups, bits, gs, dt):
     (1, 8, 8, 64, 64, 3, 1, 1, 1),      # Cg = 64: one 64-channel box per K-stage
     (2, 8, 16, 128, 96, 3, 1, 1, 2),    # Cg = 64, two conv groups, two images
     (1, 16, 8, 192, 80, 3, 1, 1, 1),    # Cg = 192, ragged weight tile
+    (1, 8, 8, 64, 20, 3, 1, 1, 1),      # Cout = 20: rows not a multiple of 8, 2-byte y stores
+    (2, 8, 8, 128, 36, 3, 1, 1, 2),     # Cg = 64, 18 rows per group: 2-byte y stores
 ])
 @pytest.mark.parametrize("bits,gs,dt", [(4, 64, 1), (8, 32, 0), (3, 64, 1)])
 def test_conv_small(B, H, W, Cin, Cout, k, stride, pad, groups, bits, gs, dt):
