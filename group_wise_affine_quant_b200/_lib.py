@@ -38,6 +38,19 @@ SIGNATURES = {
     "aq_get_input_prefetch": (_I, []),
 }
 
+
+
+class QmvProblem(ctypes.Structure):
+    """aq_qmv_problem (include/aq.h)."""
+    _fields_ = [("x", _P), ("w_q", _P), ("scales", _P), ("biases", _P), ("y", _P),
+                ("N", _I64), ("K", _I64)]
+
+
+SIGNATURES["aq_qmv_batched"] = (_I, [ctypes.POINTER(QmvProblem), _I, _I64, _I, _I, _I, _I, _P,
+                                     _SZ, _P])
+SIGNATURES["aq_qmv_batched_workspace_size"] = (_SZ, [ctypes.POINTER(QmvProblem), _I, _I64, _I,
+                                                     _I, _I])
+
 _lib = None
 
 

@@ -12,7 +12,7 @@ from . import _lib
 from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, AQ_OP_QMM,
                    AQ_OP_QMV, AqError, check, lib)
 
-__all__ = ["aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmm", "aq_qconv2d_nhwc",
+__all__ = ["aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_qconv2d_nhwc",
            "aq_workspace_size", "aq_last_error", "aq_set_weight_prefetch",
            "aq_get_weight_prefetch", "aq_set_input_prefetch", "aq_get_input_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
 
@@ -41,8 +41,10 @@ def _mode(scales):
 
 class Workspace:
     """Per-device zero-initialised scratch buffer for the ABI's workspace
-    argument, grown on demand.  The current kernels report a workspace size of
-    0 (split-K reduces inside thread block clusters), so none is allocated."""
+    argument, grown on demand (a grown buffer is zero-filled again).  The
+    tensor-core qmv kernels keep split-K partials and counters there and leave
+    it zero-filled after every call; one Workspace serves calls issued on one
+    stream at a time."""
 
     def __init__(self):
         self._bufs = {}
@@ -131,6 +133,33 @@ def _mm(fn_name, op, x, w_q, scales, biases, bits, group_size, out, workspace):
 def aq_qmv(x, w_q, scales, biases, bits=4, group_size=64, out=None, workspace=None):
     """y = x . dequant(w)^T for 1 <= M <= 16 rows of x."""
     return _mm("aq_qmv", AQ_OP_QMV, x, w_q, scales, biases, bits, group_size, out, workspace)
+
+
+def aq_qmv_batched(xs, w_qs, scales, biases, bits=4, group_size=64, outs=None, workspace=None):
+    """Independent problems y_i = x_i . dequant(w_i)^T (all x_i with the same
+    M <= 16, one dtype, one format) in one call; biases is a list (or None for
+    FP4).  Returns the list of outputs."""
+    n = len(xs)
+    if not (len(w_qs) == len(scales) == n) or (biases is not None and len(biases) != n):
+        raise ValueError("one w_q, scales (and biases) per x")
+    if n == 0:
+        return []
+    M = xs[0].shape[0]
+    mode = _mode(scales[0])
+    if outs is None:
+        outs = [torch.empty((M, w.shape[0]), dtype=x.dtype, device=x.device) for x, w in zip(xs, w_qs)]
+    arr = (_lib.QmvProblem * n)()
+    for i in range(n):
+        arr[i] = _lib.QmvProblem(_ptr(xs[i]), _ptr(w_qs[i]), _ptr(scales[i]),
+                                 None if biases is None else _ptr(biases[i]), _ptr(outs[i]),
+                                 w_qs[i].shape[0], xs[i].shape[1])
+    L = lib()
+    ws_bytes = L.aq_qmv_batched_workspace_size(arr, n, M, bits, group_size, mode)
+    ws = (workspace or _default_ws).get(xs[0].device, ws_bytes)
+    check(L.aq_qmv_batched(arr, n, M, bits, group_size, mode, _dt(xs[0]), _ptr(ws),
+                           0 if ws is None else ws.numel(), _stream(xs[0].device)),
+          "aq_qmv_batched")
+    return outs
 
 
 def aq_qmm(x, w_q, scales, biases, bits=4, group_size=64, out=None, workspace=None):

@@ -4,7 +4,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
-#include <atomic>
+#include <vector>
 
 #include "common.cuh"
 
@@ -28,8 +28,6 @@ aq_status cuda_status(cudaError_t e, const char* what) {
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
 const int64_t kMaxDim = (int64_t(1) << 31) - 1;
-// aq_qmv runs the fp32 weight-streaming kernel up to this many rows of x.
-const int64_t kQmvSimtMaxM = 2;
 
 // Format checks shared by every entry point.
 aq_status check_format(int bits, int gs, aq_mode mode, aq_dtype dt) {
@@ -73,26 +71,23 @@ aq_status check_weight(const void* w_q, const void* scales, const void* biases, 
 }  // namespace
 
 namespace {
-std::atomic<int> g_weight_prefetch{0};
-std::atomic<int> g_input_prefetch{0};
+// Per calling thread: one component's setting never reaches another's calls.
+thread_local int g_weight_prefetch = 0;
+thread_local int g_input_prefetch = 0;
 }
 
-int aq::weight_prefetch_enabled() { return g_weight_prefetch.load(std::memory_order_relaxed); }
-int aq::input_prefetch_enabled() { return g_input_prefetch.load(std::memory_order_relaxed); }
+int aq::weight_prefetch_enabled() { return g_weight_prefetch; }
+int aq::input_prefetch_enabled() { return g_input_prefetch; }
 
 extern "C" {
 
 const char* aq_last_error(void) { return g_err; }
 
-void aq_set_weight_prefetch(int enable) {
-  g_weight_prefetch.store(enable ? 1 : 0, std::memory_order_relaxed);
-}
+void aq_set_weight_prefetch(int enable) { g_weight_prefetch = enable ? 1 : 0; }
 
 int aq_get_weight_prefetch(void) { return aq::weight_prefetch_enabled(); }
 
-void aq_set_input_prefetch(int enable) {
-  g_input_prefetch.store(enable ? 1 : 0, std::memory_order_relaxed);
-}
+void aq_set_input_prefetch(int enable) { g_input_prefetch = enable ? 1 : 0; }
 
 int aq_get_input_prefetch(void) { return aq::input_prefetch_enabled(); }
 
@@ -138,6 +133,15 @@ static aq_status check_mm(const void* x, const void* y, int64_t M, int64_t N, in
   return AQ_OK;
 }
 
+static aq_status check_workspace(const void* ws, size_t bytes, size_t need) {
+  if (need == 0) return AQ_OK;
+  if (!ws || bytes < need)
+    return fail(AQ_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu%s)", need, bytes,
+                ws ? "" : ", NULL");
+  if (!aligned(ws, 256)) return fail(AQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  return AQ_OK;
+}
+
 static aq_status zero_output(void* y, int64_t M, int64_t N, aq_stream_t stream) {
   // K == 0: the empty sum is +0 in every output.
   return cuda_status(cudaMemsetAsync(y, 0, (size_t)(M * N) * 2, (cudaStream_t)stream),
@@ -155,25 +159,77 @@ aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void*
   if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
   if (N == 0) return AQ_OK;
   if (K == 0) return zero_output(y, M, N, stream);
-  // The tensor-core decode kernel dequantizes each code once for all rows of
-  // x and costs fewer instructions per code than fp32 FMAs even for one row;
-  // it takes every shape whose packed rows and scale rows are 16-byte
-  // multiples.  Other shapes: the fp32 kernel for one or two rows, the
-  // general tensor-core kernel beyond.
-  if (aq::qmv_tc_applies(M, N, K, bits, group_size, mode, scales, biases))
+  // The tensor-core decode kernel takes every shape whose packed rows and
+  // scale rows are 16-byte multiples (TMA); other shapes run the fp32
+  // CUDA-core kernel.  Both keep w_hat in fp32 (scale and bias per group).
+  if (aq::qmv_tc_applies(M, N, K, bits, group_size, mode, scales, biases)) {
+    const size_t need = aq::qmv_tc_workspace(M, N, K, bits, group_size);
+    if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
     return cuda_status(aq::launch_qmv_tc(x, w_q, scales, biases, y, M, N, K, bits, group_size,
-                                         mode, dtype, (cudaStream_t)stream),
-                       "aq_qmv launch");
-  if (M > kQmvSimtMaxM) {
-    const aq::QmmPlan p = aq::plan_qmm(M, N, K, bits, group_size, mode);
-    return cuda_status(aq::launch_qmm(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
-                                      mode, dtype, (cudaStream_t)stream),
+                                         mode, dtype, workspace, (cudaStream_t)stream),
                        "aq_qmv launch");
   }
   const aq::QmvPlan p = aq::plan_qmv(M, N, K, bits, group_size, mode);
   return cuda_status(aq::launch_qmv(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
                                     mode, dtype, workspace, (cudaStream_t)stream),
                      "aq_qmv launch");
+}
+
+static aq_status check_batch(const aq_qmv_problem* problems, int count, int64_t M, int bits,
+                             int group_size, aq_mode mode, aq_dtype dtype) {
+  aq_status st = check_format(bits, group_size, mode, dtype);
+  if (st != AQ_OK) return st;
+  if (count < 0) return fail(AQ_ERR_INVALID_ARG, "count=%d is negative", count);
+  if (count > 0 && !problems) return fail(AQ_ERR_INVALID_ARG, "problems must not be NULL");
+  if (M < 1 || M > 16) return fail(AQ_ERR_INVALID_ARG, "aq_qmv_batched takes 1 <= M <= 16 (got %lld)", (long long)M);
+  for (int i = 0; i < count; ++i) {
+    const aq_qmv_problem& q = problems[i];
+    st = check_weight(q.w_q, q.scales, q.biases, q.N, q.K, bits, group_size, mode, dtype);
+    if (st == AQ_OK) st = check_mm(q.x, q.y, M, q.N, q.K);
+    if (st != AQ_OK) {
+      char msg[640];
+      snprintf(msg, sizeof(msg), "problem %d: %s", i, g_err);
+      return fail(st, "%s", msg);
+    }
+    if (q.N == 0 || q.K == 0)
+      return fail(AQ_ERR_INVALID_ARG, "problem %d: N and K must be positive", i);
+    if (!aq::qmv_tc_applies(M, q.N, q.K, bits, group_size, mode, q.scales, q.biases))
+      return fail(AQ_ERR_UNSUPPORTED,
+                  "problem %d: packed rows and scale rows must be 16-byte multiples and scales / "
+                  "biases 16-byte aligned (use aq_qmv for this shape)", i);
+  }
+  return AQ_OK;
+}
+
+aq_status aq_qmv_batched(const aq_qmv_problem* problems, int count, int64_t M, int bits,
+                         int group_size, aq_mode mode, aq_dtype dtype, void* workspace,
+                         size_t workspace_bytes, aq_stream_t stream) {
+  g_err[0] = 0;
+  aq_status st = check_batch(problems, count, M, bits, group_size, mode, dtype);
+  if (st != AQ_OK) return st;
+  if (count == 0) return AQ_OK;
+  std::vector<aq::QmvProblemDesc> d((size_t)count);
+  for (int i = 0; i < count; ++i)
+    d[(size_t)i] = {problems[i].x, problems[i].w_q, problems[i].scales, problems[i].biases,
+                    problems[i].y, problems[i].N, problems[i].K};
+  const size_t need = aq::qmv_tc_batched_workspace(d.data(), count, M, bits, group_size);
+  if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
+  return cuda_status(aq::launch_qmv_tc_batched(d.data(), count, M, bits, group_size, mode, dtype,
+                                               workspace, (cudaStream_t)stream),
+                     "aq_qmv_batched launch");
+}
+
+size_t aq_qmv_batched_workspace_size(const aq_qmv_problem* problems, int count, int64_t M,
+                                     int bits, int group_size, aq_mode mode) {
+  if (!problems || count <= 0 || M < 1 || M > 16 || group_size <= 0) return 0;
+  std::vector<aq::QmvProblemDesc> d;
+  for (int i = 0; i < count; ++i) {
+    if (problems[i].N <= 0 || problems[i].K <= 0 || problems[i].K % group_size) return 0;
+    if (!aq::qmv_tc_shape_ok(problems[i].N, problems[i].K, bits, group_size, mode)) continue;
+    d.push_back({problems[i].x, problems[i].w_q, problems[i].scales, problems[i].biases,
+                 problems[i].y, problems[i].N, problems[i].K});
+  }
+  return d.empty() ? 0 : aq::qmv_tc_batched_workspace(d.data(), (int)d.size(), M, bits, group_size);
 }
 
 aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void* biases,
@@ -246,6 +302,8 @@ size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, in
   if (M <= 0 || N <= 0 || K <= 0 || group_size <= 0 || K % group_size) return 0;
   if (op == AQ_OP_QMV) {
     if (M > 16) return 0;
+    if (aq::qmv_tc_shape_ok(N, K, bits, group_size, mode))
+      return aq::qmv_tc_workspace(M, N, K, bits, group_size);
     return aq::plan_qmv(M, N, K, bits, group_size, mode).ws_bytes;
   }
   return 0;

@@ -126,12 +126,29 @@ cudaError_t launch_qconv(const void* x, const void* w_q, const void* scales, con
                          cudaStream_t st);
 cudaError_t read_device_error_qmm(unsigned* out);
 // Tensor-core decode path for 1 <= M <= 16 (qmv_tc.cu): applies when the
-// packed rows and the scale rows are 16-byte multiples (TMA chunks).
+// packed rows and the scale rows are 16-byte multiples (TMA chunks) and the
+// scales / biases are 16-byte aligned.
+constexpr int64_t kMaxRowsDec = (int64_t)1 << 24;      // N and K limit of the decode kernel
+constexpr int64_t kDecUnitBytes = 128 * 1024;          // packed bytes per unit, batched launches
+struct QmvProblemDesc {
+  const void* x;
+  const void* w_q;
+  const void* scales;
+  const void* biases;
+  void* y;
+  int64_t N, K;
+};
+bool qmv_tc_shape_ok(int64_t N, int64_t K, int bits, int gs, int mode);
 bool qmv_tc_applies(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode,
                     const void* scales, const void* biases);
+size_t qmv_tc_workspace(int64_t M, int64_t N, int64_t K, int bits, int gs);
+size_t qmv_tc_batched_workspace(const QmvProblemDesc* probs, int count, int64_t M, int bits,
+                                int gs);
 cudaError_t launch_qmv_tc(const void* x, const void* w_q, const void* scales, const void* biases,
                           void* y, int64_t M, int64_t N, int64_t K, int bits, int gs, int mode,
-                          int dtype, cudaStream_t st);
+                          int dtype, void* ws, cudaStream_t st);
+cudaError_t launch_qmv_tc_batched(const QmvProblemDesc* probs, int count, int64_t M, int bits,
+                                  int gs, int mode, int dtype, void* ws, cudaStream_t st);
 cudaError_t read_device_error_qmv_tc(unsigned* out);
 // aq_set_weight_prefetch's process-wide setting (0 or 1).
 int weight_prefetch_enabled();

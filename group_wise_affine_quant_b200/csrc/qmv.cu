@@ -297,8 +297,13 @@ template <typename T, int BITS, bool FP4>
 cudaError_t by_mt(const QmvPlan& p, const void* x, const void* w_q, const void* scales,
                   const void* biases, void* y, int64_t M, int64_t N, int64_t K, int gs,
                   cudaStream_t st) {
-  if (p.mt == 1) return launch_one<T, BITS, 1, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
-  return launch_one<T, BITS, 2, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+  switch (p.mt) {
+    case 1: return launch_one<T, BITS, 1, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 2: return launch_one<T, BITS, 2, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 4: return launch_one<T, BITS, 4, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    case 8: return launch_one<T, BITS, 8, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+    default: return launch_one<T, BITS, 16, FP4>(p, x, w_q, scales, biases, y, M, N, K, gs, st);
+  }
 }
 
 template <typename T>
@@ -322,7 +327,7 @@ cudaError_t by_bits(const QmvPlan& p, const void* x, const void* w_q, const void
 QmvPlan plan_qmv(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode) {
   (void)bits; (void)gs; (void)mode;
   QmvPlan p{};
-  p.mt = M <= 1 ? 1 : 2;          // aq_qmv sends M > 2 to the tensor-core kernel
+  p.mt = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
   const int64_t units = K / kUnit;
   // Shared memory per staged unit and row of x: 36 floats + 1 sum.
   const int64_t smem_cap = 160 * 1024;

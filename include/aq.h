@@ -109,17 +109,27 @@ AQ_API aq_status aq_dequantize(const void* w_q, const void* scales, const void* 
 
 /*
  * aq_qmv — y = x . w_hat^T for small M (1 <= M <= 16): the weight-streaming
- * path ("Add the 3bit packed qmm_t", affine_packed_qmv_fast, routed for few
- * rows of x).  x [M, K] T, y [M, N] T, fp32 accumulation.  When the
- * packed rows (K * bits / 8 bytes) and the rows of scales (K / group_size
- * elements) are 16-byte multiples and scales / biases are 16-byte aligned, a
- * tensor-core decode kernel: each code is dequantized once into T (the value
- * aq_dequantize writes) in tensor memory and multiplied with all rows of x.
- * Other shapes: for M <= 2 an fp32 CUDA-core kernel with the scale and bias
- * hoisted out of each group's dot product (w_hat never rounded), for M >= 3
- * the tensor-core kernel of aq_qmm.  K-slices are reduced inside a thread
- * block cluster, so no workspace is needed (aq_workspace_size returns 0;
- * workspace may be NULL and is not touched).
+ * path ("Add the 3bit packed qmm_t", affine_packed_qmv_fast, which keeps the
+ * dot product in fp32 and hoists scale and bias out of each group).
+ *   x [M, K] T, y [M, N] T.  For every output
+ *     y[m, n] = sum_g ( s[n,g] * P[g] + b[n,g] * X[g] ),
+ *     P[g] = sum_{k in g} q[n,k] x[m,k],  X[g] = sum_{k in g} x[m,k],
+ *   in fp32, with s and b (or the FP4 scale in T) applied in fp32: w_hat is
+ *   never rounded to T.
+ * When the packed rows (K * bits / 8 bytes) and the rows of scales (K /
+ * group_size elements) are 16-byte multiples and scales / biases are
+ * 16-byte aligned, the products P and the sums X come from tcgen05 tensor-
+ * core MMAs over the exact integer codes, and K may be split over several
+ * CTAs whose fp32 partials meet in `workspace`; other shapes run an fp32
+ * CUDA-core kernel that needs no workspace.
+ * Workspace: aq_workspace_size(AQ_OP_QMV, M, N, K, bits, group_size, mode,
+ * 1) bytes, 256-byte aligned, ZERO-FILLED before its first use.  Its first
+ * 65536 bytes hold per-tile counters that every call which completes leaves
+ * zero again; the rest holds fp32 partial sums that each call writes before
+ * it reads them.  So one buffer serves any sequence of calls on one stream;
+ * calls that may run at the same time (other streams) need separate
+ * buffers.  After a device error (aq_device_errors() != 0) zero it again.
+ * Returns AQ_ERR_WORKSPACE when a needed workspace is NULL or too small.
  * Returns AQ_ERR_INVALID_ARG for M outside 1..16.
  */
 AQ_API aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void* biases,
@@ -127,12 +137,45 @@ AQ_API aq_status aq_qmv(const void* x, const void* w_q, const void* scales, cons
                  aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
                  aq_stream_t stream);
 
+/* One problem of aq_qmv_batched: y [M, N] = x [M, K] . dequant(w)^T. */
+typedef struct aq_qmv_problem {
+  const void* x;        /* [M, K] T */
+  const void* w_q;      /* [N, K*bits/8] packed codes */
+  const void* scales;   /* [N, K/group_size] */
+  const void* biases;   /* [N, K/group_size] T (affine), NULL (FP4) */
+  void* y;              /* [M, N] T */
+  int64_t N, K;
+} aq_qmv_problem;
+
+/*
+ * aq_qmv_batched — `count` independent aq_qmv problems that share M, bits,
+ * group_size, mode and dtype (e.g. the projections of a decode step, or the
+ * experts selected for a batch), computed by persistent CTAs that stream the
+ * weights of all of them back to back: one launch per 40 problems instead of
+ * one per problem.  Each problem's result is the one aq_qmv defines (same
+ * fp32 arithmetic).  `problems` is a host array read before the call
+ * returns.  Every problem must satisfy the tensor-core conditions of aq_qmv
+ * (16-byte packed and scale rows, 16-byte aligned scales / biases, N, K > 0),
+ * else AQ_ERR_UNSUPPORTED names it.  Workspace as aq_qmv, sized by
+ * aq_qmv_batched_workspace_size.  Outputs must not overlap one another or any
+ * input.
+ */
+AQ_API aq_status aq_qmv_batched(const aq_qmv_problem* problems, int count, int64_t M, int bits,
+                                int group_size, aq_mode mode, aq_dtype dtype, void* workspace,
+                                size_t workspace_bytes, aq_stream_t stream);
+
+/* Workspace bytes aq_qmv_batched needs for these problems (0 if none). */
+AQ_API size_t aq_qmv_batched_workspace_size(const aq_qmv_problem* problems, int count,
+                                            int64_t M, int bits, int group_size, aq_mode mode);
+
 /*
  * aq_qmm — y = x . w_hat^T for any M >= 1 ("Add the 3bit packed qmm_t",
- * affine_packed_qmm_t): weight tiles are dequantized into shared memory in T
- * (the values aq_dequantize writes) and multiplied on the tensor cores
- * (tcgen05, fp32 accumulation in tensor memory).  Arguments as aq_qmv; M may
- * be any size.  Needs no workspace (workspace may be NULL).
+ * affine_packed_qmm_t): each weight tile is dequantized once into T (the
+ * values aq_dequantize writes), stored in tensor memory as the A operand of
+ * tcgen05 MMAs whose B operand is the x tile (TMA, shared memory), with fp32
+ * accumulation in tensor memory.  Arguments as aq_qmv; M may be any size.
+ * Needs no workspace (K-splits reduce inside a thread block cluster;
+ * workspace may be NULL).
  */
 AQ_API aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void* biases,
                  void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
@@ -178,28 +221,30 @@ AQ_API size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int b
 AQ_API unsigned aq_device_errors(void);
 
 /*
- * Weight prefetch across kernel boundaries (process-wide, default 0 = off).
+ * Weight prefetch across kernel boundaries (a setting of the CALLING THREAD,
+ * default 0 = off; it affects only the calls this thread makes afterwards).
  * Every qmv / qmm / conv kernel is launched with programmatic dependent
  * launch, so it may start while the previous kernel on its stream is still
- * running; it always waits for that kernel before reading x or writing y.
- * With prefetch on, it also streams w_q, scales and biases before that wait,
- * which hides most of a small matmul's start-up behind the previous kernel.
- * Turn it on only when no kernel launched just before a matmul on the same
- * stream writes that matmul's weights (e.g. not directly after aq_quantize
- * of the same weights without a synchronising operation in between).
+ * running; it always waits for that kernel before reading x or writing y
+ * and the workspace.  With prefetch on, it also streams w_q, scales and
+ * biases before that wait, which hides most of a small matmul's start-up
+ * behind the previous kernel.  Turn it on only when no kernel launched just
+ * before a matmul on the same stream writes that matmul's weights (e.g. not
+ * directly after aq_quantize of the same weights without a synchronising
+ * operation in between).
  */
 AQ_API void aq_set_weight_prefetch(int enable);
 AQ_API int aq_get_weight_prefetch(void);
 
 /*
- * Input prefetch (process-wide, default 0 = off).  With it on, a matmul that
- * starts while the previous kernel on its stream is still running also
- * reads x before waiting for that kernel; it still waits before writing y,
- * so y is ordered after everything earlier on the stream.  Turn it on only
- * when no kernel that may still be running when a matmul starts writes that
- * matmul's x: for instance calls whose x were all written before the first
- * of them was launched (projections that share an input, experts of one
- * batch, a sweep over fixed activations).
+ * Input prefetch (a setting of the calling thread, default 0 = off).  With
+ * it on, a matmul that starts while the previous kernel on its stream is
+ * still running also reads x before waiting for that kernel; it still waits
+ * before writing y, so y is ordered after everything earlier on the stream.
+ * Turn it on only when no kernel that may still be running when a matmul
+ * starts writes that matmul's x: for instance calls whose x were all written
+ * before the first of them was launched (projections that share an input,
+ * experts of one batch, a sweep over fixed activations).
  */
 AQ_API void aq_set_input_prefetch(int enable);
 AQ_API int aq_get_input_prefetch(void);

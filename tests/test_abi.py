@@ -66,12 +66,74 @@ def test_alignment_errors():
     assert _qmv(s=A + 1) == MISALIGNED
 
 
-def test_qmv_needs_no_workspace():
-    """qmv reduces its K-slices inside a thread block cluster: no workspace."""
-    for M in (1, 7, 16):
-        for K in (64, 16384, 1 << 20):
-            assert L().aq_workspace_size(0, M, 4096, K, 4, 64, 0, 1) == 0
-    assert L().aq_workspace_size(0, 1, 64, 0, 4, 64, 0, 1) == 0
+def test_qmv_workspace_sizes():
+    """The tensor-core qmv splits K through the workspace when a row tile's
+    K is long enough to split; shapes it does not take need none."""
+    ws = lambda M, N, K, bits=4, gs=64, mode=0: L().aq_workspace_size(0, M, N, K, bits, gs, mode, 1)
+    assert ws(16, 2048, 8192) > 0                     # 16 row tiles, K split over slices
+    assert ws(1, 2048, 8192) < ws(16, 2048, 8192)     # partials scale with M
+    assert ws(1, 64, 0) == 0
+    assert ws(1, 4096, 64) == 0                       # one 64-column stage: no split
+    assert ws(4, 40, 96, 4, 32) == 0                  # scale rows of 6 bytes: fp32 kernel
+    assert ws(17, 2048, 8192) == 0                    # not a qmv size
+    # a too-small workspace is refused before anything is launched
+    assert _qmv(M=16, N=2048, K=8192, ws=None, wsb=0) == WORKSPACE
+    assert _qmv(M=16, N=2048, K=8192, ws=A, wsb=16) == WORKSPACE
+    assert _qmv(M=16, N=2048, K=8192, ws=A + 16, wsb=1 << 30) == MISALIGNED
+
+
+def _problems(n, **kw):
+    arr = (_lib.QmvProblem * n)()
+    for i in range(n):
+        f = dict(x=A, w_q=A, scales=A, biases=A, y=A, N=256, K=2048)
+        f.update(kw)
+        arr[i] = _lib.QmvProblem(f["x"], f["w_q"], f["scales"], f["biases"], f["y"], f["N"], f["K"])
+    return arr
+
+
+def test_qmv_batched_validation():
+    b = L().aq_qmv_batched
+    assert b(None, 0, 1, 4, 64, 0, 1, None, 0, None) == OK               # nothing to do
+    assert b(None, 2, 1, 4, 64, 0, 1, None, 0, None) == INVALID
+    assert b(_problems(2), 2, 0, 4, 64, 0, 1, A, 1 << 30, None) == INVALID   # M = 0
+    assert b(_problems(2), 2, 17, 4, 64, 0, 1, A, 1 << 30, None) == INVALID
+    assert b(_problems(2), 2, 1, 7, 64, 0, 1, A, 1 << 30, None) == UNSUPPORTED
+    assert b(_problems(2, y=A + 2), 2, 1, 4, 64, 0, 1, A, 1 << 30, None) == MISALIGNED
+    assert b"problem 0" in L().aq_last_error()
+    assert b(_problems(2, K=96), 2, 1, 4, 32, 0, 1, A, 1 << 30, None) == UNSUPPORTED
+    assert b(_problems(2, N=0), 2, 1, 4, 64, 0, 1, A, 1 << 30, None) == INVALID
+    assert b(_problems(1, scales=A + 2), 1, 1, 4, 64, 0, 1, A, 1 << 30, None) == UNSUPPORTED
+    # workspace: sized for the batch, refused when missing
+    p = _problems(3, N=2048, K=8192)
+    need = L().aq_qmv_batched_workspace_size(p, 3, 16, 4, 64, 0)
+    assert need > 0
+    assert b(p, 3, 16, 4, 64, 0, 1, None, 0, None) == WORKSPACE
+    assert L().aq_qmv_batched_workspace_size(_problems(3), 3, 16, 4, 64, 0) == 0   # K = 2048: one unit per tile
+
+
+def test_prefetch_settings_are_per_thread():
+    """aq_set_weight_prefetch / aq_set_input_prefetch change only the calling
+    thread's later calls: another thread still sees the default."""
+    import threading
+    seen = {}
+
+    def other():
+        seen["w"] = L().aq_get_weight_prefetch()
+        seen["x"] = L().aq_get_input_prefetch()
+        L().aq_set_input_prefetch(1)
+        seen["x_after"] = L().aq_get_input_prefetch()
+
+    L().aq_set_weight_prefetch(1)
+    L().aq_set_input_prefetch(0)
+    try:
+        t = threading.Thread(target=other)
+        t.start()
+        t.join()
+        assert seen == {"w": 0, "x": 0, "x_after": 1}
+        assert L().aq_get_weight_prefetch() == 1
+        assert L().aq_get_input_prefetch() == 0       # the other thread's setting stayed there
+    finally:
+        L().aq_set_weight_prefetch(0)
 
 
 def test_quantize_validation():

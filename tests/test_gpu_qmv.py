@@ -1,10 +1,8 @@
-"""GPU parity for aq_qmv against the oracle, within
-|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref).
-
-aq_qmv's tensor-core kernels multiply weight tiles rounded to T (checked
-against the product over w_hat rounded to T); its fp32 kernel, used for M <= 2
-on shapes the tensor-core decode kernel does not take, keeps w_hat in fp32
-(checked against the exact product)."""
+"""GPU parity for aq_qmv and aq_qmv_batched against the oracle, within
+|y - y_ref| <= 2e-3 * sum_k |x_k w_hat_k| + 1 ulp_T(y_ref), where y_ref is the
+oracle's fp64 product over the EXACT w_hat = s q + b (LUT q * s_T for FP4):
+every aq_qmv kernel applies scale and bias in fp32 and never rounds w_hat to
+T, for every M from 1 to 16."""
 import numpy as np
 import pytest
 import torch
@@ -147,3 +145,104 @@ def test_qmv_k_zero_and_n_zero():
     wq = torch.zeros((0, 32), dtype=torch.uint8, device=DEV)
     s = torch.zeros((0, 1), dtype=torch.float16, device=DEV)
     api.aq_qmv(x, wq, s, s, 4, 64)
+
+
+@pytest.mark.parametrize("gs,scale_range", [(32, "finite"), (16, "finite"), (32, "literal"),
+                                            (16, "literal")])
+@pytest.mark.parametrize("M", [1, 16])
+def test_qmv_fp4_full_size(gs, scale_range, M):
+    """FP4 weights at full size, K = N = 4096: E8M0 (group 32) and E4M3
+    (group 16) scales over the finite and the literal ranges."""
+    N = K = 4096
+    codes, scales = inputs.fp4(N, K, gs, scale_range=scale_range, seed=11 + gs + M)
+    x = inputs.fp4_x(M, K)
+    xd, wq, sc = to_dev(x), codes.to(DEV), scales.to(DEV)
+    y = api.aq_qmv(xd, wq, sc, None, 4, gs)
+    torch.cuda.synchronize()
+    _check(xd, wq, sc, None, y, 4, gs, 1, mode=1,
+           overflow_any_nonfinite=scale_range == "literal")
+
+
+@pytest.mark.parametrize("M", [1, 3, 16])
+@pytest.mark.parametrize("bits", BITS)
+def test_qmv_batched_matches_single(M, bits):
+    """A batch of problems of different shapes (N not a multiple of 128,
+    long K that splits) in one call: every output equals the single-problem
+    call bit for bit (same fp32 arithmetic, same slice order) and is within
+    the bound of the oracle."""
+    gs = 64 if bits != 6 else 128
+    dt = 1 if M % 2 else 0
+    shapes = [(200, 1024), (512, 2048), (72, 4096), (128, 8192), (1000, 1024)]
+    cases = [_case(M, n, k, bits, gs, dt, seed=100 * i + bits + M) for i, (n, k) in enumerate(shapes)]
+    xs = [c[0] for c in cases]
+    ys = api.aq_qmv_batched(xs, [c[1] for c in cases], [c[2] for c in cases],
+                            [c[3] for c in cases], bits, gs)
+    torch.cuda.synchronize()
+    assert api.lib().aq_device_errors() == 0
+    for (x, wq, s, b), y in zip(cases, ys):
+        _check(x, wq, s, b, y, bits, gs, dt)
+
+
+@pytest.mark.parametrize("gs", [16, 32])
+def test_qmv_batched_fp4(gs):
+    shapes = [(256, 1024), (96, 2048), (130, 4096)]
+    xs, ws, ss = [], [], []
+    for i, (n, k) in enumerate(shapes):
+        codes, scales = inputs.fp4(n, k, gs, seed=40 + i + gs)
+        xs.append(to_dev(inputs.fp4_x(4, k)))
+        ws.append(codes.to(DEV))
+        ss.append(scales.to(DEV))
+    ys = api.aq_qmv_batched(xs, ws, ss, None, 4, gs)
+    torch.cuda.synchronize()
+    for x, wq, sc, y in zip(xs, ws, ss, ys):
+        _check(x, wq, sc, None, y, 4, gs, 1, mode=1)
+
+
+def test_qmv_batched_many_problems_two_launches():
+    """More problems than one launch holds: the library splits the batch and
+    reuses the workspace across launches."""
+    M, bits, gs, dt = 2, 4, 64, 1
+    cases = [_case(M, 256, 4096, bits, gs, dt, seed=200 + i) for i in range(45)]
+    ys = api.aq_qmv_batched([c[0] for c in cases], [c[1] for c in cases], [c[2] for c in cases],
+                            [c[3] for c in cases], bits, gs)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        _check(*c, y, bits, gs, dt)
+
+
+def test_qmv_deterministic_and_workspace_left_zero():
+    """Split-K partials meet in the workspace; the slices are added in slice
+    order, so repeated calls agree bit for bit, and every call leaves the
+    counters (the first 64 KB of the workspace) zero."""
+    M, bits, gs, dt = 16, 4, 64, 1
+    x, wq, s, b = _case(M, 2048, 8192, bits, gs, dt, seed=77, wstd=0.02)
+    ws = api.Workspace()
+    y1 = api.aq_qmv(x, wq, s, b, bits, gs, workspace=ws)
+    y2 = api.aq_qmv(x, wq, s, b, bits, gs, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    buf = ws.get(x.device, 1)
+    assert buf is not None and int(buf[:65536].count_nonzero()) == 0
+    _check(x, wq, s, b, y2, bits, gs, dt)
+
+
+def test_qmv_workspace_required():
+    x, wq, s, b = _case(16, 2048, 8192, 4, 64, 1, seed=3)
+    need = api.aq_workspace_size(api.AQ_OP_QMV, 16, 2048, 8192, 4, 64)
+    assert need > 0
+    y = torch.empty((16, 2048), dtype=torch.bfloat16, device=DEV)
+    st = api.lib().aq_qmv(x.data_ptr(), wq.data_ptr(), s.data_ptr(), b.data_ptr(), y.data_ptr(),
+                          16, 2048, 8192, 4, 64, 0, 1, None, 0, None)
+    assert st == 5   # AQ_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_qmv_odd_shapes_fp32_kernel(M):
+    """Shapes the tensor-core kernel cannot stream (scale rows that are not
+    16-byte multiples, 3-bit rows of 8-byte multiples) run the fp32 kernel,
+    for every M up to 16."""
+    for (N, K, bits, gs) in [(40, 96, 4, 32), (33, 64 * 3, 3, 64), (17, 448, 5, 32)]:
+        x, wq, s, b = _case(M, N, K, bits, gs, 0, seed=N + K + M)
+        y = api.aq_qmv(x, wq, s, b, bits, gs)
+        torch.cuda.synchronize()
+        _check(x, wq, s, b, y, bits, gs, 0)

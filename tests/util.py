@@ -90,10 +90,8 @@ def check_matmul(y_t_u16, y_ref, den, dt, rel=REL_TOL, what="y", overflow_any_no
 
 
 def qmv_w_in_t(M, K, bits, gs, mode=0):
-    """Which w_hat aq_qmv multiplies: the tensor-core decode kernel (taken
-    whenever the packed rows and the rows of scales are 16-byte multiples)
-    and the tensor-core fallback for M >= 3 multiply weight tiles rounded to
-    T; only the fp32 kernel (M <= 2, other shapes) keeps w_hat in fp32."""
-    esz = 1 if mode == 1 else 2
-    tc = (K * bits // 8) % 16 == 0 and (K // gs * esz) % 16 == 0
-    return tc or M > 2
+    """Which w_hat aq_qmv multiplies: every aq_qmv kernel keeps w_hat in fp32
+    (scale and bias applied per group in fp32 to the exact integer-code
+    products, as the qmv of "Add the 3bit packed qmm_t" does), so its
+    reference is the exact product for every M and shape."""
+    return False
