@@ -4,6 +4,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <algorithm>
 #include <vector>
 
 #include "common.cuh"
@@ -159,9 +160,18 @@ aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void*
   if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
   if (N == 0) return AQ_OK;
   if (K == 0) return zero_output(y, M, N, stream);
-  // The tensor-core decode kernel takes every shape whose packed rows and
-  // scale rows are 16-byte multiples (TMA); other shapes run the fp32
-  // CUDA-core kernel.  Both keep w_hat in fp32 (scale and bias per group).
+  // 4-bit affine weights with K a multiple of the sub-slice run the
+  // warp-MMA streaming kernel; other shapes whose packed rows and scale rows
+  // are 16-byte multiples (TMA) run the tcgen05 decode kernel; the rest run
+  // the fp32 CUDA-core kernel.  All keep w_hat in fp32 (scale and bias per
+  // group).
+  if (aq::qmv_mma_applies(M, N, K, bits, group_size, mode, scales, biases)) {
+    const size_t need = aq::qmv_mma_workspace(M, N, K, group_size);
+    if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
+    return cuda_status(aq::launch_qmv_mma(x, w_q, scales, biases, y, M, N, K, group_size, dtype,
+                                          workspace, (cudaStream_t)stream),
+                       "aq_qmv launch");
+  }
   if (aq::qmv_tc_applies(M, N, K, bits, group_size, mode, scales, biases)) {
     const size_t need = aq::qmv_tc_workspace(M, N, K, bits, group_size);
     if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
@@ -173,6 +183,17 @@ aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void*
   return cuda_status(aq::launch_qmv(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
                                     mode, dtype, workspace, (cudaStream_t)stream),
                      "aq_qmv launch");
+}
+
+// Whether every problem of a batch takes the warp-MMA decode kernel (the
+// batch then runs on it; otherwise on the tcgen05 decode kernel).
+static bool all_mma(const aq_qmv_problem* problems, int count, int64_t M, int bits,
+                    int group_size, aq_mode mode) {
+  for (int i = 0; i < count; ++i)
+    if (!aq::qmv_mma_applies(M, problems[i].N, problems[i].K, bits, group_size, mode,
+                             problems[i].scales, problems[i].biases))
+      return false;
+  return true;
 }
 
 static aq_status check_batch(const aq_qmv_problem* problems, int count, int64_t M, int bits,
@@ -212,6 +233,13 @@ aq_status aq_qmv_batched(const aq_qmv_problem* problems, int count, int64_t M, i
   for (int i = 0; i < count; ++i)
     d[(size_t)i] = {problems[i].x, problems[i].w_q, problems[i].scales, problems[i].biases,
                     problems[i].y, problems[i].N, problems[i].K};
+  if (all_mma(problems, count, M, bits, group_size, mode)) {
+    const size_t need = aq::qmv_mma_batched_workspace(d.data(), count, M, group_size);
+    if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
+    return cuda_status(aq::launch_qmv_mma_batched(d.data(), count, M, group_size, dtype,
+                                                  workspace, (cudaStream_t)stream),
+                       "aq_qmv_batched launch");
+  }
   const size_t need = aq::qmv_tc_batched_workspace(d.data(), count, M, bits, group_size);
   if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
   return cuda_status(aq::launch_qmv_tc_batched(d.data(), count, M, bits, group_size, mode, dtype,
@@ -223,8 +251,15 @@ size_t aq_qmv_batched_workspace_size(const aq_qmv_problem* problems, int count, 
                                      int bits, int group_size, aq_mode mode) {
   if (!problems || count <= 0 || M < 1 || M > 16 || group_size <= 0) return 0;
   std::vector<aq::QmvProblemDesc> d;
-  for (int i = 0; i < count; ++i) {
+  for (int i = 0; i < count; ++i)
     if (problems[i].N <= 0 || problems[i].K <= 0 || problems[i].K % group_size) return 0;
+  if (all_mma(problems, count, M, bits, group_size, mode)) {
+    for (int i = 0; i < count; ++i)
+      d.push_back({problems[i].x, problems[i].w_q, problems[i].scales, problems[i].biases,
+                   problems[i].y, problems[i].N, problems[i].K});
+    return aq::qmv_mma_batched_workspace(d.data(), count, M, group_size);
+  }
+  for (int i = 0; i < count; ++i) {
     if (!aq::qmv_tc_shape_ok(problems[i].N, problems[i].K, bits, group_size, mode)) continue;
     d.push_back({problems[i].x, problems[i].w_q, problems[i].scales, problems[i].biases,
                  problems[i].y, problems[i].N, problems[i].K});
@@ -253,9 +288,10 @@ unsigned aq_device_errors(void) {
   unsigned v = 0, w = 0;
   if (aq::read_device_error_qmm(&v) != cudaSuccess) return 0xFFFFFFFFu;
   if (aq::read_device_error_conv(&w) != cudaSuccess) return 0xFFFFFFFFu;
-  unsigned t = 0;
+  unsigned t = 0, u = 0;
   if (aq::read_device_error_qmv_tc(&t) != cudaSuccess) return 0xFFFFFFFFu;
-  return v | w | t;
+  if (aq::read_device_error_qmv_mma(&u) != cudaSuccess) return 0xFFFFFFFFu;
+  return v | w | t | u;
 }
 
 aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* scales,
@@ -302,9 +338,14 @@ size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, in
   if (M <= 0 || N <= 0 || K <= 0 || group_size <= 0 || K % group_size) return 0;
   if (op == AQ_OP_QMV) {
     if (M > 16) return 0;
+    // Which decode kernel runs also depends on the pointers' alignment, so
+    // size for either.
+    size_t need = 0;
+    if (aq::qmv_mma_shape_ok(N, K, bits, group_size, mode))
+      need = aq::qmv_mma_workspace(M, N, K, group_size);
     if (aq::qmv_tc_shape_ok(N, K, bits, group_size, mode))
-      return aq::qmv_tc_workspace(M, N, K, bits, group_size);
-    return aq::plan_qmv(M, N, K, bits, group_size, mode).ws_bytes;
+      return std::max(need, aq::qmv_tc_workspace(M, N, K, bits, group_size));
+    return std::max(need, aq::plan_qmv(M, N, K, bits, group_size, mode).ws_bytes);
   }
   return 0;
 }

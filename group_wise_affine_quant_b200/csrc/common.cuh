@@ -150,6 +150,20 @@ cudaError_t launch_qmv_tc(const void* x, const void* w_q, const void* scales, co
 cudaError_t launch_qmv_tc_batched(const QmvProblemDesc* probs, int count, int64_t M, int bits,
                                   int gs, int mode, int dtype, void* ws, cudaStream_t st);
 cudaError_t read_device_error_qmv_tc(unsigned* out);
+// Warp-MMA decode path for 4-bit affine weights (qmv_mma.cu): applies when K
+// is a multiple of the sub-slice (512 columns; 1024 for group size 128) and
+// the scales / biases are 16-byte aligned.
+bool qmv_mma_shape_ok(int64_t N, int64_t K, int bits, int gs, int mode);
+bool qmv_mma_applies(int64_t M, int64_t N, int64_t K, int bits, int gs, int mode,
+                     const void* scales, const void* biases);
+size_t qmv_mma_workspace(int64_t M, int64_t N, int64_t K, int gs);
+size_t qmv_mma_batched_workspace(const QmvProblemDesc* probs, int count, int64_t M, int gs);
+cudaError_t launch_qmv_mma(const void* x, const void* w_q, const void* scales,
+                           const void* biases, void* y, int64_t M, int64_t N, int64_t K, int gs,
+                           int dtype, void* ws, cudaStream_t st);
+cudaError_t launch_qmv_mma_batched(const QmvProblemDesc* probs, int count, int64_t M, int gs,
+                                   int dtype, void* ws, cudaStream_t st);
+cudaError_t read_device_error_qmv_mma(unsigned* out);
 // aq_set_weight_prefetch's process-wide setting (0 or 1).
 int weight_prefetch_enabled();
 // aq_set_input_prefetch's process-wide setting (0 or 1).
