@@ -32,6 +32,7 @@
 //     distributed shared memory.  No workspace, no global atomics.
 //   * Every mbarrier wait is bounded (2 s); a timeout sets a device error
 //     flag, every role stops issuing work and the CTA frees its TMEM.
+#include <atomic>
 #include <cooperative_groups.h>
 
 #include <string.h>
@@ -1085,23 +1086,57 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  // Resolved once per process (a function-local static is initialised
+  // exactly once even when several threads call at the same time).
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+  }();
   return fn;
 }
+
+// Encoded 2-D maps of the calling thread, keyed by every encode argument: a
+// call that repeats a previous call's operands (the usual case for weights)
+// copies the 128-byte map instead of encoding it again.  Direct-mapped, per
+// thread, so no locking; a map only describes an address range and a shape,
+// so an entry stays valid for as long as its arguments are passed again.
+struct MapKey {
+  const void* base;
+  int64_t rows, cols;
+  int type, esize, box_cols, box_rows, swz;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && rows == o.rows && cols == o.cols && type == o.type &&
+           esize == o.esize && box_cols == o.box_cols && box_rows == o.box_rows && swz == o.swz;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  bool used;
+  CUtensorMap map;
+};
+constexpr int kMapCache = 256;
 
 // 2-D tensor map over a row-major [rows, cols] array of 1- or 2-byte
 // elements; zero fill out of bounds.
 cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int esize,
                      int64_t rows, int64_t cols, int box_cols, int box_rows,
                      CUtensorMapSwizzle swz) {
+  thread_local MapEntry cache[kMapCache];
+  const MapKey key{base, rows, cols, (int)type, esize, box_cols, box_rows, (int)swz};
+  uint64_t h = (uint64_t)(uintptr_t)base * 0x9E3779B97F4A7C15ull;
+  h ^= (uint64_t)(rows * 31 + cols) * 0xC2B2AE3D27D4EB4Full;
+  h ^= (uint64_t)(((int)type * 8 + esize) * 1024 + box_cols * 4 + (int)swz) * 0x165667B19E3779F9ull;
+  h ^= (uint64_t)box_rows << 17;
+  MapEntry& slot = cache[(h >> 40) % kMapCache];
+  if (slot.used && slot.key == key) {
+    *map = slot.map;
+    return cudaSuccess;
+  }
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -1111,7 +1146,11 @@ cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType typ
   CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  slot.key = key;
+  slot.map = *map;
+  slot.used = true;
+  return cudaSuccess;
 }
 
 // 4-D tensor map over an NHWC activation [Bn, H, W, C] of 2-byte elements,
@@ -1137,14 +1176,14 @@ template <typename T, int BITS, bool FP4, int BT, bool FAST, int XMODE>
 cudaError_t launch_tc(const QmmPlan& p, const QmmMaps& maps, const QmmArgs& a, cudaStream_t st) {
   using S = QmmShape<BT, BITS, FAST>;
   auto kern = qmm_tc_kernel<T, BITS, FP4, BT, FAST, XMODE>;
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !attr_done[dev]) {
+  if (dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
     if (e != cudaSuccess) return e;
-    if (dev < 64) attr_done[dev] = true;
+    if (dev < 64) attr_done[dev].store(true, std::memory_order_release);
   }
   // Part 0: tiles [0, tiles_main) with p.splits K-slices each; part 1 (the
   // partial last wave, when the plan splits it): the remaining tiles with

@@ -1,5 +1,7 @@
-// qmv.cu — fp32 weight-streaming GEMV for one or two rows of x (aq_qmv routes
-// 3..16 rows to the tensor-core kernel, which consumes codes faster there).
+// qmv.cu — fp32 CUDA-core weight-streaming GEMV for 1 <= M <= 16 rows of x:
+// aq_qmv's fallback for the shapes that neither decode kernel takes (packed
+// rows or scale rows that are not 16-byte multiples, or scales / biases that
+// are not 16-byte aligned; see qmv_mma.cu and qmv_tc.cu).
 //
 // Prior art: affine_packed_qmv_fast in "Add the 3bit packed qmm_t" (one
 // simdgroup streams a few weight rows, fp32 accumulation, simd_sum).  The
@@ -25,6 +27,7 @@
 //     distributed shared memory.  No workspace and no global atomics.
 //   * A CTA stages x once and then walks RI groups of rows, and each lane
 //     issues the load of its first weight unit before staging x.
+#include <atomic>
 #include <cooperative_groups.h>
 
 #include <utility>
@@ -263,14 +266,14 @@ cudaError_t launch_one(const QmvPlan& p, const void* x, const void* w_q, const v
                        cudaStream_t st) {
   auto kern = qmv_kernel<T, BITS, MT, FP4>;
   if (p.smem > 48 * 1024) {
-    static bool attr_done[64] = {};   // per instantiation and device
+    static std::atomic<bool> attr_done[64];   // per instantiation and device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !attr_done[dev]) {
+    if (dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
       if (e != cudaSuccess) return e;
-      if (dev < 64) attr_done[dev] = true;
+      if (dev < 64) attr_done[dev].store(true, std::memory_order_release);
     }
   }
   cudaLaunchConfig_t cfg = {};

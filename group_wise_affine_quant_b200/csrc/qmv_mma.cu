@@ -55,7 +55,10 @@ namespace {
 
 constexpr int kMvRows = 128;                 // weight rows per unit (8 warps x 16)
 constexpr int kMvMaxProblems = 40;           // problems per launch of the batched entry
-constexpr int kMvMaxSplitTiles = 16384;      // 16-row tiles with a counter (64 KB of counters)
+constexpr int kMvSchedWords = 16;            // workspace words 0, 1: unit counter, exit counter
+constexpr int kMvMaxSplitTiles = 16384 - kMvSchedWords;  // 16-row tiles with a counter
+constexpr int kMvCntWords = 16384;           // the counter area: the first 64 KB of the workspace
+constexpr int kMvQ = 8;                      // unit-queue depth (producer -> prep and MMA warps)
 
 struct MvProblem {
   CUtensorMap w;        // [N, K/2] u8, box {128 bytes, 128 rows}, 128-byte swizzle
@@ -110,8 +113,8 @@ struct MvShape {
   static constexpr int kTabOff = kXsOff + 2 * kXsBuf;
   static constexpr int kSbOff = kTabOff + 2 * kTabBuf;
   static constexpr int kBarOff = kSbOff + 4 * kSbArr;
-  static constexpr int kBars = 2 * kST + 8;
-  static constexpr int kSmem = 1024 + kBarOff + kBars * 8 + 16;
+  static constexpr int kBars = 2 * kST + 10 + 2 * kMvQ;
+  static constexpr int kSmem = 1024 + kBarOff + kBars * 8 + 16 + 4 * kMvQ;
   static_assert(kXP % 128 == 64, "x pitch");
   static_assert(kSbOff % 128 == 0 && kXOff % 1024 == 0, "TMA destinations");
   static_assert((kGps * 2) % 16 == 0, "scale box rows are 16-byte multiples");
@@ -192,6 +195,17 @@ __device__ __forceinline__ MvUnit mv_unit(const MvParams<P>& pr, int u) {
   return un;
 }
 
+// Next unit id from the CTA's unit queue (-1: no more units; -2: a wait gave up).
+__device__ __forceinline__ int mv_take(volatile int* uq, uint64_t* uqf, uint64_t* uqe, int k,
+                                       int lane, volatile int* abort_flag) {
+  const int qs = k % kMvQ;
+  if (!mbar_wait(smem_u32(uqf + qs), (k / kMvQ) & 1, abort_flag)) return -2;
+  const int u = uq[qs];
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(uqe + qs));
+  return u;
+}
+
 __device__ __forceinline__ void mv_drain(const uint64_t* bars, int slots, int issued,
                                          volatile int* abort_flag) {
   for (int c = issued - 1; c >= 0 && c >= issued - slots; --c) {
@@ -227,7 +241,11 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
   uint64_t* sbe = sbf + 2;               // raw scales / biases converted (its prep warp)
   uint64_t* xf = sbe + 2;                // sub-slice prepared (its prep warp)
   uint64_t* xe = xf + 2;                 // sub-slice consumed (the MMA warps)
+  uint64_t* xsr = xe + 2;                // per-group x sums of a sub-slice written (the MMA warps)
+  uint64_t* uqf = xsr + 2;               // unit id posted (producer)
+  uint64_t* uqe = uqf + kMvQ;            // unit id read (every prep and MMA warp)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + S::kBars);
+  volatile int* uq = reinterpret_cast<volatile int*>(bars + S::kBars) + 4;   // [kMvQ] unit ids
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int M = pr.M;
@@ -243,6 +261,11 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
       mbar_init(smem_u32(sbe + i), 1);
       mbar_init(smem_u32(xf + i), 1);
       mbar_init(smem_u32(xe + i), kMvWarps);
+      mbar_init(smem_u32(xsr + i), kMvWarps);
+    }
+    for (int i = 0; i < kMvQ; ++i) {
+      mbar_init(smem_u32(uqf + i), 1);
+      mbar_init(smem_u32(uqe + i), kMvWarps + 2);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -254,9 +277,23 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
     // ------------------------------------------------------------ TMA issue
     int wc = 0, sc = 0;
     if (lane == 0) {
-      if (!pr.weights_early) pdl_wait();
+      bool waited = !pr.weights_early;
+      if (waited) pdl_wait();
       const uint64_t pol = l2_policy_evict_first();
-      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+      // Units: the first one of each CTA is blockIdx.x; later ones are claimed
+      // from the launch's unit counter (after the wait on the previous kernel,
+      // which leaves the counter at zero), so the CTAs stay evenly loaded.
+      int posted = 0;
+      auto post = [&](int uu) -> bool {
+        const int qs = posted % kMvQ;
+        if (!mbar_wait(smem_u32(uqe + qs), ((posted / kMvQ) & 1) ^ 1, abort_flag)) return false;
+        uq[qs] = uu;
+        mbar_arrive(smem_u32(uqf + qs));
+        ++posted;
+        return true;
+      };
+      for (int u = blockIdx.x; u < total && !*abort_flag;) {
+        if (!post(u)) break;
         const MvUnit un = mv_unit<P, SUBK>(pr, u);
         const MvProblem& q = pr.prob[un.p];
         const int row0 = un.rb * kMvRows;
@@ -279,7 +316,14 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
             ++wc;
           }
         }
+        if (!ok) break;
+        if (!waited) {
+          pdl_wait();
+          waited = true;
+        }
+        u = (int)gridDim.x + (int)atomicAdd(pr.ws, 1u);
       }
+      if (!*abort_flag) post(-1);                           // no more units
       mv_drain(full, ST, wc, abort_flag);
       mv_drain(sbf, 2, sc, abort_flag);
     }
@@ -290,7 +334,9 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
     pdl_wait();
     int c = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+      const int u = mv_take(uq, uqf, uqe, k, lane, abort_flag);
+      if (u < 0) { ok = u == -1; break; }
       const MvUnit un = mv_unit<P, SUBK>(pr, u);
       const MvProblem& q = pr.prob[un.p];
       const T* xg = reinterpret_cast<const T*>(q.x);
@@ -298,9 +344,23 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
         if ((c & 1) != b) continue;
         const uint32_t par = (c >> 1) & 1;
         uint8_t* xb = smem + S::kXOff + b * S::kXBuf;
-        if (!mbar_wait(smem_u32(xe + b), par ^ 1, abort_flag) ||
-            !mbar_wait(smem_u32(sbf + b), par, abort_flag)) { ok = false; break; }
-        // fp32 (s, b - off * s) per weight row and group
+        if (!mbar_wait(smem_u32(xe + b), par ^ 1, abort_flag)) { ok = false; break; }
+        // x columns of the sub-slice (natural order; 64-byte blocks of 32 columns
+        // at a row pitch of 64 mod 128 bytes), copied with cp.async
+        const int kk = un.k0 + j * SUBK;
+        constexpr int kCpr = SUBK / 8;                         // 16-byte chunks per x row
+        const int nch = M * kCpr;
+        for (int i = lane; i < nch; i += 32) {
+          const int m = i / kCpr, ch = i % kCpr;
+          cp_async_16(smem_u32(xb + m * S::kXP + ch * 16),
+                     reinterpret_cast<const uint4*>(xg + (int64_t)m * q.K + kk) + ch);
+        }
+        // fp32 (s, b - off * s) per weight row and group (while the x copy is in flight)
+        if (!mbar_wait(smem_u32(sbf + b), par, abort_flag)) {
+          cp_async_wait_all();                              // no copy may outlive the CTA
+          ok = false;
+          break;
+        }
         const uint16_t* sraw = reinterpret_cast<const uint16_t*>(smem + S::kSbOff + b * 2 * S::kSbArr);
         const uint16_t* braw = sraw + kMvRows * GPS;
         float2* tab = reinterpret_cast<float2*>(smem + S::kTabOff + b * S::kTabBuf);
@@ -319,16 +379,6 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(sbe + b));
-        // x columns of the sub-slice (natural order; 64-byte blocks of 32 columns
-        // at a row pitch of 64 mod 128 bytes), copied with cp.async
-        const int kk = un.k0 + j * SUBK;
-        constexpr int kCpr = SUBK / 8;                         // 16-byte chunks per x row
-        const int nch = M * kCpr;
-        for (int i = lane; i < nch; i += 32) {
-          const int m = i / kCpr, ch = i % kCpr;
-          cp_async_16(smem_u32(xb + m * S::kXP + ch * 16),
-                     reinterpret_cast<const uint4*>(xg + (int64_t)m * q.K + kk) + ch);
-        }
         cp_async_wait_all();
         // reorder each 8-column chunk in place to the order the codes unpack:
         // (x0,x4), (x2,x6), (x1,x5), (x3,x7)
@@ -343,35 +393,6 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
           *pc = o;
         }
         __syncwarp();
-        // per-group sums of each x row: MMAs with an all-ones A operand
-        float* xs = reinterpret_cast<float*>(smem + S::kXsOff + b * S::kXsBuf);
-        const uint32_t one[4] = {ones2<T>(), ones2<T>(), ones2<T>(), ones2<T>()};
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const bool live = g + 8 * nt < M;
-          const uint8_t* xr = xb + (g + 8 * nt) * S::kXP + t * 16;
-#pragma unroll 1
-          for (int g0 = 0; g0 < GPS; g0 += 4) {                // four groups at a time
-            float d[4][4];
-#pragma unroll
-            for (int bl = 0; bl < GS / 32; ++bl) {
-#pragma unroll
-              for (int gi = 0; gi < 4; ++gi) {
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (live) v = *reinterpret_cast<const uint4*>(xr + ((g0 + gi) * (GS / 32) + bl) * 64);
-                if (bl == 0) mma16816_z<T>(d[gi], one, v.x, v.y);
-                else mma16816<T>(d[gi], one, v.x, v.y);
-                mma16816<T>(d[gi], one, v.z, v.w);
-              }
-            }
-            if (g == 0) {
-#pragma unroll
-              for (int gi = 0; gi < 4; ++gi)
-                *reinterpret_cast<float2*>(xs + (g0 + gi) * 16 + 8 * nt + 2 * t) =
-                    make_float2(d[gi][0], d[gi][1]);
-            }
-          }
-        }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(xf + b));
       }
@@ -382,7 +403,9 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
     pdl_wait();                                   // y and the workspace are ordered
     int wc = 0, c = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+      const int u = mv_take(uq, uqf, uqe, k, lane, abort_flag);
+      if (u < 0) { ok = u == -1; break; }
       const MvUnit un = mv_unit<P, SUBK>(pr, u);
       const MvProblem& q = pr.prob[un.p];
       float acc[R][NT][4];
@@ -396,7 +419,41 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
         const int buf = c & 1;
         if (!mbar_wait(smem_u32(xf + buf), (c >> 1) & 1, abort_flag)) { ok = false; break; }
         const uint8_t* xb = smem + S::kXOff + buf * S::kXBuf + t * 16;
-        const float* xs = reinterpret_cast<const float*>(smem + S::kXsOff + buf * S::kXsBuf) + 2 * t;
+        float* xsw = reinterpret_cast<float*>(smem + S::kXsOff + buf * S::kXsBuf);
+        {
+          // Per-group sums of each x row, GPS / kMvWarps groups per warp: an MMA
+          // with an all-ones A operand adds the K-steps' columns.
+          const uint32_t one[4] = {ones2<T>(), ones2<T>(), ones2<T>(), ones2<T>()};
+          constexpr int kGpw = GPS / kMvWarps;
+          static_assert(GPS % kMvWarps == 0, "groups per sub-slice split over the MMA warps");
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            float dd[kGpw][4];
+#pragma unroll
+            for (int bl = 0; bl < GS / 32; ++bl) {
+#pragma unroll
+              for (int j2 = 0; j2 < kGpw; ++j2) {
+                const int gi = warp * kGpw + j2;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (g + 8 * nt < M)
+                  v = *reinterpret_cast<const uint4*>(xb + (g + 8 * nt) * S::kXP + (gi * (GS / 32) + bl) * 64);
+                if (bl == 0) mma16816_z<T>(dd[j2], one, v.x, v.y);
+                else mma16816<T>(dd[j2], one, v.x, v.y);
+                mma16816<T>(dd[j2], one, v.z, v.w);
+              }
+            }
+            if (g == 0) {
+#pragma unroll
+              for (int j2 = 0; j2 < kGpw; ++j2)
+                *reinterpret_cast<float2*>(xsw + (warp * kGpw + j2) * 16 + 8 * nt + 2 * t) =
+                    make_float2(dd[j2][0], dd[j2][1]);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(xsr + buf));
+          if (!mbar_wait(smem_u32(xsr + buf), (c >> 1) & 1, abort_flag)) { ok = false; break; }
+        }
+        const float* xs = xsw + 2 * t;
         const float2* tab = reinterpret_cast<const float2*>(smem + S::kTabOff + buf * S::kTabBuf) +
                             (warp * 16 * R + g) * S::kTabPitch;
         for (int st = 0; st < S::kSps; ++st) {
@@ -548,7 +605,15 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
   }
 
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) atomicOr(&g_aq_device_error, 1u);
+  if (threadIdx.x == 0) {
+    if (*abort_flag) atomicOr(&g_aq_device_error, 1u);
+    // The last CTA to leave puts the launch's unit counter back to zero.
+    __threadfence();
+    if (atomicAdd(pr.ws + 1, 1u) == gridDim.x - 1) {
+      atomicExch(pr.ws, 0u);
+      atomicExch(pr.ws + 1, 0u);
+    }
+  }
 }
 
 // ------------------------------------------------------------------- host
@@ -586,8 +651,7 @@ struct MvGroupPlan {
 void mv_plan_group(MvGroupPlan& g, const QmvProblemDesc* probs, int count, int64_t M, int gs,
                    int64_t slots, int64_t unit_bytes) {
   int tiles_used = 0;
-  int64_t part = kMvMaxSplitTiles;
-  bool any = false;
+  int64_t part = kMvCntWords;
   for (int i = 0; i < count; ++i) {
     MvSplit d = mv_split(probs[i].N, probs[i].K, gs, slots, unit_bytes);
     const int64_t tiles = (probs[i].N + kMvRows - 1) / kMvRows * 8;
@@ -596,20 +660,19 @@ void mv_plan_group(MvGroupPlan& g, const QmvProblemDesc* probs, int count, int64
       d.kslice = (int)probs[i].K;
     }
     g.sp[i] = d;
-    g.cnt0[i] = tiles_used;
+    g.cnt0[i] = kMvSchedWords + tiles_used;
     g.part[i] = part;
     if (d.splits > 1) {
-      any = true;
       tiles_used += (int)tiles;
       part += (tiles * d.splits * M * 16 + 31) / 32 * 32;
     }
   }
-  g.words = any ? part : 0;
+  g.words = part;                                     // the counters are always needed
 }
 
 template <typename T, int GS, int NT, int P>
 struct MvKernel {
-  static constexpr int R = NT == 1 ? 1 : 2;                   // M <= 8: one tile per MMA warp
+  static constexpr int R = 1;                                 // one 16-row tile per MMA warp
   using S = MvShape<GS, NT, R>;
   static cudaError_t prepare(int* slots) {
     static std::atomic<int> occ[64];
@@ -679,9 +742,14 @@ cudaError_t mv_launch_group(const QmvProblemDesc* probs, int count, int64_t M, v
   int slots = 0;
   cudaError_t e = MvKernel<T, GS, NT, P>::prepare(&slots);
   if (e != cudaSuccess) return e;
+  // A single matmul runs one CTA per SM: the next kernel of the stream (launched
+  // with programmatic dependent launch) then fits beside it and can start
+  // streaming its weights while this one finishes.  Batched launches fill
+  // both CTA slots of every SM.
+  if (unit_bytes == 0) slots = std::max(1, slots / 2);
   MvGroupPlan g;
   mv_plan_group(g, probs, count, M, GS, slots, unit_bytes);
-  if (g.words > 0 && !ws) return cudaErrorInvalidValue;
+  if (!ws) return cudaErrorInvalidValue;
   MvParams<P> pr;
   memset(&pr, 0, sizeof(pr));
   int units = 0;

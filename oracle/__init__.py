@@ -30,6 +30,8 @@ def lib():
         I64 = ctypes.c_int64
         I = ctypes.c_int
         _lib.orc_num_threads.restype = I
+        _lib.orc_set_num_threads.argtypes = [I]
+        _lib.orc_set_num_threads.restype = None
         _lib.orc_t_to_double.argtypes = [ctypes.c_uint16, I]
         _lib.orc_t_to_double.restype = ctypes.c_double
         _lib.orc_round_to_t.argtypes = [ctypes.c_double, I]
@@ -65,6 +67,11 @@ def _check(rc, what):
 
 def num_threads() -> int:
     return lib().orc_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops (results do not depend on it)."""
+    lib().orc_set_num_threads(int(n))
 
 
 def t_to_double(bits16, dt):

@@ -232,6 +232,17 @@ int check_common(int64_t N, int64_t K, int bits, int gs, int mode, int dt) {
 
 extern "C" {
 
+// Threads the oracle's parallel loops use (OpenMP); the timed CPU baseline
+// also runs it on one thread.  Changes no result: every output element is
+// computed by one thread in the same order either way.
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -108,7 +108,9 @@ def test_qmv_batched_validation():
     need = L().aq_qmv_batched_workspace_size(p, 3, 16, 4, 64, 0)
     assert need > 0
     assert b(p, 3, 16, 4, 64, 0, 1, None, 0, None) == WORKSPACE
-    assert L().aq_qmv_batched_workspace_size(_problems(3), 3, 16, 4, 64, 0) == 0   # K = 2048: one unit per tile
+    # K = 2048: one K-slice per row tile, so only the 64 KB counter area (the
+    # unit scheduler's counters) and no partial sums
+    assert L().aq_qmv_batched_workspace_size(_problems(3), 3, 16, 4, 64, 0) == 65536
 
 
 def test_prefetch_settings_are_per_thread():
