@@ -27,6 +27,7 @@ SIGNATURES = {
     "aq_dequantize": (_I, [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _P]),
     "aq_qmv": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
     "aq_qmm": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
+    "aq_qmv_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P]),
     "aq_qconv2d_nhwc": (_I, [_P, _P, _P, _P, _P] + [_I] * 15 + [_P, _SZ, _P]),
     "aq_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I, _I, _I, _I]),
     "aq_last_error": (ctypes.c_char_p, []),

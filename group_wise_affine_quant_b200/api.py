@@ -13,7 +13,7 @@ from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, 
                    AQ_OP_QMV, AqError, check, lib)
 
 __all__ = ["aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_qconv2d_nhwc",
-           "aq_workspace_size", "aq_last_error", "aq_set_weight_prefetch",
+           "aq_workspace_size", "aq_qmv_noalloc", "aq_last_error", "aq_set_weight_prefetch",
            "aq_get_weight_prefetch", "aq_set_input_prefetch", "aq_get_input_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
 
 _DT = {torch.float16: AQ_F16, torch.bfloat16: AQ_BF16}
@@ -133,6 +133,19 @@ def _mm(fn_name, op, x, w_q, scales, biases, bits, group_size, out, workspace):
 def aq_qmv(x, w_q, scales, biases, bits=4, group_size=64, out=None, workspace=None):
     """y = x . dequant(w)^T for 1 <= M <= 16 rows of x."""
     return _mm("aq_qmv", AQ_OP_QMV, x, w_q, scales, biases, bits, group_size, out, workspace)
+
+
+def aq_qmv_noalloc(x, w_q, scales, biases, bits=4, group_size=64, out=None):
+    """aq_qmv on the library's fixed scratch (no workspace; the C call
+    allocates nothing).  `out` is allocated here by torch if not given."""
+    M, K = x.shape
+    N = w_q.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    check(lib().aq_qmv_noalloc(_ptr(x), _ptr(w_q), _ptr(scales), _ptr(biases), _ptr(out), M, N,
+                               K, bits, group_size, _mode(scales), _dt(x), _stream(x.device)),
+          "aq_qmv_noalloc")
+    return out
 
 
 def aq_qmv_batched(xs, w_qs, scales, biases, bits=4, group_size=64, outs=None, workspace=None):

@@ -196,6 +196,32 @@ static bool all_mma(const aq_qmv_problem* problems, int count, int64_t M, int bi
   return true;
 }
 
+aq_status aq_qmv_noalloc(const void* x, const void* w_q, const void* scales,
+                         const void* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+                         int group_size, aq_mode mode, aq_dtype dtype, aq_stream_t stream) {
+  g_err[0] = 0;
+  aq_status st = check_weight(w_q, scales, biases, N, K, bits, group_size, mode, dtype);
+  if (st != AQ_OK) return st;
+  if (M < 1 || M > 16)
+    return fail(AQ_ERR_INVALID_ARG, "aq_qmv_noalloc takes 1 <= M <= 16 (got %lld)", (long long)M);
+  if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
+  if (N == 0 || K == 0)
+    return fail(AQ_ERR_INVALID_ARG, "aq_qmv_noalloc needs N, K > 0");
+  if (!aq::qmv_mma_applies(M, N, K, bits, group_size, mode, scales, biases))
+    return fail(AQ_ERR_UNSUPPORTED,
+                "aq_qmv_noalloc takes 4-bit affine weights with K a multiple of 512 (1024 for "
+                "group_size 128) and 16-byte aligned scales / biases; use aq_qmv");
+  size_t need = 0;
+  const cudaError_t e = aq::launch_qmv_noalloc(x, w_q, scales, biases, y, M, N, K, group_size,
+                                               dtype, (cudaStream_t)stream, &need);
+  if (e == cudaErrorMemoryAllocation)
+    return fail(AQ_ERR_UNSUPPORTED,
+                "aq_qmv_noalloc: this shape needs %zu bytes of scratch, more than the %zu "
+                "bytes it holds; use aq_qmv with a workspace",
+                need, aq::kQmvNoallocScratchBytes);
+  return cuda_status(e, "aq_qmv_noalloc launch");
+}
+
 static aq_status check_batch(const aq_qmv_problem* problems, int count, int64_t M, int bits,
                              int group_size, aq_mode mode, aq_dtype dtype) {
   aq_status st = check_format(bits, group_size, mode, dtype);

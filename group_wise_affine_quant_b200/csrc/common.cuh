@@ -164,6 +164,14 @@ cudaError_t launch_qmv_mma(const void* x, const void* w_q, const void* scales,
 cudaError_t launch_qmv_mma_batched(const QmvProblemDesc* probs, int count, int64_t M, int gs,
                                    int dtype, void* ws, cudaStream_t st);
 cudaError_t read_device_error_qmv_mma(unsigned* out);
+// aq_qmv_noalloc's fixed scratch (a file-scope device array in qmv_mma.cu).
+constexpr size_t kQmvNoallocScratchBytes = (size_t)4 << 20;
+// Launches the warp-MMA decode kernel on that scratch.  Sets *need to the
+// scratch bytes the shape needs; returns cudaErrorMemoryAllocation (nothing
+// launched, nothing allocated) when that exceeds kQmvNoallocScratchBytes.
+cudaError_t launch_qmv_noalloc(const void* x, const void* w_q, const void* scales,
+                               const void* biases, void* y, int64_t M, int64_t N, int64_t K,
+                               int gs, int dtype, cudaStream_t st, size_t* need);
 // aq_set_weight_prefetch's process-wide setting (0 or 1).
 int weight_prefetch_enabled();
 // aq_set_input_prefetch's process-wide setting (0 or 1).

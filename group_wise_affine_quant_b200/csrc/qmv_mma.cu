@@ -838,4 +838,37 @@ cudaError_t launch_qmv_mma_batched(const QmvProblemDesc* probs, int count, int64
 
 cudaError_t read_device_error_qmv_mma(unsigned* out) { return read_tu_error(out); }
 
+// ------------------------------------------------ no-allocation entry point
+// Scratch of aq_qmv_noalloc, in place of a caller-supplied workspace: the
+// unit and split-K counters (its first 64 KB, which must start at zero: the
+// array is zero when the module loads, and every call that completes leaves
+// them zero) and the fp32 split-K partials.  Every call on a device shares
+// it, so calls whose kernels may overlap on the GPU (other streams, or no
+// ordering between them) race on it.
+static __device__ __align__(256) unsigned char g_qmv_scratch[kQmvNoallocScratchBytes];
+
+namespace {
+std::atomic<void*> g_scratch_ptr[64];
+}  // namespace
+
+cudaError_t launch_qmv_noalloc(const void* x, const void* w_q, const void* scales,
+                               const void* biases, void* y, int64_t M, int64_t N, int64_t K,
+                               int gs, int dtype, cudaStream_t st, size_t* need) {
+  *need = qmv_mma_workspace(M, N, K, gs);
+  if (*need > kQmvNoallocScratchBytes) return cudaErrorMemoryAllocation;   // caller reports
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  // Set-up on the first call on this device (with it current): the address
+  // of the scratch array in this device's copy of the module.
+  void* ptr = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!ptr) {
+    e = cudaGetSymbolAddress(&ptr, g_qmv_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev].store(ptr, std::memory_order_release);
+  }
+  return launch_qmv_mma(x, w_q, scales, biases, y, M, N, K, gs, dtype, ptr, st);
+}
+
 }  // namespace aq

@@ -164,6 +164,37 @@ AQ_API aq_status aq_qmv_batched(const aq_qmv_problem* problems, int count, int64
                                 int group_size, aq_mode mode, aq_dtype dtype, void* workspace,
                                 size_t workspace_bytes, aq_stream_t stream);
 
+/*
+ * aq_qmv_noalloc — aq_qmv for callers that cannot allocate device memory or
+ * manage a workspace buffer: e.g. code that runs after a serving process has
+ * fixed its device memory (no cudaMalloc allowed past start-up), or that has
+ * no allocator handle to obtain a workspace from.  The pages have no
+ * counterpart: this is the same computation as aq_qmv (the same kernel and
+ * result), run on a fixed scratch array inside the library instead of a
+ * caller workspace.
+ *   Arguments as aq_qmv, minus the workspace.  Only shapes that run the
+ *   warp-MMA decode kernel: 4-bit affine weights, 1 <= M <= 16, N, K > 0, K a
+ *   multiple of 512 (1024 for group_size 128), 16-byte aligned scales and
+ *   biases; others return AQ_ERR_UNSUPPORTED.
+ *   Limit: the scratch holds 4 MiB (64 KB of counters plus fp32 split-K
+ *   partials).  A shape that needs more returns AQ_ERR_UNSUPPORTED with the
+ *   size in aq_last_error(); e.g. every projection of a Llama-3.2-1B-sized
+ *   layer at M <= 16 fits.
+ *   Allocates nothing: no cudaMalloc / cudaFree and no allocating library
+ *   call.  The first call on a device (with that device current) looks up
+ *   the scratch array's device address once (cudaGetSymbolAddress); make
+ *   that first call before any stream capture.
+ *   The scratch is shared by every call on the device: its counters start at
+ *   zero and every call that completes leaves them zero; calls whose kernels
+ *   may overlap on the GPU (different streams without ordering) race on it.
+ *   After a device error (aq_device_errors() != 0) the scratch counters may
+ *   be left non-zero: do not use this entry point again in the process.
+ */
+AQ_API aq_status aq_qmv_noalloc(const void* x, const void* w_q, const void* scales,
+                                const void* biases, void* y, int64_t M, int64_t N, int64_t K,
+                                int bits, int group_size, aq_mode mode, aq_dtype dtype,
+                                aq_stream_t stream);
+
 /* Workspace bytes aq_qmv_batched needs for these problems (0 if none). */
 AQ_API size_t aq_qmv_batched_workspace_size(const aq_qmv_problem* problems, int count,
                                             int64_t M, int bits, int group_size, aq_mode mode);
