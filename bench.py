@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="layers of the stack (default 16; fewer for small profiling runs)")
     ap.add_argument("--no-qmm", action="store_true", help="skip the side configurations")
     ap.add_argument("--only", default="all", choices=["all", "qmm"],
                     help="qmm: run only the side configurations")
@@ -430,8 +432,9 @@ def main():
     # Quantize the stack once (on the device, through the library).  The
     # timed calls never follow a kernel that writes their weights, so the
     # library may stream weights before waiting on the previous kernel.
+    n_layers = args.layers
     layers = []
-    for li in range(LAYERS):
+    for li in range(n_layers):
         ws = inputs.decode_layer(seed=100 + li)
         layers.append({name: api.aq_quantize(w.to(dev), BITS, GS) for name, w in ws.items()})
         del ws
@@ -441,9 +444,9 @@ def main():
     all_m = QMV_M + QMM_M
     xs = {(M, k): inputs.decode_x(M, k, seed=M).to(dev) for M in all_m for k in (2048, 8192)}
     ys = {(M, li, name): torch.empty((M, n), dtype=torch.bfloat16, device=dev)
-          for M in all_m for li in range(LAYERS) for name, n, _ in projs}
+          for M in all_m for li in range(n_layers) for name, n, _ in projs}
     probs = {M: stack_problems(layers, xs, ys, M) for M in QMV_M}
-    n_problems = LAYERS * len(projs)
+    n_problems = n_layers * len(projs)
     launches_per_m = (n_problems + 39) // 40
     launches_per_step = len(QMV_M) * launches_per_m
 
@@ -477,14 +480,14 @@ def main():
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms, world)
-    step_bytes = LAYERS * sum(layer_bytes(M) for M in QMV_M)
+    step_bytes = n_layers * sum(layer_bytes(M) for M in QMV_M)
     value = world * step_bytes / (ms * 1e-3) / 1e9
 
     # Per-M views of the batched step.
     per_m = {}
     for M in QMV_M:
         t = graph_time_ms(torch, stream, lambda: step_m(M), 1)
-        per_m[str(M)] = {"gbs": round(LAYERS * layer_bytes(M) / (t * 1e-3) / 1e9, 1),
+        per_m[str(M)] = {"gbs": round(n_layers * layer_bytes(M) / (t * 1e-3) / 1e9, 1),
                          "ms": round(t, 4)}
 
     # The same products as 560 aq_qmv calls in order (each kernel waits for
@@ -504,13 +507,13 @@ def main():
         for M in (1, 16):
             t = graph_time_ms(torch, stream, lambda: calls(M, (name,)), 1)
             chain["per_projection"]["%s_M%d" % (name, M)] = {
-                "us_per_call": round(t * 1e3 / LAYERS, 2),
-                "gbs": round(LAYERS * proj_bytes(n, k, M) / (t * 1e-3) / 1e9, 1)}
+                "us_per_call": round(t * 1e3 / n_layers, 2),
+                "gbs": round(n_layers * proj_bytes(n, k, M) / (t * 1e-3) / 1e9, 1)}
     # the sweep's M = 32 and 64 rows through aq_qmm (per call, same stack)
     qmm_m = {}
     for M in QMM_M:
         t = graph_time_ms(torch, stream, lambda: calls(M), 1)
-        qmm_m[str(M)] = {"gbs": round(LAYERS * layer_bytes(M) / (t * 1e-3) / 1e9, 1),
+        qmm_m[str(M)] = {"gbs": round(n_layers * layer_bytes(M) / (t * 1e-3) / 1e9, 1),
                          "us_per_call": round(t * 1e3 / n_problems, 2)}
 
     # End to end through the public API with host buffers: pinned x in,
@@ -557,9 +560,10 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "layers": LAYERS, "M": list(QMV_M), "bits": BITS,
+            "config": {"workload": WORKLOAD, "layers": n_layers, "M": list(QMV_M), "bits": BITS,
                        "group_size": GS, "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "weights 547 MB > 4x L2 per step; no flush needed",
+                       "l2": "stack of %.0f MB of weights (> L2) streamed once per M; no flush "
+                             "needed" % (n_layers * layer_bytes(0) / 1e6),
                        "timing": "CUDA graph replay, CUDA events on the launching stream",
                        "weight_prefetch": "on (weights streamed before each kernel's dependency wait)"},
             "per_m": per_m, "per_call_chain": chain, "qmm_decode_m": qmm_m, "roofline": roof,
