@@ -37,6 +37,9 @@ SIGNATURES = {
     "aq_get_weight_prefetch": (_I, []),
     "aq_set_input_prefetch": (None, [_I]),
     "aq_get_input_prefetch": (_I, []),
+    "aq_testing_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "aq_testing_set_start_delay_ns": (None, [ctypes.c_uint64]),
+    "aq_testing_clear_device_errors": (_I, []),
 }
 
 
@@ -83,8 +86,11 @@ def check(status, fn):
 
 
 def declared_symbols():
-    """Names of the functions include/aq.h declares with AQ_API."""
+    """Names of the functions the headers under include/ declare with AQ_API."""
+    import glob
     import re
-    with open(HEADER) as f:
-        text = f.read()
-    return re.findall(r"AQ_API\s+[\w\s\*]+?\b(aq_\w+)\s*\(", text)
+    names = []
+    for path in sorted(glob.glob(os.path.join(os.path.dirname(HEADER), "*.h"))):
+        with open(path) as f:
+            names += re.findall(r"AQ_API\s+[\w\s\*]+?\b(aq_\w+)\s*\(", f.read())
+    return names

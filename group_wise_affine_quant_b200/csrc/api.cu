@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "../../include/aq_testing.h"
 
 namespace {
 
@@ -308,6 +309,15 @@ aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void*
   return cuda_status(aq::launch_qmm(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
                                     mode, dtype, (cudaStream_t)stream),
                      "aq_qmm launch");
+}
+
+void aq_testing_set_wait_limit_ns(uint64_t ns) { aq::testing_set_mv_wait_ns(ns); }
+void aq_testing_set_start_delay_ns(uint64_t ns) { aq::testing_set_mv_delay_ns(ns); }
+aq_status aq_testing_clear_device_errors(void) {
+  g_err[0] = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = aq::testing_clear_device_error_qmv_mma();
+  return cuda_status(e, "aq_testing_clear_device_errors");
 }
 
 unsigned aq_device_errors(void) {

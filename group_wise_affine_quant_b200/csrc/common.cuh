@@ -164,6 +164,10 @@ cudaError_t launch_qmv_mma(const void* x, const void* w_q, const void* scales,
 cudaError_t launch_qmv_mma_batched(const QmvProblemDesc* probs, int count, int64_t M, int gs,
                                    int dtype, void* ws, cudaStream_t st);
 cudaError_t read_device_error_qmv_mma(unsigned* out);
+// Test hooks of the warp-MMA decode kernel (aq_testing.h).
+void testing_set_mv_wait_ns(uint64_t ns);
+void testing_set_mv_delay_ns(uint64_t ns);
+cudaError_t testing_clear_device_error_qmv_mma();
 // aq_qmv_noalloc's fixed scratch (a file-scope device array in qmv_mma.cu).
 constexpr size_t kQmvNoallocScratchBytes = (size_t)4 << 20;
 // Launches the warp-MMA decode kernel on that scratch.  Sets *need to the

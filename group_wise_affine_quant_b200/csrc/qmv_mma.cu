@@ -83,6 +83,8 @@ struct MvParams {
   int weights_early;    // stream weights / scales / biases before the grid dependency wait
   int pad_;
   uint32_t* ws;
+  uint64_t wait_ns;     // bound of every mbarrier wait
+  uint64_t delay_ns;    // test hook: TMA warp start delay (0 = none)
 };
 
 // K columns per sub-slice: 8 groups (the scale boxes are 16-byte rows),
@@ -197,9 +199,9 @@ __device__ __forceinline__ MvUnit mv_unit(const MvParams<P>& pr, int u) {
 
 // Next unit id from the CTA's unit queue (-1: no more units; -2: a wait gave up).
 __device__ __forceinline__ int mv_take(volatile int* uq, uint64_t* uqf, uint64_t* uqe, int k,
-                                       int lane, volatile int* abort_flag) {
+                                       int lane, volatile int* abort_flag, uint64_t wl) {
   const int qs = k % kMvQ;
-  if (!mbar_wait(smem_u32(uqf + qs), (k / kMvQ) & 1, abort_flag)) return -2;
+  if (!mbar_wait(smem_u32(uqf + qs), (k / kMvQ) & 1, abort_flag, wl)) return -2;
   const int u = uq[qs];
   __syncwarp();
   if (lane == 0) mbar_arrive(smem_u32(uqe + qs));
@@ -250,6 +252,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
   const int g = lane >> 2, t = lane & 3;
   const int M = pr.M;
   const int total = pr.unit_end[pr.count - 1];
+  const uint64_t wl = pr.wait_ns;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
@@ -279,6 +282,11 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
     if (lane == 0) {
       bool waited = !pr.weights_early;
       if (waited) pdl_wait();
+      if (pr.delay_ns) {                       // test hook: hold back the first copy
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < pr.delay_ns && !*abort_flag) {
+        }
+      }
       const uint64_t pol = l2_policy_evict_first();
       // Units: the first one of each CTA is blockIdx.x; later ones are claimed
       // from the launch's unit counter (after the wait on the previous kernel,
@@ -286,7 +294,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
       int posted = 0;
       auto post = [&](int uu) -> bool {
         const int qs = posted % kMvQ;
-        if (!mbar_wait(smem_u32(uqe + qs), ((posted / kMvQ) & 1) ^ 1, abort_flag)) return false;
+        if (!mbar_wait(smem_u32(uqe + qs), ((posted / kMvQ) & 1) ^ 1, abort_flag, wl)) return false;
         uq[qs] = uu;
         mbar_arrive(smem_u32(uqf + qs));
         ++posted;
@@ -301,7 +309,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
         for (int j = 0; j < un.nsub && ok; ++j) {
           const int kk = un.k0 + j * SUBK;
           const int buf = sc & 1;
-          if (!mbar_wait(smem_u32(sbe + buf), ((sc >> 1) & 1) ^ 1, abort_flag)) break;
+          if (!mbar_wait(smem_u32(sbe + buf), ((sc >> 1) & 1) ^ 1, abort_flag, wl)) break;
           mbar_arrive_expect_tx(smem_u32(sbf + buf), 2 * S::kSbArr);
           uint8_t* sb = smem + S::kSbOff + buf * 2 * S::kSbArr;
           tma_load_2d(smem_u32(sb), &q.s, smem_u32(sbf + buf), kk / GS, row0);
@@ -309,7 +317,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
           ++sc;
           for (int st = 0; st < S::kSps; ++st) {
             const int slot = wc % ST;
-            if (!mbar_wait(smem_u32(empty + slot), ((wc / ST) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(smem_u32(empty + slot), ((wc / ST) & 1) ^ 1, abort_flag, wl)) { ok = false; break; }
             mbar_arrive_expect_tx(smem_u32(full + slot), S::kStage);
             tma_load_2d_hint(smem_u32(smem + S::kRingOff + slot * S::kStage), &q.w,
                              smem_u32(full + slot), (kk + st * S::kStageK) / 2, row0, pol);
@@ -335,7 +343,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
     int c = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int u = mv_take(uq, uqf, uqe, k, lane, abort_flag);
+      const int u = mv_take(uq, uqf, uqe, k, lane, abort_flag, wl);
       if (u < 0) { ok = u == -1; break; }
       const MvUnit un = mv_unit<P, SUBK>(pr, u);
       const MvProblem& q = pr.prob[un.p];
@@ -344,7 +352,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
         if ((c & 1) != b) continue;
         const uint32_t par = (c >> 1) & 1;
         uint8_t* xb = smem + S::kXOff + b * S::kXBuf;
-        if (!mbar_wait(smem_u32(xe + b), par ^ 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(xe + b), par ^ 1, abort_flag, wl)) { ok = false; break; }
         // x columns of the sub-slice (natural order; 64-byte blocks of 32 columns
         // at a row pitch of 64 mod 128 bytes), copied with cp.async
         const int kk = un.k0 + j * SUBK;
@@ -356,7 +364,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
                      reinterpret_cast<const uint4*>(xg + (int64_t)m * q.K + kk) + ch);
         }
         // fp32 (s, b - off * s) per weight row and group (while the x copy is in flight)
-        if (!mbar_wait(smem_u32(sbf + b), par, abort_flag)) {
+        if (!mbar_wait(smem_u32(sbf + b), par, abort_flag, wl)) {
           cp_async_wait_all();                              // no copy may outlive the CTA
           ok = false;
           break;
@@ -404,7 +412,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
     int wc = 0, c = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int u = mv_take(uq, uqf, uqe, k, lane, abort_flag);
+      const int u = mv_take(uq, uqf, uqe, k, lane, abort_flag, wl);
       if (u < 0) { ok = u == -1; break; }
       const MvUnit un = mv_unit<P, SUBK>(pr, u);
       const MvProblem& q = pr.prob[un.p];
@@ -417,7 +425,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
           for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.0f;
       for (int j = 0; j < un.nsub && ok; ++j) {
         const int buf = c & 1;
-        if (!mbar_wait(smem_u32(xf + buf), (c >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(xf + buf), (c >> 1) & 1, abort_flag, wl)) { ok = false; break; }
         const uint8_t* xb = smem + S::kXOff + buf * S::kXBuf + t * 16;
         float* xsw = reinterpret_cast<float*>(smem + S::kXsOff + buf * S::kXsBuf);
         {
@@ -451,14 +459,14 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(xsr + buf));
-          if (!mbar_wait(smem_u32(xsr + buf), (c >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(xsr + buf), (c >> 1) & 1, abort_flag, wl)) { ok = false; break; }
         }
         const float* xs = xsw + 2 * t;
         const float2* tab = reinterpret_cast<const float2*>(smem + S::kTabOff + buf * S::kTabBuf) +
                             (warp * 16 * R + g) * S::kTabPitch;
         for (int st = 0; st < S::kSps; ++st) {
           const int slot = wc % ST;
-          if (!mbar_wait(smem_u32(full + slot), (wc / ST) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(full + slot), (wc / ST) & 1, abort_flag, wl)) { ok = false; break; }
           const uint8_t* w0 = smem + S::kRingOff + slot * S::kStage + (warp * 16 * R + g) * 128 + t * 4;
           float d[R][NT][4];
           // codes of rows g and g + 8 of both tiles, and x, one step ahead
@@ -617,6 +625,9 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
 }
 
 // ------------------------------------------------------------------- host
+// Test hooks (aq_testing.h): wait bound and TMA-warp start delay, in ns.
+std::atomic<uint64_t> g_mv_wait_ns{0}, g_mv_delay_ns{0};
+
 struct MvSplit {
   int splits, kslice;
 };
@@ -763,6 +774,9 @@ cudaError_t mv_launch_group(const QmvProblemDesc* probs, int count, int64_t M, v
   pr.M = (int)M;
   pr.weights_early = weight_prefetch_enabled();
   pr.ws = reinterpret_cast<uint32_t*>(ws);
+  const uint64_t wl = g_mv_wait_ns.load(std::memory_order_relaxed);
+  pr.wait_ns = wl ? wl : 2000000000ull;
+  pr.delay_ns = g_mv_delay_ns.load(std::memory_order_relaxed);
   const int grid = std::min(units, slots);
   return MvKernel<T, GS, NT, P>::launch(pr, grid, st);
 }
@@ -837,6 +851,13 @@ cudaError_t launch_qmv_mma_batched(const QmvProblemDesc* probs, int count, int64
 }
 
 cudaError_t read_device_error_qmv_mma(unsigned* out) { return read_tu_error(out); }
+
+void testing_set_mv_wait_ns(uint64_t ns) { g_mv_wait_ns.store(ns, std::memory_order_relaxed); }
+void testing_set_mv_delay_ns(uint64_t ns) { g_mv_delay_ns.store(ns, std::memory_order_relaxed); }
+cudaError_t testing_clear_device_error_qmv_mma() {
+  const unsigned z = 0;
+  return cudaMemcpyToSymbol(g_aq_device_error, &z, sizeof(z));
+}
 
 // ------------------------------------------------ no-allocation entry point
 // Scratch of aq_qmv_noalloc, in place of a caller-supplied workspace: the

@@ -1,0 +1,39 @@
+/*
+ * aq_testing.h — test hooks of libaq (not for production use).
+ *
+ * They let a test drive the failure path of the decode kernels' bounded waits
+ * (the bound every mbarrier wait of a kernel has, after which the kernel stops
+ * issuing work, lets its copies in flight land, sets bit 0 of
+ * aq_device_errors() and returns) without faulting the GPU: the host shortens
+ * the bound and delays one role of the kernel past it, so that the waits of
+ * the other roles run out.  The pages have no counterpart.
+ *
+ * Scope: the warp-MMA decode kernel behind aq_qmv / aq_qmv_batched /
+ * aq_qmv_noalloc (4-bit affine weights).  The settings are process-wide and
+ * apply to launches made after the call; 0 restores the default.
+ */
+#ifndef AQ_TESTING_H
+#define AQ_TESTING_H
+
+#include "aq.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Bound of every mbarrier wait of the decode kernel, in ns (default 2 s). */
+AQ_API void aq_testing_set_wait_limit_ns(uint64_t ns);
+
+/* Delay, in ns, before the decode kernel's TMA warp issues its first copy
+ * (default 0).  The delay ends early once another role has given up. */
+AQ_API void aq_testing_set_start_delay_ns(uint64_t ns);
+
+/* Clears the device error bits that aq_device_errors() reports.  Synchronises
+ * the current device first. */
+AQ_API aq_status aq_testing_clear_device_errors(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif
