@@ -71,13 +71,27 @@ def test_conv_full_size(groups, bits):
 
 
 def test_conv_matches_qmm_on_explicit_im2col():
-    """A 1x1 stride-1 conv is a plain matmul over pixels: compare with aq_qmm."""
+    """A 1x1 stride-1 conv is a plain matmul over pixels: the conv and aq_qmm
+    on the pixels-by-channels matrix both meet the matmul bound against the
+    oracle's product of that matrix (w_hat rounded to T, as both kernels
+    dequantize into T)."""
     B, H, W, C, Co, gs, bits = 2, 16, 16, 64, 96, 64, 4
     xd, wq, s, b, y = _conv_case(B, H, W, C, Co, 1, 1, 0, 1, bits, gs, 1, seed=5)
-    y2 = api.aq_qmm(xd.reshape(B * H * W, C), wq, s, b, bits, gs)
+    x2 = xd.reshape(B * H * W, C)
+    y2 = api.aq_qmm(x2, wq, s, b, bits, gs)
     torch.cuda.synchronize()
-    d = (y.reshape(-1, Co).float() - y2.float()).abs().max().item()
-    assert d <= 2e-2, d
+    yr, den = oracle.qmm(dev_u16(x2), dev_u8(wq), dev_u16(s), dev_u16(b), Co, bits, gs, 0, 1,
+                         w_in_t=True)
+    check_matmul(dev_u16(y).reshape(-1, Co), yr, den, 1, what="1x1 conv")
+    check_matmul(dev_u16(y2), yr, den, 1, what="aq_qmm")
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors():
+    """Every conv case must finish without a bounded wait running out."""
+    yield
+    torch.cuda.synchronize()
+    assert api.lib().aq_device_errors() == 0
 
 
 def test_conv_rejects_unaligned_channels():
