@@ -12,21 +12,24 @@
 //     operand (N = BT in 16..256 rows of M), so a decode-sized M still fills a
 //     full 128-row MMA: one wave of tiles covers M = 1..64 at the weight
 //     stream's cost.
-//   * Warp 0 (one thread) loads x tiles with TMA into 128-byte-swizzled shared
-//     memory; warp 6 streams the packed codes and the words holding each
-//     row's scales and biases into a deep shared-memory ring with cp.async,
-//     completing on an mbarrier; warp 1 allocates TMEM and one of its threads
-//     issues tcgen05.mma (kind::f16, fp32 accumulate in TMEM); warps 2-5 are
-//     the dequantizers (one weight row per thread): from shared memory they
-//     form w_hat = s*q + b in T with packed half2/bfloat162 FMAs (single
-//     rounding, the same value aq_dequantize writes) and store it in the
-//     swizzled K-major layout.  The dequantizers issue no global loads, so
-//     their async-proxy fence before each hand-over never waits on memory
-//     latency.  Stages hand over through mbarriers; the MMA's commit frees an
-//     operand stage for both producers.
+//   * Warp 0 is the x producer: a warp-uniform loop whose elected lane issues
+//     each x tile's TMA into 128-byte-swizzled shared memory (or, for the
+//     conv, 4-D boxes per filter tap / a cp.async gather).  Warp 1 allocates
+//     TMEM and issues the tcgen05.mma (kind::f16, fp32 accumulate in TMEM)
+//     from an elected lane, one wait and one commit per stage.  The last warp
+//     streams the packed codes and the scale / bias chunks by TMA (128 rows x
+//     128 bytes, 128-byte swizzle) into a ring, or by cp.async when the rows
+//     are not 16-byte multiples.  Warps 2 .. 2+4G-1 are G groups of four
+//     dequantizers on interleaved K-stages (one weight row per thread): they
+//     form w_hat = s*q + b in T with packed FMAs (single rounding, the value
+//     aq_dequantize writes) and store it into tensor memory with
+//     tcgen05.st; the MMA reads its A operand from TMEM, so the dequantized
+//     tile never passes through shared memory.  Stages hand over through
+//     mbarriers; the MMA's commit frees an operand slot for both producers.
 //   * K-step 64 (one 128-byte swizzle atom of 16-bit values); a K tail of 32
 //     reads zero x through TMA's out-of-bounds fill and writes zero w_hat.
-//   * The epilogue (warps 2-5) reads TMEM with tcgen05.ld.  With split-K the
+//   * The epilogue (the dequantizer warps) reads TMEM with tcgen05.ld and
+//     stores y through shared memory in 16-byte runs.  With split-K the
 //     K-slices of a tile form a thread block cluster: each CTA parks its fp32
 //     tile in shared memory and the slices are added in slice order through
 //     distributed shared memory.  No workspace, no global atomics.

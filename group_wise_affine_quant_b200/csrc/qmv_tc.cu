@@ -2,7 +2,10 @@
 // tensor cores, with the scale and bias applied in fp32 per group:
 //   y[m, n] = sum_g ( s[n,g] * sum_{k in g} q[n,k] x[m,k]  +  b[n,g] * sum_{k in g} x[m,k] )
 // for one problem (aq_qmv) or for a list of independent problems in one
-// launch (aq_qmv_batched).
+// launch (aq_qmv_batched).  4-bit affine weights whose K is a multiple of the
+// 512-column sub-slice run the warp-MMA kernel of qmv_mma.cu instead; this
+// kernel serves the other widths (2, 3, 5, 6, 8 bits), FP4 and the other
+// shapes with 16-byte packed and scale rows.
 //
 // Prior art: affine_packed_qmv_fast in "Add the 3bit packed qmm_t" keeps the
 // dot product in fp32 and hoists scale and bias out of each group (result +=
