@@ -30,8 +30,9 @@
 //     9-10 prepare each 512-column sub-slice (1024 for group size 128): they
 //     turn the raw scales and biases into fp32 (s, b - off * s) pairs, copy
 //     the x columns into shared memory in the order the codes unpack, and add
-//     the per-group x sums.  Sub-slice buffers are double-buffered, so the
-//     MMA warps' inner loop waits only on weight stages.
+//     the per-group x sums (fp32, a fixed shuffle tree over a group's lanes).
+//     Sub-slice buffers are double-buffered, so the MMA warps' inner loop
+//     waits only on weight stages.
 //   * Unpack: a 32-bit word holds codes c0..c7 at bits 4i; the pair
 //     (c_i, c_{i+4}) is ((w >> 4i) & 0x000F000F) | magic, which is one
 //     bf16x2 / fp16x2 A register.  x is stored as (x0,x4),(x2,x6),(x1,x5),
@@ -225,6 +226,12 @@ template <typename T> constexpr uint32_t ones2() {
   return std::is_same<T, __nv_bfloat16>::value ? 0x3F803F80u : 0x3C003C00u;
 }
 
+// Up to this many rows of x, the prep warp adds the per-group x sums (fp32
+// adds and a shuffle tree); above it the MMA warps do, with an all-ones MMA
+// each for its share of the groups, because the prep warp's adds over more
+// rows would fall behind the weight stream.
+constexpr int kMvPrepSumsMaxM = 4;
+
 template <typename T, int GS, int NT, int R, int P>
 __global__ void __launch_bounds__(MvShape<GS, NT, R>::kThreads, 2)
 qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
@@ -243,7 +250,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
   uint64_t* sbe = sbf + 2;               // raw scales / biases converted (its prep warp)
   uint64_t* xf = sbe + 2;                // sub-slice prepared (its prep warp)
   uint64_t* xe = xf + 2;                 // sub-slice consumed (the MMA warps)
-  uint64_t* xsr = xe + 2;                // per-group x sums of a sub-slice written (the MMA warps)
+  uint64_t* xsr = xe + 2;                // per-group x sums written (the MMA warps, M > kMvPrepSumsMaxM)
   uint64_t* uqf = xsr + 2;               // unit id posted (producer)
   uint64_t* uqe = uqf + kMvQ;            // unit id read (every prep and MMA warp)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + S::kBars);
@@ -388,17 +395,37 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(sbe + b));
         cp_async_wait_all();
-        // reorder each 8-column chunk in place to the order the codes unpack:
-        // (x0,x4), (x2,x6), (x1,x5), (x3,x7)
-        for (int i = lane; i < nch; i += 32) {
-          uint4* pc = reinterpret_cast<uint4*>(xb + (i / kCpr) * S::kXP + (i % kCpr) * 16);
+        // Reorder each 8-column chunk in place to the order the codes unpack,
+        // (x0,x4), (x2,x6), (x1,x5), (x3,x7), and add the per-group x sums: a
+        // group's GS/8 chunks sit on GS/8 consecutive lanes of one pass (a row
+        // has a multiple of 32 chunks), which add their chunk sums by a fixed
+        // shuffle tree.
+        float* xs = reinterpret_cast<float*>(smem + S::kXsOff + b * S::kXsBuf);
+        constexpr int kSeg = GS / 8;                          // lanes per group
+        static_assert(kCpr % 32 == 0, "a pass of the warp covers whole groups of one row");
+        for (int i0 = 0; i0 < nch; i0 += 32) {
+          const int i = i0 + lane;                            // nch is a multiple of 32
+          const int m = i / kCpr, ch = i % kCpr;
+          uint4* pc = reinterpret_cast<uint4*>(xb + m * S::kXP + ch * 16);
           const uint4 v = *pc;
-          uint4 o;
-          o.x = __byte_perm(v.x, v.z, 0x5410);
-          o.y = __byte_perm(v.y, v.w, 0x5410);
-          o.z = __byte_perm(v.x, v.z, 0x7632);
-          o.w = __byte_perm(v.y, v.w, 0x7632);
-          *pc = o;
+          const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+          if (M <= kMvPrepSumsMaxM) {                         // warp-uniform
+            float sum = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              sum += t_to_f(r[e] & 0xFFFFu, kBf16);
+              sum += t_to_f(r[e] >> 16, kBf16);
+            }
+#pragma unroll
+            for (int o = 1; o < kSeg; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if ((lane & (kSeg - 1)) == 0) xs[(ch / kSeg) * 16 + m] = sum;
+          }
+          uint4 ov;
+          ov.x = __byte_perm(v.x, v.z, 0x5410);
+          ov.y = __byte_perm(v.y, v.w, 0x5410);
+          ov.z = __byte_perm(v.x, v.z, 0x7632);
+          ov.w = __byte_perm(v.y, v.w, 0x7632);
+          *pc = ov;
         }
         __syncwarp();
         __syncwarp();
@@ -428,7 +455,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
         if (!mbar_wait(smem_u32(xf + buf), (c >> 1) & 1, abort_flag, wl)) { ok = false; break; }
         const uint8_t* xb = smem + S::kXOff + buf * S::kXBuf + t * 16;
         float* xsw = reinterpret_cast<float*>(smem + S::kXsOff + buf * S::kXsBuf);
-        {
+        if (M > kMvPrepSumsMaxM) {
           // Per-group sums of each x row, GPS / kMvWarps groups per warp: an MMA
           // with an all-ones A operand adds the K-steps' columns.
           const uint32_t one[4] = {ones2<T>(), ones2<T>(), ones2<T>(), ones2<T>()};
