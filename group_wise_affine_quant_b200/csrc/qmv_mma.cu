@@ -174,6 +174,15 @@ __device__ __forceinline__ uint32_t and_or(uint32_t v, uint32_t mask, uint32_t m
   return r;
 }
 
+// Atomic add at GPU scope with release semantics: the calling thread's prior
+// writes, and those it has observed (a warp's, after __syncwarp), are visible
+// before the addition is.
+__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ float t_to_f(uint32_t h, bool bf16) {
   return bf16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
 }
@@ -339,6 +348,17 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
         u = (int)gridDim.x + (int)atomicAdd(pr.ws, 1u);
       }
       if (!*abort_flag) post(-1);                           // no more units
+      // This CTA claims no more units: count it out, and the last CTA to do so
+      // puts the launch's unit counter back to zero (every claim of the launch
+      // has then been made), off the critical path of the last unit.
+      if (!waited) {
+        pdl_wait();
+        waited = true;
+      }
+      if (atomicAdd(pr.ws + 1, 1u) == gridDim.x - 1) {
+        atomicExch(pr.ws, 0u);
+        atomicExch(pr.ws + 1, 0u);
+      }
       mv_drain(full, ST, wc, abort_flag);
       mv_drain(sbf, 2, sc, abort_flag);
     }
@@ -602,10 +622,9 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
               const int m = 8 * nt + 2 * t + (i & 1), rr = g + 8 * (i >> 1);
               if (m < M) __stcg(mine + m * 16 + rr, acc[r][nt][i]);
             }
-          __threadfence();
-          __syncwarp();
+          __syncwarp();                                     // the warp's partial stores ...
           unsigned old = 0;
-          if (lane == 0) old = atomicAdd(cnt, 1u);
+          if (lane == 0) old = atom_add_release_gpu(cnt, 1u); // ... released with the count
           old = __shfl_sync(0xffffffffu, old, 0);
           if (old == (unsigned)(q.splits - 1)) {
             __threadfence();
@@ -640,15 +659,7 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
   }
 
   __syncthreads();
-  if (threadIdx.x == 0) {
-    if (*abort_flag) atomicOr(&g_aq_device_error, 1u);
-    // The last CTA to leave puts the launch's unit counter back to zero.
-    __threadfence();
-    if (atomicAdd(pr.ws + 1, 1u) == gridDim.x - 1) {
-      atomicExch(pr.ws, 0u);
-      atomicExch(pr.ws + 1, 0u);
-    }
-  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(&g_aq_device_error, 1u);
 }
 
 // ------------------------------------------------------------------- host

@@ -34,7 +34,8 @@ def _check(x, wq, s, b, y, bits, gs, dt, mode=0, w_in_t=True, **kw):
     return check_matmul(dev_u16(y), yr, den, dt, **kw)
 
 
-def _check_sampled(x, wq, s, b, y, bits, gs, dt, n_samples=512, seed=0, mode=0, **kw):
+def _check_sampled(x, wq, s, b, y, bits, gs, dt, n_samples=512, seed=0, mode=0, w_in_t=True,
+                   **kw):
     M, N = y.shape
     rng = np.random.default_rng(seed)
     ms = np.concatenate([[0, M - 1, M - 1, 0], rng.integers(0, M, n_samples)])
@@ -42,7 +43,7 @@ def _check_sampled(x, wq, s, b, y, bits, gs, dt, n_samples=512, seed=0, mode=0, 
     sc = dev_u8(s) if mode == 1 else dev_u16(s)
     bi = None if b is None else dev_u16(b)
     yr, den = oracle.qmm_sampled(dev_u16(x), dev_u8(wq), sc, bi, N, bits, gs, mode, dt, ms, ns,
-                                 w_in_t=True)
+                                 w_in_t=w_in_t)
     ys = dev_u16(y)[ms, ns]
     return check_matmul(ys, yr, den, dt, **kw)
 
@@ -181,6 +182,32 @@ def test_qmm_fp4_full_size(gs, scale_range, M):
     torch.cuda.synchronize()
     _check_sampled(xd, wq, sc, None, y, 4, gs, 1, mode=1,
                    overflow_any_nonfinite=(scale_range == "literal"))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_qmm_chained_meets_bound_over_exact_w(bits):
+    """The literal tolerance over the EXACT w_hat (not w_hat rounded to T) at
+    the chained workload's size (fp16, K = 1024): the tensor-core product of
+    the T-rounded tile stays within 2e-3 * sum |x w_hat| + 1 ulp."""
+    x, w1, _ = inputs.chained()
+    q1 = api.aq_quantize(to_dev(w1), bits, 64)
+    xd = to_dev(x)
+    h = api.aq_qmm(xd, *q1, bits, 64)
+    torch.cuda.synchronize()
+    _check_sampled(xd, *q1, h, bits, 64, 0, seed=40 + bits, w_in_t=False)
+
+
+@pytest.mark.parametrize("M", [32, 64])
+def test_qmm_decode_projection_meets_bound_over_exact_w(M):
+    """The same at the decode sweep's gate projection through aq_qmm (bf16,
+    8192 x 2048, the coarser T)."""
+    g = inputs.gen(60 + M)
+    w = inputs.normal((8192, 2048), 0.02, 1, g)
+    x = to_dev(inputs.normal((M, 2048), 1.0, 1, g))
+    wq, s, b = api.aq_quantize(to_dev(w), 4, 64)
+    y = api.aq_qmm(x, wq, s, b, 4, 64)
+    torch.cuda.synchronize()
+    _check_sampled(x, wq, s, b, y, 4, 64, 1, seed=M, w_in_t=False)
 
 
 def test_qmm_matches_qmv_small_m():
