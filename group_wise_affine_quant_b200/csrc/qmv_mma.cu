@@ -102,7 +102,7 @@ struct MvShape {
   static constexpr int kGps = kSubK / GS;                      // groups per sub-slice
   static constexpr int kStageK = 256;                          // 128 bytes of 4-bit codes per row
   static constexpr int kSps = kSubK / kStageK;                 // stages per sub-slice
-  static constexpr int kST = 3;                                // weight stages
+  static constexpr int kST = NT == 1 ? 4 : 3;                  // weight stages (shared memory: 2 CTAs per SM)
   static constexpr int kStage = kMvRows * 128;                 // 16 KB
   static constexpr int kXP = kSubK * 2 + 64;                   // x row pitch: 64 mod 128 bytes
   static constexpr int kXBuf = 8 * NT * kXP;
@@ -193,8 +193,14 @@ struct MvUnit {
 
 template <int P, int SUBK>
 __device__ __forceinline__ MvUnit mv_unit(const MvParams<P>& pr, int u) {
-  int p = 0;
-  while (p + 1 < pr.count && u >= pr.unit_end[p]) ++p;
+  // the problem whose cumulative unit range holds u (binary search)
+  int lo = 0, hi = pr.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (u >= pr.unit_end[mid]) lo = mid + 1;
+    else hi = mid;
+  }
+  const int p = lo;
   const MvProblem& q = pr.prob[p];
   const int local = u - (p ? pr.unit_end[p - 1] : 0);
   const int rbs = (q.N + kMvRows - 1) / kMvRows;
