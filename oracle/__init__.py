@@ -39,6 +39,11 @@ def lib():
         for name in ("orc_e2m1", "orc_e8m0", "orc_e4m3"):
             getattr(_lib, name).argtypes = [I]
             getattr(_lib, name).restype = ctypes.c_double
+        for name in ("orc_e8m0_encode", "orc_e4m3_encode", "orc_e2m1_encode"):
+            getattr(_lib, name).argtypes = [ctypes.c_float]
+            getattr(_lib, name).restype = I
+        _lib.orc_quantize_fp4.argtypes = [P, I64, I64, I, I, P, P]
+        _lib.orc_quantize_fp4.restype = I
         _lib.orc_quantize.argtypes = [P, I64, I64, I, I, I, P, P, P]
         _lib.orc_unpack.argtypes = [P, I64, I64, I, P]
         _lib.orc_dequantize.argtypes = [P, P, P, I64, I64, I, I, I, I, P, P]
@@ -108,6 +113,32 @@ def quantize(w16, bits, gs, dt):
     b = np.zeros((N, G), np.uint16)
     _check(lib().orc_quantize(_p(w16), N, K, bits, gs, dt, _p(wq), _p(s), _p(b)), "quantize")
     return wq, s, b
+
+
+def e8m0_encode(x):
+    """[P4] to_fp8_e8m0 of a float (the exact log-scale reading)."""
+    return lib().orc_e8m0_encode(float(x))
+
+
+def e4m3_encode(x):
+    """E4M3FN encoding of a float: ties to even, saturating at 448."""
+    return lib().orc_e4m3_encode(float(x))
+
+
+def e2m1_encode(x):
+    """[P4] to_fp4_e2m1 of a float."""
+    return lib().orc_e2m1_encode(float(x))
+
+
+def quantize_fp4(w16, gs, dt):
+    """w16: [N, K] uint16 T patterns -> (codes [N, K/2] u8, scales [N, K/gs] u8);
+    E8M0 scales for gs = 32, E4M3 for gs = 16."""
+    w16 = _c(w16, np.uint16)
+    N, K = w16.shape
+    codes = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, K // gs), np.uint8)
+    _check(lib().orc_quantize_fp4(_p(w16), N, K, gs, dt, _p(codes), _p(scales)), "quantize_fp4")
+    return codes, scales
 
 
 def unpack(wq, N, K, bits):

@@ -19,7 +19,9 @@
 //        min..max, scale adjusted so that 0 lands on the grid.
 //   [P4] "mlx 1.0.0, mlx/backend/cpu/quantized.cpp": the quantize routine
 //        (fp32 arithmetic, packing), get_pack_factor / get_bytes_per_pack,
-//        extract_bits, FP4_LUT, dequantize_scale (E8M0 / FP8 scales), fp_qmm_t.
+//        extract_bits, FP4_LUT, dequantize_scale (E8M0 / FP8 scales), fp_qmm_t,
+//        and the FP4 quantizer's steps: to_fp8_e8m0, to_fp4_e2m1 and
+//        fp_quantize_dequantize (scale = absmax / 6).
 //
 // Precision.  The quantizer runs in fp32, in the order the quantize routine of
 // [P4] takes its steps, because its codes, scales and biases are fixed by fp32
@@ -174,6 +176,69 @@ double fp_scale_in_t(uint8_t s, int gs, int dt) {
   return t_to_double(round_to_t(v, dt), dt);
 }
 
+// ------------------------------------------------------- FP4 quantizer
+// The steps of [P4] fp_quantize_dequantize for 4-bit codes, up to the codes
+// and the scale byte (the library's FP4 weight format), with two readings:
+//   * to_fp8_e8m0 takes n = round(log2(x)) in float.  Reading: the exact
+//     nearest power of two on a log scale, i.e. x = m * 2^e (m in [1, 2))
+//     rounds to 2^(e+1) exactly when m >= sqrt(2) (a float is never equal
+//     to sqrt(2), so the tie rule never applies).  x = 0 has log2 = -inf,
+//     which the clamp maps to -127.
+//   * detail::ToFP8 (the E4M3 scale of group 16) has no body on the pages.
+//     Reading: OCP E4M3FN, round to nearest with ties to even, finite values
+//     and infinities saturated to +-448, NaN to 0x7F.
+unsigned e8m0_encode(float x) {
+  if (!std::isfinite(x)) return 0xFF;
+  if (x < 0.0f) return 0x00;
+  if (x == 0.0f) return 0x00;                    // n = -127
+  int e;
+  const double fr = std::frexp((double)x, &e);   // x = fr * 2^e, fr in [0.5, 1)
+  const double m = 2.0 * fr;                     // x = m * 2^(e-1), m in [1, 2)
+  int n = (m * m >= 2.0) ? e : e - 1;            // m >= sqrt(2); m*m is exact in double
+  n = n < -127 ? -127 : (n > 127 ? 127 : n);
+  return (unsigned)(n + 127);
+}
+
+unsigned e4m3_encode(float xf) {
+  if (std::isnan(xf)) return 0x7F;
+  const unsigned sign = std::signbit(xf) ? 0x80u : 0u;
+  const double a = std::fabs((double)xf);
+  if (a == 0.0) return sign;
+  const double kMax = 448.0;
+  if (a > kMax) return sign | 0x7E;              // saturate (infinities too)
+  int e;
+  std::frexp(a, &e);
+  e -= 1;                                        // a in [2^e, 2^(e+1))
+  const int q = e < -6 ? -6 : e;                 // below 2^-6: the subnormal quantum
+  const double quantum = std::ldexp(1.0, q - 3); // 3 fraction bits
+  double r = std::nearbyint(a / quantum) * quantum;   // ties to even (default mode)
+  if (r > kMax) r = kMax;
+  if (r == 0.0) return sign;
+  int re;
+  std::frexp(r, &re);
+  re -= 1;
+  if (re < -6) return sign | (unsigned)std::ldexp(r, 9);          // E = 0: m * 2^-9
+  const unsigned m = (unsigned)(std::ldexp(r, 3 - re) - 8.0);
+  return sign | ((unsigned)(re + 7) << 3) | m;
+}
+
+// [P4] to_fp4_e2m1: the threshold table (round to nearest, ties to even).
+unsigned e2m1_encode(float x) {
+  if (std::isnan(x)) return 0x7;
+  const unsigned sign = std::signbit(x) ? 0x8u : 0u;
+  const float a = std::fabs(x);
+  unsigned bits;
+  if (a > 5.0f) bits = 0x7;
+  else if (a >= 3.5f) bits = 0x6;
+  else if (a > 2.5f) bits = 0x5;
+  else if (a >= 1.75f) bits = 0x4;
+  else if (a > 1.25f) bits = 0x3;
+  else if (a >= 0.75f) bits = 0x2;
+  else if (a > 0.25f) bits = 0x1;
+  else bits = 0x0;
+  return bits | sign;
+}
+
 // ----------------------------------------------------------------- dequant
 // One dequantized row: w_hat[k] exactly, in fp64.
 //   affine [P4] _qmm_t:      scale * q + bias   (scale, bias are T values)
@@ -256,6 +321,48 @@ uint16_t orc_round_to_t(double v, int dt) { return round_to_t(v, dt); }
 double orc_e2m1(int code) { return e2m1_value((unsigned)code & 15); }
 double orc_e8m0(int s) { return e8m0_value((unsigned)s & 255); }
 double orc_e4m3(int s) { return e4m3_value((unsigned)s & 255); }
+int orc_e8m0_encode(float x) { return (int)e8m0_encode(x); }
+int orc_e4m3_encode(float x) { return (int)e4m3_encode(x); }
+int orc_e2m1_encode(float x) { return (int)e2m1_encode(x); }
+
+// FP4 quantizer ([P4] fp_quantize_dequantize, 4-bit, up to the codes).  w is
+// [N, K] T; codes receives N rows of K/2 bytes (code k in the low nibble of
+// byte k/2 when k is even, the high nibble when odd); scales is [N, K/gs]
+// bytes: E8M0 for gs = 32, E4M3 for gs = 16.  Per group, in fp32:
+//   absmax = max_j |w_j|  (starting from -inf, as std::max does: NaN ignored)
+//   scale  = absmax / 6
+//   byte   = gs == 16 ? ToFP8(scale) : to_fp8_e8m0(scale)
+//   s      = the byte decoded to float (dequantize_scale<float>)
+//   code_j = to_fp4_e2m1(s == 0 ? 0 : w_j / s)
+int orc_quantize_fp4(const uint16_t* w, int64_t N, int64_t K, int gs, int dt, uint8_t* codes,
+                     uint8_t* scales) {
+  if (dt != DT_F16 && dt != DT_BF16) return 1;
+  if ((gs != 16 && gs != 32) || N < 0 || K < 0 || K % gs) return 1;
+  const int64_t G = K / gs;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < G; ++g) {
+      const uint16_t* wg = w + n * K + g * gs;
+      float amax = -std::numeric_limits<float>::infinity();
+      for (int j = 0; j < gs; ++j) {
+        const float a = std::fabs(t_to_float(wg[j], dt));
+        amax = (amax < a) ? a : amax;            // std::max(amax, a)
+      }
+      const float scale = amax / 6.0f;
+      const unsigned byte = gs == 16 ? e4m3_encode(scale) : e8m0_encode(scale);
+      const float sdec = (float)(gs == 16 ? e4m3_value(byte) : e8m0_value(byte));
+      scales[n * G + g] = (uint8_t)byte;
+      for (int j = 0; j < gs; ++j) {
+        const float el = sdec == 0.0f ? 0.0f : t_to_float(wg[j], dt) / sdec;
+        const unsigned c = e2m1_encode(el);
+        const int64_t k = g * gs + j;
+        uint8_t& dst = codes[n * (K / 2) + k / 2];
+        if (k % 2 == 0) dst = (uint8_t)((dst & 0xF0) | c);
+        else dst = (uint8_t)((dst & 0x0F) | (c << 4));
+      }
+    }
+  }
+  return 0;
+}
 
 // Affine quantizer, [P4] quantize and [P3] item 1.  w is [N, K] T row-major;
 // w_q receives N rows of K*bits/8 bytes; scales/biases are [N, K/gs] T.

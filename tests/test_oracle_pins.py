@@ -8,6 +8,7 @@ FP4_LUT, dequantize_scale, fp_qmm_t); "Improvements in the quantizer and
 dequantization kernel" (the scale/bias rule); "[Feature] Quantized
 Convolution 2D - Possible PR?" (flatten, pad, im2col order, grouped conv).
 """
+import math
 import os
 
 import numpy as np
@@ -503,3 +504,123 @@ def test_oracle_rejects_bad_arguments():
         oracle.quantize(w, 4, 16, F16)
     with pytest.raises(ValueError):
         oracle.quantize(np.zeros((2, 96), np.uint16), 4, 64, F16)
+
+
+# ---------------------------------------------------------------- FP4 quantizer
+# The steps of the FP4 quantize-dequantize in "mlx 1.0.0, .../quantized.cpp"
+# (to_fp8_e8m0, to_fp4_e2m1, fp_quantize_dequantize): pinned against brute
+# force over the FP4 value table, exact log2 arithmetic and torch's own
+# float8_e4m3fn conversion.
+
+def _fp4_magnitudes():
+    return [oracle.e2m1(c) for c in range(8)]          # the table pinned above
+
+
+def test_e2m1_encode_is_the_nearest_value_ties_to_even():
+    """to_fp4_e2m1's thresholds: every |x| maps to the nearest table value;
+    at a midpoint, to the one with an even mantissa bit (code bit 0 = 0)."""
+    mags = _fp4_magnitudes()
+    xs = np.concatenate([np.linspace(0.0, 7.0, 7001), [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]])
+    for x in xs:
+        x = float(np.float32(x))
+        d = [abs(x - v) for v in mags]
+        best = min(d)
+        cand = [c for c in range(8) if d[c] == best]
+        want = cand[0] if len(cand) == 1 else [c for c in cand if c % 2 == 0][0]
+        assert oracle.e2m1_encode(x) == want, x
+        assert oracle.e2m1_encode(-x) == want | 8, -x
+    assert oracle.e2m1_encode(float("nan")) == 7            # the page's NaN rule
+    assert oracle.e2m1_encode(100.0) == 7                   # saturates at 6
+
+
+def test_e8m0_encode_is_the_nearest_power_of_two_in_log_scale():
+    rng = np.random.default_rng(0)
+    xs = np.concatenate([2.0 ** np.arange(-126, 128, dtype=np.float64),
+                         rng.uniform(0.5, 2.0, 4000) * 2.0 ** rng.integers(-120, 120, 4000)])
+    for x in xs.astype(np.float32):
+        x = float(x)
+        # exact: log2(x) rounds up past k + 0.5 iff x >= 2^k * sqrt(2), i.e. x^2 >= 2^(2k+1)
+        k = math.floor(math.log2(x))
+        while 2.0 ** k > x:
+            k -= 1
+        while 2.0 ** (k + 1) <= x:
+            k += 1
+        n = k + 1 if x * x >= 2.0 ** (2 * k + 1) else k
+        n = max(-127, min(127, n))
+        assert oracle.e8m0_encode(x) == n + 127, x
+    # around sqrt(2): the last float below rounds down, the first above rounds up
+    lo = float(np.float32(1.4142135))
+    hi = float(np.nextafter(np.float32(lo), np.float32(2.0)))
+    assert lo * lo < 2.0 < hi * hi
+    assert oracle.e8m0_encode(lo) == 127 and oracle.e8m0_encode(hi) == 128
+    assert oracle.e8m0_encode(0.0) == 0                     # log2(0) = -inf, clamped
+    assert oracle.e8m0_encode(float("inf")) == 255 and oracle.e8m0_encode(float("nan")) == 255
+    assert oracle.e8m0_encode(3.0e38) == 254                # clamped to 127
+
+
+def test_e4m3_encode_matches_torch_float8():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(1)
+    xs = np.concatenate([np.linspace(0.0, 448.0, 20001),
+                         rng.uniform(0.0, 1.0, 4000) * 2.0 ** rng.integers(-12, 9, 4000)])
+    xs = xs[xs <= 448.0].astype(np.float32)
+    want = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(v)) for v in xs], np.uint8)
+    assert np.array_equal(got, want)
+    # the reading past the largest finite value: saturation (the scale is >= 0)
+    assert oracle.e4m3_encode(449.0) == 0x7E and oracle.e4m3_encode(float("inf")) == 0x7E
+    assert oracle.e4m3_encode(float("nan")) == 0x7F
+
+
+@pytest.mark.parametrize("gs", [16, 32])
+def test_quantize_fp4_recovers_table_multiples(gs):
+    """A group whose largest magnitude is 6 * 2^k: the scale is 2^k (exact in
+    both scale formats for the k used), and every element that is a table
+    value times 2^k comes back as its own code."""
+    rng = np.random.default_rng(gs)
+    mags = _fp4_magnitudes()
+    for dt in (0, 1):
+        for k in (-3, 0, 2):
+            codes = rng.integers(0, 16, gs)
+            codes[0] = 7                                     # the group's max: 6 * 2^k
+            vals = np.array([(-1.0 if c & 8 else 1.0) * mags[c & 7] * 2.0 ** k for c in codes])
+            w16 = np.array([[oracle.round_to_t(v, dt) for v in vals]], np.uint16)
+            q, s = oracle.quantize_fp4(w16, gs, dt)
+            assert s[0, 0] == (oracle.e4m3_encode(2.0 ** k) if gs == 16 else 127 + k)
+            got = np.stack([q[0] & 15, q[0] >> 4], axis=1).reshape(-1)
+            # -0 (code 8) encodes as sign 8 | 0 only when the value is -0.0
+            want = np.where((codes & 7) == 0, np.where(np.signbit(vals), 8, 0), codes)
+            assert np.array_equal(got, want), (dt, k, got, want)
+
+
+@pytest.mark.parametrize("gs", [16, 32])
+def test_quantize_fp4_is_nearest_on_the_scaled_table(gs):
+    """Random groups: the scale byte encodes absmax / 6, and each code is the
+    table value nearest to w / s (ties to even), with s the decoded scale."""
+    rng = np.random.default_rng(10 + gs)
+    mags = np.array(_fp4_magnitudes())
+    w = (rng.standard_normal((8, 4 * gs)) * 0.05).astype(np.float32)
+    w16 = np.array([[oracle.round_to_t(float(v), 1) for v in row] for row in w], np.uint16)
+    q, s = oracle.quantize_fp4(w16, gs, 1)
+    for n in range(8):
+        for g in range(4):
+            wg = np.array([oracle.t_to_double(h, 1) for h in w16[n, g * gs:(g + 1) * gs]])
+            amax = np.float32(np.max(np.abs(wg)))
+            sc = np.float32(amax / np.float32(6.0))
+            enc = oracle.e4m3_encode(float(sc)) if gs == 16 else oracle.e8m0_encode(float(sc))
+            assert s[n, g] == enc
+            sd = oracle.e4m3(enc) if gs == 16 else oracle.e8m0(enc)
+            for j in range(gs):
+                k = g * gs + j
+                c = (q[n, k // 2] >> (4 * (k % 2))) & 15
+                x = float(np.float32(wg[j]) / np.float32(sd))
+                d = np.abs(abs(x) - mags)
+                best = np.flatnonzero(d == d.min())
+                want = best[0] if len(best) == 1 else best[best % 2 == 0][0]
+                assert (c & 7) == want, (n, g, j, x)
+                assert (c >> 3) == (1 if np.signbit(x) else 0)
+
+
+def test_quantize_fp4_zero_group():
+    q, s = oracle.quantize_fp4(np.zeros((2, 64), np.uint16), 32, 1)
+    assert not q.any() and not s.any()
