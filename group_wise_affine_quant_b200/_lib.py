@@ -25,6 +25,7 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "aq_quantize": (_I, [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _P]),
     "aq_dequantize": (_I, [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _P]),
+    "aq_quantize_fp4": (_I, [_P, _P, _P, _I64, _I64, _I, _I, _P]),
     "aq_qmv": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
     "aq_qmm": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
     "aq_qmv_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P]),

@@ -12,7 +12,7 @@ from . import _lib
 from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, AQ_OP_QMM,
                    AQ_OP_QMV, AqError, check, lib)
 
-__all__ = ["aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_qconv2d_nhwc",
+__all__ = ["aq_quantize", "aq_quantize_fp4", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_qconv2d_nhwc",
            "aq_workspace_size", "aq_qmv_noalloc", "aq_last_error", "aq_set_weight_prefetch",
            "aq_get_weight_prefetch", "aq_set_input_prefetch", "aq_get_input_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
 
@@ -100,6 +100,18 @@ def aq_quantize(w, bits=4, group_size=64, out=None):
     check(lib().aq_quantize(_ptr(w), _ptr(w_q), _ptr(s), _ptr(b), N, K, bits, group_size, _dt(w),
                             _stream(w.device)), "aq_quantize")
     return w_q, s, b
+
+
+def aq_quantize_fp4(w, group_size=32, out=None):
+    """w [N, K] fp16/bf16 -> (codes [N, K/2] uint8, scales [N, K/group_size]
+    uint8): E2M1 codes with E8M0 (group 32) or E4M3 (group 16) scales."""
+    N, K = w.shape
+    if out is None:
+        out = (torch.empty((N, K // 2), dtype=torch.uint8, device=w.device),
+               torch.empty((N, K // group_size), dtype=torch.uint8, device=w.device))
+    check(lib().aq_quantize_fp4(_ptr(w), _ptr(out[0]), _ptr(out[1]), N, K, group_size, _dt(w),
+                                _stream(w.device)), "aq_quantize_fp4")
+    return out
 
 
 def aq_dequantize(w_q, scales, biases, K, bits=4, group_size=64, dtype=None, out=None):

@@ -108,6 +108,25 @@ aq_status aq_quantize(const void* w, void* w_q, void* scales, void* biases, int6
                      "aq_quantize launch");
 }
 
+aq_status aq_quantize_fp4(const void* w, void* codes, void* scales, int64_t N, int64_t K,
+                          int group_size, aq_dtype dtype, aq_stream_t stream) {
+  g_err[0] = 0;
+  if (dtype != AQ_F16 && dtype != AQ_BF16)
+    return fail(AQ_ERR_UNSUPPORTED, "dtype %d is not fp16 (0) or bf16 (1)", (int)dtype);
+  if (group_size != 16 && group_size != 32)
+    return fail(AQ_ERR_UNSUPPORTED, "group_size %d: FP4 scales are E8M0 (32) or E4M3 (16)", group_size);
+  if (N < 0 || K < 0 || N > kMaxDim || K > kMaxDim)
+    return fail(AQ_ERR_INVALID_ARG, "N=%lld K=%lld out of range", (long long)N, (long long)K);
+  if (K % 32)
+    return fail(AQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 32", (long long)K);
+  if (N == 0 || K == 0) return AQ_OK;
+  if (!w || !codes || !scales) return fail(AQ_ERR_INVALID_ARG, "w, codes and scales must not be NULL");
+  if (!aligned(w, 2)) return fail(AQ_ERR_MISALIGNED, "w must be 2-byte aligned");
+  return cuda_status(aq::launch_quantize_fp4(w, codes, scales, N, K, group_size, dtype,
+                                             (cudaStream_t)stream),
+                     "aq_quantize_fp4 launch");
+}
+
 aq_status aq_dequantize(const void* w_q, const void* scales, const void* biases, void* w_out,
                         int64_t N, int64_t K, int bits, int group_size, aq_mode mode,
                         aq_dtype dtype, aq_stream_t stream) {

@@ -10,10 +10,21 @@
 // stores with 32-bit writes (a group's packed size, gs*bits/8 bytes, is a
 // multiple of 4 for every supported width).
 //
+// FP4 quantizer (the steps of fp_quantize_dequantize, to_fp8_e8m0 and
+// to_fp4_e2m1 in "mlx 1.0.0, mlx/backend/cpu/quantized.cpp", up to the codes
+// and the scale byte): one element per lane, a warp per 32 elements (one
+// group of 32, or two groups of 16).  Per group, in fp32: absmax (NaN
+// ignored), scale = absmax / 6 (IEEE division), the scale byte (E8M0 for
+// group 32: the nearest power of two on a log scale; E4M3 for group 16: ties
+// to even, saturating), the byte decoded back to float, and each code from
+// the E2M1 threshold table applied to w / decoded scale.
+//
 // Dequantizer: one thread per 8 consecutive elements (8 codes = `bits`
 // bytes), w_hat = fma(s, q, b) in T (a single rounding of the exact value;
 // q is exact in fp16 and bf16 for q <= 256), or LUT[q] * s_T in fp32 (exact)
 // rounded once to T in FP4 mode.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 
 namespace aq {
@@ -84,6 +95,63 @@ quantize_kernel(const T* __restrict__ w, uint8_t* __restrict__ wq, T* __restrict
       biases[grp] = TT<T>::from_f(bias);
     }
     __syncwarp();
+  }
+}
+
+// E8M0 byte of a float: 0xFF for NaN / inf, 0 for x <= 0; otherwise
+// round(log2(x)) taken exactly (x = m * 2^e with m in [1, 2) rounds up to
+// 2^(e+1) when m >= sqrt(2), i.e. m * m >= 2, exact in double), clamped to
+// [-127, 127], plus 127.
+__device__ __forceinline__ unsigned e8m0_byte(float x) {
+  if (!isfinite(x)) return 0xFFu;
+  if (!(x > 0.0f)) return 0u;
+  int e;
+  const double m = 2.0 * frexp((double)x, &e);     // x = m * 2^(e-1)
+  int n = (m * m >= 2.0) ? e : e - 1;
+  n = n < -127 ? -127 : (n > 127 ? 127 : n);
+  return (unsigned)(n + 127);
+}
+
+// E2M1 code of a float (the threshold table: round to nearest, ties to even,
+// saturating at 6; NaN gives 0x7).
+__device__ __forceinline__ unsigned e2m1_code(float x) {
+  if (isnan(x)) return 0x7u;
+  const unsigned sign = signbit(x) ? 0x8u : 0u;
+  const float a = fabsf(x);
+  unsigned b = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+               (a >= 3.5f) + (a > 5.0f);
+  return b | sign;
+}
+
+template <typename T, int GS>
+__global__ void __launch_bounds__(256)
+quantize_fp4_kernel(const T* __restrict__ w, uint8_t* __restrict__ codes,
+                    uint8_t* __restrict__ scales, int64_t N, int64_t K) {
+  const int lane = threadIdx.x & 31;
+  const int64_t chunks = N * (K / 32);                  // 32-element runs of a row
+  const int64_t G = K / GS;
+  for (int64_t ch = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; ch < chunks;
+       ch += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int64_t n = ch / (K / 32), k0 = (ch - n * (K / 32)) * 32;
+    const float v = TT<T>::to_f(w[n * K + k0 + lane]);
+    float amax = isnan(v) ? -INFINITY : fabsf(v);
+#pragma unroll
+    for (int o = GS / 2; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float scale = __fdiv_rn(amax, 6.0f);
+    unsigned byte;
+    float sdec;
+    if (GS == 32) {
+      byte = e8m0_byte(scale);
+      sdec = e8m0_to_float(byte);
+    } else {
+      byte = (unsigned)__nv_cvt_float_to_fp8(scale, __NV_SATFINITE, __NV_E4M3);
+      sdec = e4m3_to_float(byte);
+    }
+    const float el = sdec == 0.0f ? 0.0f : __fdiv_rn(v, sdec);
+    const unsigned c = e2m1_code(el);
+    const unsigned hi = __shfl_down_sync(0xffffffffu, c, 1);
+    if ((lane & 1) == 0) codes[n * (K / 2) + (k0 + lane) / 2] = (uint8_t)(c | (hi << 4));
+    if ((lane & (GS - 1)) == 0) scales[n * G + (k0 + lane) / GS] = (uint8_t)byte;
   }
 }
 
@@ -192,7 +260,28 @@ cudaError_t dequantize_t(const void* w_q, const void* scales, const void* biases
   return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t quantize_fp4_t(const void* w, void* codes, void* scales, int64_t N, int64_t K,
+                           int gs, cudaStream_t st) {
+  const int64_t chunks = N * (K / 32);
+  if (chunks == 0) return cudaSuccess;
+  dim3 grid(grid_for(chunks, 8)), block(256);
+  if (gs == 32)
+    quantize_fp4_kernel<T, 32><<<grid, block, 0, st>>>((const T*)w, (uint8_t*)codes,
+                                                       (uint8_t*)scales, N, K);
+  else
+    quantize_fp4_kernel<T, 16><<<grid, block, 0, st>>>((const T*)w, (uint8_t*)codes,
+                                                       (uint8_t*)scales, N, K);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_fp4(const void* w, void* codes, void* scales, int64_t N, int64_t K,
+                                int gs, int dtype, cudaStream_t st) {
+  return dtype == AQ_F16 ? quantize_fp4_t<__half>(w, codes, scales, N, K, gs, st)
+                         : quantize_fp4_t<__nv_bfloat16>(w, codes, scales, N, K, gs, st);
+}
 
 cudaError_t launch_quantize(const void* w, void* w_q, void* scales, void* biases, int64_t N,
                             int64_t K, int bits, int gs, int dtype, cudaStream_t st) {

@@ -99,6 +99,31 @@ AQ_API aq_status aq_quantize(const void* w, void* w_q, void* scales, void* biase
                       aq_stream_t stream);
 
 /*
+ * aq_quantize_fp4 — FP4 (E2M1) quantizer with per-group scales ("mlx 1.0.0,
+ * mlx/backend/cpu/quantized.cpp": the steps of fp_quantize_dequantize,
+ * to_fp8_e8m0 and to_fp4_e2m1, up to the codes and the scale byte).  It
+ * writes the FP4 weights that aq_qmv / aq_qmm / aq_dequantize take in
+ * AQ_MODE_FP4.  Per group of group_size consecutive elements of a row, in
+ * fp32:
+ *   absmax = max |w| (NaN elements ignored);  scale = absmax / 6
+ *   group_size 32: byte = E8M0 of scale: 0xFF for NaN / inf, else
+ *                  round(log2(scale)) (the exact nearest power of two on a
+ *                  log scale; 0 -> -127), clamped to [-127, 127], + 127
+ *   group_size 16: byte = E4M3FN of scale (ties to even, saturating at 448)
+ *   s = the byte decoded (E8M0: 2^(byte-127), byte 0 -> 2^-127; E4M3FN)
+ *   code = E2M1 of (s == 0 ? 0 : w / s): round to nearest (ties to even),
+ *          saturating at +-6, sign kept (-0 -> code 8), NaN -> code 7.
+ *   w      [N, K] T, row-major;  K a multiple of 32.
+ *   codes  [N, K/2] bytes: code k in the low nibble of byte k/2 for even k,
+ *          the high nibble for odd k.
+ *   scales [N, K/group_size] bytes.
+ * Bit-exact with the definition above.  Returns AQ_ERR_UNSUPPORTED for
+ * group_size other than 16 / 32 or a dtype other than fp16 / bf16.
+ */
+AQ_API aq_status aq_quantize_fp4(const void* w, void* codes, void* scales, int64_t N, int64_t K,
+                                 int group_size, aq_dtype dtype, aq_stream_t stream);
+
+/*
  * aq_dequantize — writes w_out [N, K] T with every element rounded once
  * (to nearest, ties to even) from the exact value s*q + b (affine) or
  * LUT[q] * s_T (FP4).  Same weight arguments as aq_qmm.

@@ -166,3 +166,13 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         _lib.lib()
+
+
+def test_quantize_fp4_validation():
+    q = L().aq_quantize_fp4
+    assert q(A, A, A, 4, 64, 64, 1, None) == UNSUPPORTED        # scales are for 16 or 32
+    assert q(A, A, A, 4, 64, 32, 2, None) == UNSUPPORTED        # fp16 / bf16 only
+    assert q(A, A, A, 4, 48, 16, 1, None) == INVALID            # K a multiple of 32
+    assert q(A + 1, A, A, 4, 64, 32, 1, None) == MISALIGNED
+    assert q(None, A, A, 4, 64, 32, 1, None) == INVALID
+    assert q(None, None, None, 0, 64, 32, 1, None) == OK        # empty: nothing to do
