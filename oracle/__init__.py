@@ -44,6 +44,8 @@ def lib():
             getattr(_lib, name).restype = I
         _lib.orc_quantize_fp4.argtypes = [P, I64, I64, I, I, P, P]
         _lib.orc_quantize_fp4.restype = I
+        _lib.orc_quantize_dequantize_fp.argtypes = [P, I64, I64, I, I, I, P]
+        _lib.orc_quantize_dequantize_fp.restype = I
         _lib.orc_quantize.argtypes = [P, I64, I64, I, I, I, P, P, P]
         _lib.orc_unpack.argtypes = [P, I64, I64, I, P]
         _lib.orc_dequantize.argtypes = [P, P, P, I64, I64, I, I, I, I, P, P]
@@ -139,6 +141,25 @@ def quantize_fp4(w16, gs, dt):
     scales = np.zeros((N, K // gs), np.uint8)
     _check(lib().orc_quantize_fp4(_p(w16), N, K, gs, dt, _p(codes), _p(scales)), "quantize_fp4")
     return codes, scales
+
+
+def quantize_dequantize_fp(w16, bits, gs, dt):
+    """[P4] fp_quantize_dequantize: w16 [N, K] uint16 T patterns -> the fake-
+    quantized [N, K] T patterns (E2M1 elements for bits 4, E4M3 for bits 8;
+    E8M0 scales for gs = 32, E4M3 for gs = 16)."""
+    w16 = _c(w16, np.uint16)
+    N, K = w16.shape
+    out = np.zeros((N, K), np.uint16)
+    _check(lib().orc_quantize_dequantize_fp(_p(w16), N, K, bits, gs, dt, _p(out)),
+           "quantize_dequantize_fp")
+    return out
+
+
+def qqmm(x16, wq, scales, N, gs, dt, w_in_t=False):
+    """[P4] QQMatmul: x fake-quantized to FP4 (quantize_dequantize_fp, bits 4)
+    times the FP4 weights' transpose -> (y [M, N], den [M, N]) as qmm."""
+    xh = quantize_dequantize_fp(x16, 4, gs, dt)
+    return qmm(xh, wq, scales, None, N, 4, gs, FP4, dt, w_in_t=w_in_t)
 
 
 def unpack(wq, N, K, bits):

@@ -21,7 +21,8 @@
 //        (fp32 arithmetic, packing), get_pack_factor / get_bytes_per_pack,
 //        extract_bits, FP4_LUT, dequantize_scale (E8M0 / FP8 scales), fp_qmm_t,
 //        and the FP4 quantizer's steps: to_fp8_e8m0, to_fp4_e2m1 and
-//        fp_quantize_dequantize (scale = absmax / 6).
+//        fp_quantize_dequantize (scale = absmax / 6, or / 448 for 8-bit
+//        elements), which QQMatmul applies to x before the FP4 matmul.
 //
 // Precision.  The quantizer runs in fp32, in the order the quantize routine of
 // [P4] takes its steps, because its codes, scales and biases are fixed by fp32
@@ -358,6 +359,44 @@ int orc_quantize_fp4(const uint16_t* w, int64_t N, int64_t K, int gs, int dt, ui
         uint8_t& dst = codes[n * (K / 2) + k / 2];
         if (k % 2 == 0) dst = (uint8_t)((dst & 0xF0) | c);
         else dst = (uint8_t)((dst & 0x0F) | (c << 4));
+      }
+    }
+  }
+  return 0;
+}
+
+// Fake quantization of activations, the other use of [P4]
+// fp_quantize_dequantize (QQMatmul quantizes x with it before the FP4
+// matmul).  w is [N, K] T; out is [N, K] T.  Per group, in fp32:
+//   absmax = max_j |w_j|  (NaN ignored, as above)
+//   scale  = absmax / (bits == 4 ? 6 : 448)
+//   s      = the scale byte decoded to float (E4M3 for gs = 16, E8M0 for 32)
+//   e_j    = s == 0 ? 0 : w_j / s
+//   v_j    = bits == 4 ? the E2M1 table value of to_fp4_e2m1(e_j)
+//                      : the E4M3 value of ToFP8(e_j)  (FromFP8 o ToFP8)
+//   out_j  = T(s * v_j)   (one fp32 multiplication, then the cast to T)
+int orc_quantize_dequantize_fp(const uint16_t* w, int64_t N, int64_t K, int bits, int gs, int dt,
+                               uint16_t* out) {
+  if (dt != DT_F16 && dt != DT_BF16) return 1;
+  if ((bits != 4 && bits != 8) || (gs != 16 && gs != 32) || N < 0 || K < 0 || K % gs) return 1;
+  const float div = bits == 4 ? 6.0f : 448.0f;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < K / gs; ++g) {
+      const uint16_t* wg = w + n * K + g * gs;
+      float amax = -std::numeric_limits<float>::infinity();
+      for (int j = 0; j < gs; ++j) {
+        const float a = std::fabs(t_to_float(wg[j], dt));
+        amax = (amax < a) ? a : amax;
+      }
+      const float scale = amax / div;
+      const float sdec = (float)(gs == 16 ? e4m3_value(e4m3_encode(scale))
+                                          : e8m0_value(e8m0_encode(scale)));
+      for (int j = 0; j < gs; ++j) {
+        const float el = sdec == 0.0f ? 0.0f : t_to_float(wg[j], dt) / sdec;
+        const float v = (float)(bits == 4 ? e2m1_value(e2m1_encode(el))
+                                          : e4m3_value(e4m3_encode(el)));
+        const float prod = sdec * v;
+        out[n * K + g * gs + j] = round_to_t((double)prod, dt);
       }
     }
   }

@@ -624,3 +624,73 @@ def test_quantize_fp4_is_nearest_on_the_scaled_table(gs):
 def test_quantize_fp4_zero_group():
     q, s = oracle.quantize_fp4(np.zeros((2, 64), np.uint16), 32, 1)
     assert not q.any() and not s.any()
+
+
+# ------------------------------------------- activation fake quantization (QQMatmul)
+
+@pytest.mark.parametrize("dt", [0, 1])
+@pytest.mark.parametrize("gs", [16, 32])
+def test_fake_quant_fp4_is_the_dequantized_fp4_codes(dt, gs):
+    """bits 4: fp_quantize_dequantize's output is the FP4 quantizer's codes
+    times the decoded scale (both pinned above), cast once to T."""
+    rng = np.random.default_rng(dt * 7 + gs)
+    N, K = 6, 8 * gs
+    w = rng.standard_normal((N, K)) * np.exp(rng.standard_normal((N, 1)))
+    w16 = f64_to_u16(w, dt)
+    xh = oracle.quantize_dequantize_fp(w16, 4, gs, dt)
+    q, s = oracle.quantize_fp4(w16, gs, dt)
+    _, wt = oracle.dequantize(q, s, None, N, K, 4, gs, FP4, dt)
+    assert np.array_equal(xh, wt)
+
+
+@pytest.mark.parametrize("gs", [16, 32])
+def test_fake_quant_fp8_elements_match_torch_float8(gs):
+    """bits 8: each element is s * E4M3(w / s).  Groups whose absmax is
+    448 * 2^k have s = 2^k exactly in both scale formats, so w / s is exact
+    and torch's float8_e4m3fn conversion (round to nearest even) gives the
+    element."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(gs)
+    rows = []
+    for k in (-3, 0, 2):
+        for _ in range(2):
+            v = rng.uniform(-1.0, 1.0, gs) * 448.0
+            v[rng.integers(0, gs)] = 448.0 * (1 if rng.integers(0, 2) else -1)
+            rows.append(v * 2.0 ** k)
+    w16 = f64_to_u16(np.array(rows), BF16)
+    out = oracle.quantize_dequantize_fp(w16, 8, gs, BF16)
+    w = u16_to_f64(w16, BF16)
+    for i, k in enumerate([k for k in (-3, 0, 2) for _ in range(2)]):
+        e = torch.from_numpy((w[i] / 2.0 ** k).astype(np.float32))
+        v = e.to(torch.float8_e4m3fn).to(torch.float64).numpy() * 2.0 ** k
+        assert np.array_equal(u16_to_f64(out[i], BF16), v), i
+
+
+def test_fake_quant_special_groups():
+    """A zero group stays zero; a NaN element is ignored by absmax and comes
+    out as the code-7 value 6 s for E2M1 (the page's NaN rule) and NaN for
+    E4M3."""
+    z = oracle.quantize_dequantize_fp(np.zeros((1, 32), np.uint16), 4, 32, BF16)
+    assert not z.any()
+    w = np.ones((1, 32)) * 3.0
+    w16 = f64_to_u16(w, BF16)
+    w16[0, 5] = 0x7FC0                                     # bf16 NaN
+    out4 = u16_to_f64(oracle.quantize_dequantize_fp(w16, 4, 32, BF16), BF16)[0]
+    # absmax 3 -> scale 0.5 -> E8M0 2^-1; 3 / 0.5 = 6 -> 6 * 0.5 = 3
+    assert out4[5] == 3.0 and np.all(np.delete(out4, 5) == 3.0)
+    out8 = u16_to_f64(oracle.quantize_dequantize_fp(w16, 8, 32, BF16), BF16)[0]
+    assert np.isnan(out8[5]) and np.all(np.delete(out8, 5) == 3.0)
+
+
+def test_qqmm_is_qmm_over_fake_quantized_x():
+    rng = np.random.default_rng(5)
+    M, N, K, gs = 2, 8, 128, 32
+    codes = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    wq = np_pack(codes, 4)
+    sc = rng.integers(120, 134, size=(N, K // gs)).astype(np.uint8)
+    x16 = f64_to_u16(rng.standard_normal((M, K)), BF16)
+    y, _ = oracle.qqmm(x16, wq, sc, N, gs, BF16)
+    xh = u16_to_f64(oracle.quantize_dequantize_fp(x16, 4, gs, BF16), BF16)
+    lut = np.array([float(v) for _, v in _golden_rows("fp4_e2m1_lut.txt")])
+    W = lut[codes] * np.repeat(np.ldexp(1.0, sc.astype(np.int64) - 127), gs, axis=1)
+    assert np.allclose(y, xh @ W.T, rtol=1e-12, atol=0)
