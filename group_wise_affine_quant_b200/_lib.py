@@ -15,7 +15,7 @@ STATUS_NAMES = {0: "AQ_OK", 1: "AQ_ERR_INVALID_ARG", 2: "AQ_ERR_UNSUPPORTED",
                 3: "AQ_ERR_MISALIGNED", 4: "AQ_ERR_CUDA", 5: "AQ_ERR_WORKSPACE"}
 AQ_F16, AQ_BF16 = 0, 1
 AQ_MODE_AFFINE, AQ_MODE_FP4 = 0, 1
-AQ_OP_QMV, AQ_OP_QMM, AQ_OP_QCONV2D = 0, 1, 2
+AQ_OP_QMV, AQ_OP_QMM, AQ_OP_QCONV2D, AQ_OP_QQMM = 0, 1, 2, 3
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -26,6 +26,8 @@ SIGNATURES = {
     "aq_quantize": (_I, [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _P]),
     "aq_dequantize": (_I, [_P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _P]),
     "aq_quantize_fp4": (_I, [_P, _P, _P, _I64, _I64, _I, _I, _P]),
+    "aq_quantize_dequantize_fp": (_I, [_P, _P, _I64, _I64, _I, _I, _I, _P]),
+    "aq_qqmm": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _SZ, _P]),
     "aq_qmv": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
     "aq_qmm": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
     "aq_qmv_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P]),
@@ -41,6 +43,7 @@ SIGNATURES = {
     "aq_testing_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "aq_testing_set_start_delay_ns": (None, [ctypes.c_uint64]),
     "aq_testing_clear_device_errors": (_I, []),
+    "aq_testing_set_qmv_kernel": (None, [_I]),
 }
 
 

@@ -10,9 +10,9 @@ import torch
 
 from . import _lib
 from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, AQ_OP_QMM,
-                   AQ_OP_QMV, AqError, check, lib)
+                   AQ_OP_QMV, AQ_OP_QQMM, AqError, check, lib)
 
-__all__ = ["aq_quantize", "aq_quantize_fp4", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_qconv2d_nhwc",
+__all__ = ["aq_quantize", "aq_quantize_fp4", "aq_quantize_dequantize_fp", "aq_qqmm", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_qconv2d_nhwc",
            "aq_workspace_size", "aq_qmv_noalloc", "aq_last_error", "aq_set_weight_prefetch",
            "aq_get_weight_prefetch", "aq_set_input_prefetch", "aq_get_input_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
 
@@ -111,6 +111,31 @@ def aq_quantize_fp4(w, group_size=32, out=None):
                torch.empty((N, K // group_size), dtype=torch.uint8, device=w.device))
     check(lib().aq_quantize_fp4(_ptr(w), _ptr(out[0]), _ptr(out[1]), N, K, group_size, _dt(w),
                                 _stream(w.device)), "aq_quantize_fp4")
+    return out
+
+
+def aq_quantize_dequantize_fp(x, bits=4, group_size=32, out=None):
+    """Fake quantization of x [N, K] fp16/bf16: E2M1 (bits 4) or E4M3 (bits 8)
+    elements under E8M0 (group 32) or E4M3 (group 16) scales, back in T."""
+    N, K = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    check(lib().aq_quantize_dequantize_fp(_ptr(x), _ptr(out), N, K, bits, group_size, _dt(x),
+                                          _stream(x.device)), "aq_quantize_dequantize_fp")
+    return out
+
+
+def aq_qqmm(x, w_q, scales, group_size=32, out=None, workspace=None):
+    """W4A4: y = fq(x) . dequant(w)^T with FP4 weights and x fake-quantized to
+    the weights' FP4 format."""
+    M, K = x.shape
+    N = w_q.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    ws_bytes = aq_workspace_size(AQ_OP_QQMM, M, N, K, 4, group_size, AQ_MODE_FP4)
+    ws = (workspace or _default_ws).get(x.device, ws_bytes)
+    check(lib().aq_qqmm(_ptr(x), _ptr(w_q), _ptr(scales), _ptr(out), M, N, K, group_size, _dt(x),
+                        _ptr(ws), 0 if ws is None else ws.numel(), _stream(x.device)), "aq_qqmm")
     return out
 
 

@@ -5,6 +5,7 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <atomic>
 #include <vector>
 
 #include "common.cuh"
@@ -169,6 +170,9 @@ static aq_status zero_output(void* y, int64_t M, int64_t N, aq_stream_t stream) 
                      "zero-fill of y");
 }
 
+// Kernel choice of aq_qmv forced by a test (0: automatic).
+static std::atomic<int> g_qmv_kernel{0};
+
 aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void* biases,
                  void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
                  aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
@@ -185,14 +189,29 @@ aq_status aq_qmv(const void* x, const void* w_q, const void* scales, const void*
   // are 16-byte multiples (TMA) run the tcgen05 decode kernel; the rest run
   // the fp32 CUDA-core kernel.  All keep w_hat in fp32 (scale and bias per
   // group).
-  if (aq::qmv_mma_applies(M, N, K, bits, group_size, mode, scales, biases)) {
+  // A single small problem (M = 1 up to 2^24 weights, M <= 2 up to 2^22,
+  // M <= 4 up to 2^20) runs the fp32 kernel: it has fewer serial phases per
+  // call than the warp-MMA kernel's TMA / prep / MMA pipeline, and a lone call
+  // of that size is bound by those phases, not by the weight stream.  Measured
+  // on B200 in chains of dependent calls: at M = 1, 4.1 against 7.5 us for
+  // 512 x 2048 and 10.8 against 14.1 us for 2048 x 8192; at M = 2, 8.3
+  // against 9.3 us for 2048 x 2048; from 8192 x 8192 (M = 1), 8192 x 2048
+  // (M = 2) and 2048 x 2048 (M = 4) on the warp-MMA kernel is faster.
+  const int force = g_qmv_kernel.load(std::memory_order_relaxed);
+  const int64_t nk = N * K;
+  const bool lone_small = (M == 1 && nk <= ((int64_t)1 << 24)) ||
+                          (M <= 2 && nk <= ((int64_t)1 << 22)) ||
+                          (M <= 4 && nk <= ((int64_t)1 << 20));
+  if (force != 2 && force != 3 && (force == 1 || !lone_small) &&
+      aq::qmv_mma_applies(M, N, K, bits, group_size, mode, scales, biases)) {
     const size_t need = aq::qmv_mma_workspace(M, N, K, group_size);
     if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
     return cuda_status(aq::launch_qmv_mma(x, w_q, scales, biases, y, M, N, K, group_size, dtype,
                                           workspace, (cudaStream_t)stream),
                        "aq_qmv launch");
   }
-  if (aq::qmv_tc_applies(M, N, K, bits, group_size, mode, scales, biases)) {
+  if (force != 3 && !(force == 0 && lone_small && mode == AQ_MODE_AFFINE && bits == 4) &&
+      aq::qmv_tc_applies(M, N, K, bits, group_size, mode, scales, biases)) {
     const size_t need = aq::qmv_tc_workspace(M, N, K, bits, group_size);
     if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
     return cuda_status(aq::launch_qmv_tc(x, w_q, scales, biases, y, M, N, K, bits, group_size,
@@ -330,8 +349,68 @@ aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void*
                      "aq_qmm launch");
 }
 
+aq_status aq_quantize_dequantize_fp(const void* x, void* out, int64_t N, int64_t K, int bits,
+                                    int group_size, aq_dtype dtype, aq_stream_t stream) {
+  g_err[0] = 0;
+  if (dtype != AQ_F16 && dtype != AQ_BF16)
+    return fail(AQ_ERR_UNSUPPORTED, "dtype %d is not fp16 (0) or bf16 (1)", (int)dtype);
+  if (bits != 4 && bits != 8)
+    return fail(AQ_ERR_UNSUPPORTED, "bits %d: elements are E2M1 (4) or E4M3 (8)", bits);
+  if (group_size != 16 && group_size != 32)
+    return fail(AQ_ERR_UNSUPPORTED, "group_size %d: scales are E8M0 (32) or E4M3 (16)", group_size);
+  if (N < 0 || K < 0 || N > kMaxDim || K > kMaxDim)
+    return fail(AQ_ERR_INVALID_ARG, "N=%lld K=%lld out of range", (long long)N, (long long)K);
+  if (K % 32) return fail(AQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 32", (long long)K);
+  if (N == 0 || K == 0) return AQ_OK;
+  if (!x || !out) return fail(AQ_ERR_INVALID_ARG, "x and out must not be NULL");
+  if (!aligned(x, 2) || !aligned(out, 2)) return fail(AQ_ERR_MISALIGNED, "x and out must be 2-byte aligned");
+  return cuda_status(aq::launch_quantize_dequantize_fp(x, out, N, K, bits, group_size, dtype,
+                                                       (cudaStream_t)stream),
+                     "aq_quantize_dequantize_fp launch");
+}
+
+// Workspace of aq_qqmm: the matmul's own first, then the fake-quantized x,
+// never inside the first 64 KB (the counters that every call leaves zero, so
+// that the buffer still serves the other calls).
+static size_t qqmm_mm_bytes(int64_t M, int64_t N, int64_t K, int group_size) {
+  const size_t b = M <= 16 ? aq_workspace_size(AQ_OP_QMV, M, N, K, 4, group_size, AQ_MODE_FP4, 1) : 0;
+  return std::max((size_t)65536, (b + 255) & ~(size_t)255);
+}
+
+aq_status aq_qqmm(const void* x, const void* w_q, const void* scales, void* y, int64_t M,
+                  int64_t N, int64_t K, int group_size, aq_dtype dtype, void* workspace,
+                  size_t workspace_bytes, aq_stream_t stream) {
+  g_err[0] = 0;
+  aq_status st = check_weight(w_q, scales, nullptr, N, K, 4, group_size, AQ_MODE_FP4, dtype);
+  if (st != AQ_OK) return st;
+  if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
+  if (M == 0 || N == 0) return AQ_OK;
+  if (K == 0) return zero_output(y, M, N, stream);
+  if (K % 32) return fail(AQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 32", (long long)K);
+  const size_t need = aq_workspace_size(AQ_OP_QQMM, M, N, K, 4, group_size, AQ_MODE_FP4, 1);
+  if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
+  const size_t mb = qqmm_mm_bytes(M, N, K, group_size);
+  void* xq = static_cast<uint8_t*>(workspace) + mb;
+  if ((st = aq_quantize_dequantize_fp(x, xq, M, K, 4, group_size, dtype, stream)) != AQ_OK)
+    return st;
+  // The matmul reads the fake-quantized x that the launch above writes, so
+  // it must not read x before its dependency wait: input prefetch is off for
+  // this thread's inner call.
+  const int input_prefetch = g_input_prefetch;
+  g_input_prefetch = 0;
+  if (M <= 16)
+    st = aq_qmv(xq, w_q, scales, nullptr, y, M, N, K, 4, group_size, AQ_MODE_FP4, dtype,
+                workspace, mb, stream);
+  else
+    st = aq_qmm(xq, w_q, scales, nullptr, y, M, N, K, 4, group_size, AQ_MODE_FP4, dtype,
+                nullptr, 0, stream);
+  g_input_prefetch = input_prefetch;
+  return st;
+}
+
 void aq_testing_set_wait_limit_ns(uint64_t ns) { aq::testing_set_mv_wait_ns(ns); }
 void aq_testing_set_start_delay_ns(uint64_t ns) { aq::testing_set_mv_delay_ns(ns); }
+void aq_testing_set_qmv_kernel(int which) { g_qmv_kernel.store(which, std::memory_order_relaxed); }
 aq_status aq_testing_clear_device_errors(void) {
   g_err[0] = 0;
   cudaError_t e = cudaDeviceSynchronize();
@@ -399,9 +478,10 @@ size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, in
     if (aq::qmv_mma_shape_ok(N, K, bits, group_size, mode))
       need = aq::qmv_mma_workspace(M, N, K, group_size);
     if (aq::qmv_tc_shape_ok(N, K, bits, group_size, mode))
-      return std::max(need, aq::qmv_tc_workspace(M, N, K, bits, group_size));
+      need = std::max(need, aq::qmv_tc_workspace(M, N, K, bits, group_size));
     return std::max(need, aq::plan_qmv(M, N, K, bits, group_size, mode).ws_bytes);
   }
+  if (op == AQ_OP_QQMM) return qqmm_mm_bytes(M, N, K, group_size) + (size_t)(M * K) * 2;
   return 0;
 }
 

@@ -19,6 +19,12 @@
 // to even, saturating), the byte decoded back to float, and each code from
 // the E2M1 threshold table applied to w / decoded scale.
 //
+// Fake quantization of activations (the same page's fp_quantize_dequantize,
+// which QQMatmul applies to x): the FP4 quantizer's group steps with the
+// scale divided by 6 (E2M1 elements) or 448 (E4M3 elements), each element
+// replaced by T(s * v) with v the element's E2M1 / E4M3 value and s the
+// decoded scale (one fp32 multiplication, one rounding to T).
+//
 // Dequantizer: one thread per 8 consecutive elements (8 codes = `bits`
 // bytes), w_hat = fma(s, q, b) in T (a single rounding of the exact value;
 // q is exact in fp16 and bf16 for q <= 256), or LUT[q] * s_T in fp32 (exact)
@@ -155,6 +161,30 @@ quantize_fp4_kernel(const T* __restrict__ w, uint8_t* __restrict__ codes,
   }
 }
 
+template <typename T, int GS, int BITS>
+__global__ void __launch_bounds__(256)
+quantize_dequantize_fp_kernel(const T* __restrict__ w, T* __restrict__ out, int64_t N, int64_t K) {
+  const int lane = threadIdx.x & 31;
+  const int64_t chunks = N * (K / 32);
+  for (int64_t ch = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; ch < chunks;
+       ch += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int64_t e = ch * 32 + lane;                   // rows are whole 32-element runs
+    const float v = TT<T>::to_f(w[e]);
+    float amax = isnan(v) ? -INFINITY : fabsf(v);
+#pragma unroll
+    for (int o = GS / 2; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float scale = __fdiv_rn(amax, BITS == 4 ? 6.0f : 448.0f);
+    const float sdec =
+        GS == 32 ? e8m0_to_float(e8m0_byte(scale))
+                 : e4m3_to_float((unsigned)__nv_cvt_float_to_fp8(scale, __NV_SATFINITE, __NV_E4M3));
+    const float el = sdec == 0.0f ? 0.0f : __fdiv_rn(v, sdec);
+    const float q = BITS == 4
+                        ? e2m1_to_float(e2m1_code(el))
+                        : e4m3_to_float((unsigned)__nv_cvt_float_to_fp8(el, __NV_SATFINITE, __NV_E4M3));
+    out[e] = TT<T>::from_f(__fmul_rn(sdec, q));
+  }
+}
+
 template <typename T, int BITS>
 __global__ void __launch_bounds__(256)
 dequantize_affine_kernel(const uint8_t* __restrict__ wq, const T* __restrict__ scales,
@@ -275,7 +305,28 @@ cudaError_t quantize_fp4_t(const void* w, void* codes, void* scales, int64_t N, 
   return cudaGetLastError();
 }
 
+template <typename T, int BITS>
+cudaError_t qdq_fp_t(const void* w, void* out, int64_t N, int64_t K, int gs, cudaStream_t st) {
+  const int64_t chunks = N * (K / 32);
+  if (chunks == 0) return cudaSuccess;
+  dim3 grid(grid_for(chunks, 8)), block(256);
+  if (gs == 32)
+    quantize_dequantize_fp_kernel<T, 32, BITS><<<grid, block, 0, st>>>((const T*)w, (T*)out, N, K);
+  else
+    quantize_dequantize_fp_kernel<T, 16, BITS><<<grid, block, 0, st>>>((const T*)w, (T*)out, N, K);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_dequantize_fp(const void* w, void* out, int64_t N, int64_t K, int bits,
+                                          int gs, int dtype, cudaStream_t st) {
+  if (dtype == AQ_F16)
+    return bits == 4 ? qdq_fp_t<__half, 4>(w, out, N, K, gs, st)
+                     : qdq_fp_t<__half, 8>(w, out, N, K, gs, st);
+  return bits == 4 ? qdq_fp_t<__nv_bfloat16, 4>(w, out, N, K, gs, st)
+                   : qdq_fp_t<__nv_bfloat16, 8>(w, out, N, K, gs, st);
+}
 
 cudaError_t launch_quantize_fp4(const void* w, void* codes, void* scales, int64_t N, int64_t K,
                                 int gs, int dtype, cudaStream_t st) {

@@ -76,7 +76,7 @@ typedef enum {
   AQ_MODE_FP4 = 1           /* bits = 4; group_size 32 (E8M0) or 16 (E4M3); biases NULL */
 } aq_mode;
 
-typedef enum { AQ_OP_QMV = 0, AQ_OP_QMM = 1, AQ_OP_QCONV2D = 2 } aq_op;
+typedef enum { AQ_OP_QMV = 0, AQ_OP_QMM = 1, AQ_OP_QCONV2D = 2, AQ_OP_QQMM = 3 } aq_op;
 
 /*
  * aq_quantize — affine group quantizer ("mlx 1.0.0, .../quantized.cpp",
@@ -260,9 +260,51 @@ AQ_API aq_status aq_qconv2d_nhwc(const void* x, const void* w_q, const void* sca
                           void* workspace, size_t workspace_bytes, aq_stream_t stream);
 
 /*
+ * aq_quantize_dequantize_fp — fake quantization of activations ("mlx 1.0.0,
+ * mlx/backend/cpu/quantized.cpp", fp_quantize_dequantize: the step that
+ * QQMatmul applies to x).  Per group of group_size consecutive elements of a
+ * row, in fp32:
+ *   scale = absmax / (bits == 4 ? 6 : 448)   (NaN elements ignored)
+ *   s     = scale through its byte and back: E8M0 for group_size 32, E4M3FN
+ *           for 16 (the same encodings as aq_quantize_fp4)
+ *   e     = s == 0 ? 0 : x / s
+ *   out   = T(s * v), v = the E2M1 value of e (bits 4; NaN -> 6) or its
+ *           E4M3FN value (bits 8; ties to even, saturating at 448, NaN stays
+ *           NaN); one fp32 multiplication, one rounding to T.
+ *   x, out [N, K] T row-major (out may equal x); K a multiple of 32.
+ * Bit-exact with the definition.  AQ_ERR_UNSUPPORTED for bits other than
+ * 4 / 8, group_size other than 16 / 32, or a dtype other than fp16 / bf16.
+ */
+AQ_API aq_status aq_quantize_dequantize_fp(const void* x, void* out, int64_t N, int64_t K,
+                                           int bits, int group_size, aq_dtype dtype,
+                                           aq_stream_t stream);
+
+/*
+ * aq_qqmm — W4A4 matmul, y = fq(x) . w_hat^T ("mlx 1.0.0,
+ * mlx/backend/cpu/quantized.cpp", QQMatmul::eval_cpu: x fake-quantized with
+ * the weights' FP4 format, then the FP4 matmul; the page runs it for one row
+ * of x, this call for any M).  fq is aq_quantize_dequantize_fp with bits 4 and
+ * the weights' group_size; w_q / scales are FP4 weights as aq_qmv / aq_qmm
+ * take them (aq_quantize_fp4 writes them).  x [M, K] T, y [M, N] T, K a
+ * multiple of 32.  Two launches on `stream`: the fake quantization into the
+ * workspace, then aq_qmv (M <= 16) or aq_qmm.  The matmul tolerance is
+ * aq_qmv's / aq_qmm's over fq(x).
+ * Workspace: aq_workspace_size(AQ_OP_QQMM, M, N, K, 4, group_size,
+ * AQ_MODE_FP4, 1) bytes, 256-byte aligned, under aq_qmv's rules (zero-filled
+ * before its first use): aq_qmv's workspace first (M <= 16), then fq(x),
+ * which never starts inside the first 64 KB (the counters that every call
+ * leaves zero).  So one buffer serves aq_qmv and aq_qqmm calls on one
+ * stream.
+ */
+AQ_API aq_status aq_qqmm(const void* x, const void* w_q, const void* scales, void* y, int64_t M,
+                         int64_t N, int64_t K, int group_size, aq_dtype dtype, void* workspace,
+                         size_t workspace_bytes, aq_stream_t stream);
+
+/*
  * aq_workspace_size — bytes of workspace the given call needs (0 if none).
  * For AQ_OP_QCONV2D pass M = B*Ho*Wo, N = Cout / groups, K = Kp and the
- * number of conv groups in `groups`; for the others pass groups = 1.
+ * number of conv groups in `groups`; for the others pass groups = 1 (and for
+ * AQ_OP_QQMM bits = 4, mode = AQ_MODE_FP4).
  */
 AQ_API size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, int group_size,
                          aq_mode mode, int groups);

@@ -9,8 +9,9 @@
  * the other roles run out.  The pages have no counterpart.
  *
  * Scope: the warp-MMA decode kernel behind aq_qmv / aq_qmv_batched /
- * aq_qmv_noalloc (4-bit affine weights).  The settings are process-wide and
- * apply to launches made after the call; 0 restores the default.
+ * aq_qmv_noalloc (4-bit affine weights), and aq_qmv's kernel choice.  The
+ * settings are process-wide and apply to launches made after the call; 0
+ * restores the default.
  */
 #ifndef AQ_TESTING_H
 #define AQ_TESTING_H
@@ -27,6 +28,14 @@ AQ_API void aq_testing_set_wait_limit_ns(uint64_t ns);
 /* Delay, in ns, before the decode kernel's TMA warp issues its first copy
  * (default 0).  The delay ends early once another role has given up. */
 AQ_API void aq_testing_set_start_delay_ns(uint64_t ns);
+
+/* Kernel that later aq_qmv calls of this process use where it applies:
+ * 0 the automatic choice (default), 1 the warp-MMA decode kernel, 2 the
+ * tcgen05 decode kernel, 3 the fp32 CUDA-core kernel (any other value:
+ * automatic).  Lets a test run each
+ * kernel on the same shapes; the workspace that aq_workspace_size reports
+ * covers every kernel. */
+AQ_API void aq_testing_set_qmv_kernel(int which);
 
 /* Clears the device error bits that aq_device_errors() reports.  Synchronises
  * the current device first. */

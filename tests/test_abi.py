@@ -176,3 +176,33 @@ def test_quantize_fp4_validation():
     assert q(A + 1, A, A, 4, 64, 32, 1, None) == MISALIGNED
     assert q(None, A, A, 4, 64, 32, 1, None) == INVALID
     assert q(None, None, None, 0, 64, 32, 1, None) == OK        # empty: nothing to do
+
+
+def test_quantize_dequantize_fp_validation():
+    f = L().aq_quantize_dequantize_fp
+    assert f(A, A, 4, 64, 6, 32, 1, None) == UNSUPPORTED         # bits 4 or 8
+    assert f(A, A, 4, 64, 4, 64, 1, None) == UNSUPPORTED         # group 16 or 32
+    assert f(A, A, 4, 64, 8, 16, 2, None) == UNSUPPORTED
+    assert f(A, A, 4, 40, 4, 16, 1, None) == INVALID
+    assert f(A, A + 1, 4, 64, 4, 32, 1, None) == MISALIGNED
+    assert f(None, None, 0, 64, 4, 32, 1, None) == OK
+
+
+def test_qqmm_validation_and_workspace():
+    q = L().aq_qqmm
+    need = L().aq_workspace_size(3, 4, 256, 1024, 4, 32, 1, 1)
+    assert need >= 4 * 1024 * 2 and need % 2 == 0
+    # the qmv workspace comes first, 256-byte aligned, then x, never inside
+    # the first 64 KB (the counters every call leaves zero)
+    qmv = L().aq_workspace_size(0, 4, 256, 1024, 4, 32, 1, 1)
+    assert need == max(65536, ((qmv + 255) // 256) * 256) + 4 * 1024 * 2
+    big = L().aq_workspace_size(0, 16, 4096, 65536, 4, 32, 1, 1)
+    assert big > 65536
+    assert (L().aq_workspace_size(3, 16, 4096, 65536, 4, 32, 1, 1) ==
+            ((big + 255) // 256) * 256 + 16 * 65536 * 2)
+    assert L().aq_workspace_size(3, 64, 256, 1024, 4, 32, 1, 1) == 65536 + 64 * 1024 * 2
+    assert q(A, A, A, A, 4, 256, 1024, 64, 1, A, 1 << 30, None) == UNSUPPORTED  # FP4 group
+    assert q(A, A, A, A, 4, 256, 1024, 32, 1, None, 0, None) == WORKSPACE
+    assert q(A, A, A, A, 4, 256, 1024, 32, 1, A + 16, 1 << 30, None) == MISALIGNED
+    assert q(A + 2, A, A, A, 4, 256, 1024, 32, 1, A, 1 << 30, None) == MISALIGNED
+    assert q(A, A, A, A, 0, 256, 1024, 32, 1, None, 0, None) == OK             # M = 0

@@ -32,6 +32,7 @@ def test_wait_runs_out_then_next_call_is_correct(M, N, K):
     assert lib().aq_device_errors() == 0
     ws = api.Workspace()
     try:
+        lib().aq_testing_set_qmv_kernel(1)                    # the warp-MMA kernel
         lib().aq_testing_set_wait_limit_ns(2_000_000)         # 2 ms
         lib().aq_testing_set_start_delay_ns(50_000_000)       # 50 ms
         api.aq_qmv(x, wq, s, b, 4, 64, workspace=ws)          # the launch itself succeeds
@@ -39,6 +40,7 @@ def test_wait_runs_out_then_next_call_is_correct(M, N, K):
     finally:
         lib().aq_testing_set_wait_limit_ns(0)
         lib().aq_testing_set_start_delay_ns(0)
+        lib().aq_testing_set_qmv_kernel(0)
     assert lib().aq_device_errors() & 1, "the bounded waits did not report running out"
     assert lib().aq_testing_clear_device_errors() == AQ_OK
     assert lib().aq_device_errors() == 0

@@ -35,7 +35,11 @@ def test_noalloc_matches_qmv_twice(M, N, K, gs):
     w = inputs.normal((N, K), 0.02, 1, g)
     x = to_dev(inputs.normal((M, K), 1.0, 1, g))
     wq, s, b = api.aq_quantize(to_dev(w), 4, gs)
-    y_ref_gpu = api.aq_qmv(x, wq, s, b, 4, gs)
+    lib().aq_testing_set_qmv_kernel(1)            # aq_qmv on the warp-MMA kernel too
+    try:
+        y_ref_gpu = api.aq_qmv(x, wq, s, b, 4, gs)
+    finally:
+        lib().aq_testing_set_qmv_kernel(0)
     ys = []
     for _ in range(2):
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
