@@ -196,6 +196,21 @@ def qmm(x16, wq, scales, biases, N, bits, gs, mode, dt, w_in_t=False):
     return y, den
 
 
+def gather_qmm(x16, wq, scales, biases, lhs, rhs, N, bits, gs, mode, dt, w_in_t=False):
+    """gather_qmm ("Add the 3bit packed qmm_t", ops and GatherQMM; the batch
+    offsets of adjust_matrix_offsets): x16 [Bx, M, K], wq [E, N, row bytes],
+    scales / biases [E, N, K/gs]; pair i multiplies x batch lhs[i] by the
+    transpose of weight matrix rhs[i].  -> (y [P, M, N], den [P, M, N])."""
+    ys, dens = [], []
+    for l, r in zip(lhs, rhs):
+        y, den = qmm(x16[int(l)], wq[int(r)], scales[int(r)],
+                     None if biases is None else biases[int(r)], N, bits, gs, mode, dt,
+                     w_in_t=w_in_t)
+        ys.append(y)
+        dens.append(den)
+    return np.stack(ys), np.stack(dens)
+
+
 def qmm_sampled(x16, wq, scales, biases, N, bits, gs, mode, dt, ms, ns, w_in_t=False):
     x16 = _c(x16, np.uint16)
     M, K = x16.shape

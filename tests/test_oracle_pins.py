@@ -694,3 +694,27 @@ def test_qqmm_is_qmm_over_fake_quantized_x():
     lut = np.array([float(v) for _, v in _golden_rows("fp4_e2m1_lut.txt")])
     W = lut[codes] * np.repeat(np.ldexp(1.0, sc.astype(np.int64) - 127), gs, axis=1)
     assert np.allclose(y, xh @ W.T, rtol=1e-12, atol=0)
+
+
+# ---------------------------------------------------------------- gather qmm
+
+def test_gather_qmm_selects_x_batch_and_weight_by_index():
+    """Pair i is x[lhs[i]] times the transpose of dequant(w[rhs[i]]), checked
+    against numpy on weights dequantized per expert; x batches and experts
+    differ in count and content, so swapped or ignored indices fail."""
+    rng = np.random.default_rng(11)
+    Bx, E, M, N, K, gs = 3, 4, 2, 8, 128, 64
+    x16 = f64_to_u16(rng.standard_normal((Bx, M, K)), BF16)
+    wq, sc, bi, W = [], [], [], []
+    for e in range(E):
+        w16 = f64_to_u16(rng.standard_normal((N, K)) * (e + 1), BF16)
+        q, s, b = oracle.quantize(w16, 4, gs, BF16)
+        wh, _ = oracle.dequantize(q, s, b, N, K, 4, gs, AFFINE, BF16)
+        wq.append(q); sc.append(s); bi.append(b); W.append(wh)
+    lhs = [2, 0, 1, 2, 0]
+    rhs = [1, 3, 3, 0, 2]
+    y, _ = oracle.gather_qmm(x16, np.stack(wq), np.stack(sc), np.stack(bi), lhs, rhs, N, 4, gs,
+                             AFFINE, BF16)
+    x = u16_to_f64(x16, BF16)
+    for i, (l, r) in enumerate(zip(lhs, rhs)):
+        assert np.allclose(y[i], x[l] @ W[r].T, rtol=1e-12, atol=1e-12), i
