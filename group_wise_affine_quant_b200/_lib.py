@@ -58,6 +58,10 @@ SIGNATURES["aq_qmv_batched"] = (_I, [ctypes.POINTER(QmvProblem), _I, _I64, _I, _
                                      _SZ, _P])
 SIGNATURES["aq_qmv_batched_workspace_size"] = (_SZ, [ctypes.POINTER(QmvProblem), _I, _I64, _I,
                                                      _I, _I])
+_I32P = ctypes.POINTER(ctypes.c_int32)
+SIGNATURES["aq_gather_qmm"] = (_I, [_P, _P, _P, _P, _I32P, _I32P, _P, _I64, _I64, _I64, _I64, _I64,
+                                    _I64, _I, _I, _I, _I, _P, _SZ, _P])
+SIGNATURES["aq_gather_qmm_workspace_size"] = (_SZ, [_I64, _I64, _I64, _I64, _I, _I, _I])
 
 _lib = None
 

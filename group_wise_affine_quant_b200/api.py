@@ -12,7 +12,7 @@ from . import _lib
 from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, AQ_OP_QMM,
                    AQ_OP_QMV, AQ_OP_QQMM, AqError, check, lib)
 
-__all__ = ["aq_quantize", "aq_quantize_fp4", "aq_quantize_dequantize_fp", "aq_qqmm", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_qconv2d_nhwc",
+__all__ = ["aq_quantize", "aq_quantize_fp4", "aq_quantize_dequantize_fp", "aq_qqmm", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_gather_qmm", "aq_qconv2d_nhwc",
            "aq_workspace_size", "aq_qmv_noalloc", "aq_last_error", "aq_set_weight_prefetch",
            "aq_get_weight_prefetch", "aq_set_input_prefetch", "aq_get_input_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
 
@@ -210,6 +210,34 @@ def aq_qmv_batched(xs, w_qs, scales, biases, bits=4, group_size=64, outs=None, w
                            0 if ws is None else ws.numel(), _stream(xs[0].device)),
           "aq_qmv_batched")
     return outs
+
+
+def aq_gather_qmm(x, w_q, scales, biases, lhs_indices=None, rhs_indices=None, bits=4,
+                  group_size=64, out=None, workspace=None):
+    """Pair i: y[i] = x[lhs[i]] . dequant(w[rhs[i]])^T, with x [Bx, M, K],
+    w_q [E, N, K*bits/8], scales / biases [E, N, K/group_size]; the index
+    lists are host sequences of int (None: 0, 1, ...).  Returns [P, M, N]."""
+    import ctypes
+    Bx, M, K = x.shape
+    E, N = w_q.shape[0], w_q.shape[1]
+    n = len(lhs_indices) if lhs_indices is not None else (
+        len(rhs_indices) if rhs_indices is not None else min(Bx, E))
+    mode = _mode(scales)
+
+    def arr(ix):
+        if ix is None:
+            return None
+        return (ctypes.c_int32 * n)(*[int(v) for v in ix])
+    if out is None:
+        out = torch.empty((n, M, N), dtype=x.dtype, device=x.device)
+    L = lib()
+    ws_bytes = L.aq_gather_qmm_workspace_size(n, M, N, K, bits, group_size, mode)
+    ws = (workspace or _default_ws).get(x.device, ws_bytes)
+    check(L.aq_gather_qmm(_ptr(x), _ptr(w_q), _ptr(scales), _ptr(biases), arr(lhs_indices),
+                          arr(rhs_indices), _ptr(out), n, M, N, K, Bx, E, bits, group_size, mode,
+                          _dt(x), _ptr(ws), 0 if ws is None else ws.numel(),
+                          _stream(x.device)), "aq_gather_qmm")
+    return out
 
 
 def aq_qmm(x, w_q, scales, biases, bits=4, group_size=64, out=None, workspace=None):

@@ -2,6 +2,7 @@
 // Every entry point validates on the host before it enqueues anything and
 // reports failures through its return value and a thread-local message.
 #include <stdarg.h>
+#include <stdint.h>
 #include <stdio.h>
 
 #include <algorithm>
@@ -347,6 +348,92 @@ aq_status aq_qmm(const void* x, const void* w_q, const void* scales, const void*
   return cuda_status(aq::launch_qmm(p, x, w_q, scales, biases, y, M, N, K, bits, group_size,
                                     mode, dtype, (cudaStream_t)stream),
                      "aq_qmm launch");
+}
+
+// Pointers of gather pair i (byte offsets of the batch strides).
+static aq_qmv_problem gather_pair(const void* x, const void* w_q, const void* scales,
+                                  const void* biases, void* y, int64_t l, int64_t r, int64_t i,
+                                  int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                                  aq_mode mode) {
+  const int64_t G = K / group_size;
+  const int64_t sb = mode == AQ_MODE_FP4 ? 1 : 2;            // bytes per scale / bias
+  aq_qmv_problem q;
+  q.x = static_cast<const uint8_t*>(x) + l * M * K * 2;
+  q.w_q = static_cast<const uint8_t*>(w_q) + r * N * (K * bits / 8);
+  q.scales = static_cast<const uint8_t*>(scales) + r * N * G * sb;
+  q.biases = biases ? static_cast<const uint8_t*>(biases) + r * N * G * sb : nullptr;
+  q.y = static_cast<uint8_t*>(y) + i * M * N * 2;
+  q.N = N;
+  q.K = K;
+  return q;
+}
+
+static aq_status check_gather(const int32_t* lhs, const int32_t* rhs, int64_t n_pairs,
+                              int64_t x_batch, int64_t w_batch) {
+  if (n_pairs < 0 || n_pairs > INT32_MAX)
+    return fail(AQ_ERR_INVALID_ARG, "n_pairs=%lld out of range", (long long)n_pairs);
+  if (x_batch < 1 || w_batch < 1)
+    return fail(AQ_ERR_INVALID_ARG, "x_batch and w_batch must be positive");
+  for (int64_t i = 0; i < n_pairs; ++i) {
+    const int64_t l = lhs ? lhs[i] : i, r = rhs ? rhs[i] : i;
+    if (l < 0 || l >= x_batch || r < 0 || r >= w_batch)
+      return fail(AQ_ERR_INVALID_ARG, "pair %lld: indices (%lld, %lld) outside x_batch %lld / w_batch %lld",
+                  (long long)i, (long long)l, (long long)r, (long long)x_batch, (long long)w_batch);
+  }
+  return AQ_OK;
+}
+
+aq_status aq_gather_qmm(const void* x, const void* w_q, const void* scales, const void* biases,
+                        const int32_t* lhs_indices, const int32_t* rhs_indices, void* y,
+                        int64_t n_pairs, int64_t M, int64_t N, int64_t K, int64_t x_batch,
+                        int64_t w_batch, int bits, int group_size, aq_mode mode, aq_dtype dtype,
+                        void* workspace, size_t workspace_bytes, aq_stream_t stream) {
+  g_err[0] = 0;
+  aq_status st = check_gather(lhs_indices, rhs_indices, n_pairs, x_batch, w_batch);
+  if (st != AQ_OK) return st;
+  if ((st = check_weight(w_q, scales, biases, N, K, bits, group_size, mode, dtype)) != AQ_OK)
+    return st;
+  if ((st = check_mm(x, y, M, N, K)) != AQ_OK) return st;
+  if (n_pairs == 0 || M == 0 || N == 0) return AQ_OK;
+  if (K == 0) return zero_output(y, n_pairs * M, N, stream);
+  std::vector<aq_qmv_problem> P((size_t)n_pairs);
+  for (int64_t i = 0; i < n_pairs; ++i)
+    P[(size_t)i] = gather_pair(x, w_q, scales, biases, y,
+                               lhs_indices ? lhs_indices[i] : i, rhs_indices ? rhs_indices[i] : i,
+                               i, M, N, K, bits, group_size, mode);
+  // Decode-sized pairs whose matrices the batched decode kernels take run as
+  // one batch (the unit scheduler walks every pair's row tiles and K-slices);
+  // the others, and M > 16, run one call per pair.
+  if (M <= 16 && check_batch(P.data(), (int)n_pairs, M, bits, group_size, mode, dtype) == AQ_OK)
+    return aq_qmv_batched(P.data(), (int)n_pairs, M, bits, group_size, mode, dtype, workspace,
+                          workspace_bytes, stream);
+  g_err[0] = 0;
+  for (int64_t i = 0; i < n_pairs; ++i) {
+    const aq_qmv_problem& q = P[(size_t)i];
+    st = M <= 16 ? aq_qmv(q.x, q.w_q, q.scales, q.biases, q.y, M, N, K, bits, group_size, mode,
+                          dtype, workspace, workspace_bytes, stream)
+                 : aq_qmm(q.x, q.w_q, q.scales, q.biases, q.y, M, N, K, bits, group_size, mode,
+                          dtype, nullptr, 0, stream);
+    if (st != AQ_OK) {
+      char msg[640];
+      snprintf(msg, sizeof(msg), "pair %lld: %s", (long long)i, g_err);
+      return fail(st, "%s", msg);
+    }
+  }
+  return AQ_OK;
+}
+
+size_t aq_gather_qmm_workspace_size(int64_t n_pairs, int64_t M, int64_t N, int64_t K, int bits,
+                                    int group_size, aq_mode mode) {
+  if (n_pairs <= 0 || n_pairs > INT32_MAX || M < 1 || M > 16 || N <= 0 || K <= 0 ||
+      group_size <= 0 || K % group_size)
+    return 0;
+  // Sized for either path: the batch (aligned stand-in pointers; the size
+  // depends on the shapes only) and one call per pair.
+  const void* a = reinterpret_cast<const void*>((uintptr_t)1 << 20);
+  std::vector<aq_qmv_problem> P((size_t)n_pairs, aq_qmv_problem{a, a, a, a, const_cast<void*>(a), N, K});
+  return std::max(aq_qmv_batched_workspace_size(P.data(), (int)n_pairs, M, bits, group_size, mode),
+                  aq_workspace_size(AQ_OP_QMV, M, N, K, bits, group_size, mode, 1));
 }
 
 aq_status aq_quantize_dequantize_fp(const void* x, void* out, int64_t N, int64_t K, int bits,

@@ -521,7 +521,13 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
           const int slot = wc % ST;
           if (!mbar_wait(smem_u32(full + slot), (wc / ST) & 1, abort_flag, wl)) { ok = false; break; }
           const uint8_t* w0 = smem + S::kRingOff + slot * S::kStage + (warp * 16 * R + g) * 128 + t * 4;
-          float d[R][NT][4];
+          // NT == 1: two accumulators per tile (the aA and aB K-steps of a word),
+          // so a group's MMAs form two chains of half the depth; the epilogue
+          // adds them.  With the group's epilogue operands loaded at its first
+          // step (below), this measured 1.4 % faster on the batched decode step
+          // than one accumulator with the operands loaded at the last step.
+          constexpr bool kTwoAcc = NT == 1;
+          float d[R][NT][4], d2[R][NT][4];
           // codes of rows g and g + 8 of both tiles, and x, one step ahead
           uint32_t cw[R][2], cn[R][2];
           uint4 xc[NT], xn[NT];
@@ -540,10 +546,21 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
             }
           };
           load_step(0, cw, xc);
+          float2 pe0[R], pe1[R], psx[NT];             // the group's (s, b') rows and x sums
 #pragma unroll
           for (int s = 0; s < 8; ++s) {
+            if ((s & (GS / 32 - 1)) == 0) {             // first step of a group
+              const int gi0 = ((st * 8 + s) * 32) / GS;
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                psx[nt] = *reinterpret_cast<const float2*>(xs + gi0 * 16 + 8 * nt);
+#pragma unroll
+              for (int r = 0; r < R; ++r) {
+                pe0[r] = tab[r * 16 * S::kTabPitch + gi0];
+                pe1[r] = tab[(r * 16 + 8) * S::kTabPitch + gi0];
+              }
+            }
             if (s < 7) load_step(s + 1, cn, xn);
-            const int blk = st * 8 + s;                       // 32-column block of the sub-slice
             constexpr int kFirstMask = GS / 32 - 1;
             constexpr uint32_t kLo = 0x000F000Fu;
 #pragma unroll
@@ -560,25 +577,37 @@ qmv_mma_kernel(const __grid_constant__ MvParams<P> pr) {
               aB[3] = and_or(wb >> 12, kLo, kMag);
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
-                if ((s & kFirstMask) == 0)
-                  mma16816_z<T>(d[r][nt], aA, xc[nt].x, xc[nt].y);
-                else
-                  mma16816<T>(d[r][nt], aA, xc[nt].x, xc[nt].y);
-                mma16816<T>(d[r][nt], aB, xc[nt].z, xc[nt].w);
+                if (kTwoAcc) {
+                  if ((s & kFirstMask) == 0) {
+                    mma16816_z<T>(d[r][nt], aA, xc[nt].x, xc[nt].y);
+                    mma16816_z<T>(d2[r][nt], aB, xc[nt].z, xc[nt].w);
+                  } else {
+                    mma16816<T>(d[r][nt], aA, xc[nt].x, xc[nt].y);
+                    mma16816<T>(d2[r][nt], aB, xc[nt].z, xc[nt].w);
+                  }
+                } else {
+                  if ((s & kFirstMask) == 0)
+                    mma16816_z<T>(d[r][nt], aA, xc[nt].x, xc[nt].y);
+                  else
+                    mma16816<T>(d[r][nt], aA, xc[nt].x, xc[nt].y);
+                  mma16816<T>(d[r][nt], aB, xc[nt].z, xc[nt].w);
+                }
               }
             }
             if ((s & kFirstMask) == kFirstMask) {
-              const int gi = (blk * 32) / GS;
               float2 sx[NT];
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-                sx[nt] = *reinterpret_cast<const float2*>(xs + gi * 16 + 8 * nt);
+              for (int nt = 0; nt < NT; ++nt) sx[nt] = psx[nt];
 #pragma unroll
               for (int r = 0; r < R; ++r) {
-                const float2 e0 = tab[r * 16 * S::kTabPitch + gi];
-                const float2 e1 = tab[(r * 16 + 8) * S::kTabPitch + gi];
+                const float2 e0 = pe0[r];
+                const float2 e1 = pe1[r];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
+                  if (kTwoAcc) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) d[r][nt][i] += d2[r][nt][i];
+                  }
                   acc[r][nt][0] = fmaf(e0.x, d[r][nt][0], fmaf(e0.y, sx[nt].x, acc[r][nt][0]));
                   acc[r][nt][1] = fmaf(e0.x, d[r][nt][1], fmaf(e0.y, sx[nt].y, acc[r][nt][1]));
                   acc[r][nt][2] = fmaf(e1.x, d[r][nt][2], fmaf(e1.y, sx[nt].x, acc[r][nt][2]));

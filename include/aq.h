@@ -190,6 +190,35 @@ AQ_API aq_status aq_qmv_batched(const aq_qmv_problem* problems, int count, int64
                                 size_t workspace_bytes, aq_stream_t stream);
 
 /*
+ * aq_gather_qmm — batched matmul over index pairs ("Add the 3bit packed
+ * qmm_t": gather_qmm in the ops and bindings, GatherQMM, and the per-matrix
+ * offsets of adjust_matrix_offsets): for pair i,
+ *   y[i] [M, N] = x[lhs_indices[i]] [M, K] . dequant(w[rhs_indices[i]])^T
+ * e.g. the experts a mixture-of-experts layer routes each token block to.
+ *   x        [x_batch, M, K] T;   y [n_pairs, M, N] T
+ *   w_q      [w_batch, N, K*bits/8];  scales / biases [w_batch, N, K/group_size]
+ *   lhs_indices, rhs_indices: HOST arrays of n_pairs int32 (read before the
+ *            call returns; NULL means index i), each in range or
+ *            AQ_ERR_INVALID_ARG.
+ * Each pair's result is the one aq_qmv (M <= 16) or aq_qmm defines.  Pairs of
+ * decode size whose matrices meet aq_qmv_batched's conditions run as one
+ * batch (one launch per 40 pairs); the others run one call per pair, and
+ * every pair's pointers must then meet that call's alignment rules (the
+ * error names the pair).  Workspace: aq_gather_qmm_workspace_size bytes,
+ * under aq_qmv's rules.
+ */
+AQ_API aq_status aq_gather_qmm(const void* x, const void* w_q, const void* scales,
+                               const void* biases, const int32_t* lhs_indices,
+                               const int32_t* rhs_indices, void* y, int64_t n_pairs, int64_t M,
+                               int64_t N, int64_t K, int64_t x_batch, int64_t w_batch, int bits,
+                               int group_size, aq_mode mode, aq_dtype dtype, void* workspace,
+                               size_t workspace_bytes, aq_stream_t stream);
+
+/* Workspace bytes for aq_gather_qmm with these sizes (0 for M > 16). */
+AQ_API size_t aq_gather_qmm_workspace_size(int64_t n_pairs, int64_t M, int64_t N, int64_t K,
+                                           int bits, int group_size, aq_mode mode);
+
+/*
  * aq_qmv_noalloc — aq_qmv for callers that cannot allocate device memory or
  * manage a workspace buffer: e.g. code that runs after a serving process has
  * fixed its device memory (no cudaMalloc allowed past start-up), or that has

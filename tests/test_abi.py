@@ -206,3 +206,27 @@ def test_qqmm_validation_and_workspace():
     assert q(A, A, A, A, 4, 256, 1024, 32, 1, A + 16, 1 << 30, None) == MISALIGNED
     assert q(A + 2, A, A, A, 4, 256, 1024, 32, 1, A, 1 << 30, None) == MISALIGNED
     assert q(A, A, A, A, 0, 256, 1024, 32, 1, None, 0, None) == OK             # M = 0
+
+
+def test_gather_qmm_validation():
+    g = L().aq_gather_qmm
+    I32 = ctypes.c_int32 * 3
+
+    def call(lhs=None, rhs=None, n=3, M=1, xb=3, wb=3, **kw):
+        a = dict(x=A, w=A, s=A, b=A, y=A, N=256, K=2048, bits=4, gs=64, mode=0, dt=1, ws=A,
+                 wsb=1 << 30)
+        a.update(kw)
+        return g(a["x"], a["w"], a["s"], a["b"], lhs, rhs, a["y"], n, M, a["N"], a["K"], xb, wb,
+                 a["bits"], a["gs"], a["mode"], a["dt"], a["ws"], a["wsb"], None)
+    assert call(n=0) == OK
+    assert call(lhs=I32(0, 1, 3)) == INVALID                      # x batch 3 out of range
+    assert b"pair 2" in L().aq_last_error()
+    assert call(rhs=I32(0, -1, 1)) == INVALID
+    assert call(n=4) == INVALID                                   # identity needs 4 batches
+    assert call(xb=0) == INVALID
+    assert call(bits=7) == UNSUPPORTED
+    assert call(b=None) == INVALID                                # affine needs biases
+    ws = L().aq_gather_qmm_workspace_size
+    assert ws(3, 16, 2048, 8192, 4, 64, 0) > 0
+    assert ws(3, 17, 2048, 8192, 4, 64, 0) == 0                   # qmm pairs need none
+    assert ws(0, 1, 2048, 8192, 4, 64, 0) == 0
