@@ -196,6 +196,18 @@ def qmm(x16, wq, scales, biases, N, bits, gs, mode, dt, w_in_t=False):
     return y, den
 
 
+def qmm_nt(x16, wq, scales, biases, K, bits, gs, mode, dt):
+    """The non-transposed product of quantized_matmul (transpose = false; the
+    product its VJP forms for x): with the weight stored as [N, K] rows
+    quantized along K, y [M, K] = x [M, N] . w_hat [N, K], in fp64 over the
+    exact w_hat.  -> (y [M, K], den [M, K] = sum_n |x w_hat|)."""
+    x16 = _c(x16, np.uint16)
+    M, N = x16.shape
+    wh, _ = dequantize(wq, scales, biases, N, K, bits, gs, mode, dt)
+    x = np.array([[t_to_double(int(v), dt) for v in row] for row in x16], np.float64).reshape(M, N)
+    return x @ wh, np.abs(x) @ np.abs(wh)
+
+
 def gather_qmm(x16, wq, scales, biases, lhs, rhs, N, bits, gs, mode, dt, w_in_t=False):
     """gather_qmm ("Add the 3bit packed qmm_t", ops and GatherQMM; the batch
     offsets of adjust_matrix_offsets): x16 [Bx, M, K], wq [E, N, row bytes],

@@ -718,3 +718,28 @@ def test_gather_qmm_selects_x_batch_and_weight_by_index():
     x = u16_to_f64(x16, BF16)
     for i, (l, r) in enumerate(zip(lhs, rhs)):
         assert np.allclose(y[i], x[l] @ W[r].T, rtol=1e-12, atol=1e-12), i
+
+
+# ------------------------------------------------------- non-transposed qmm
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_qmm_nt_is_x_times_w_hat_by_brute_force(bits):
+    """y[m, k] = sum_n x[m, n] (s[n, k/gs] q[n, k] + b[n, k/gs]), summed by
+    plain loops over codes unpacked with the numpy packer (not the oracle's
+    dequantize); a transposed operand or a group index along the wrong axis
+    fails."""
+    rng = np.random.default_rng(bits)
+    M, N, K, gs = 2, 5, 64, 32
+    codes = rng.integers(0, 2 ** bits, size=(N, K)).astype(np.uint8)
+    wq = np_pack(codes, bits)
+    s16 = f64_to_u16(rng.standard_normal((N, K // gs)) * 0.1, BF16)
+    b16 = f64_to_u16(rng.standard_normal((N, K // gs)) * 0.1, BF16)
+    x16 = f64_to_u16(rng.standard_normal((M, N)), BF16)
+    y, den = oracle.qmm_nt(x16, wq, s16, b16, K, bits, gs, AFFINE, BF16)
+    assert y.shape == (M, K)
+    s, b, x = u16_to_f64(s16, BF16), u16_to_f64(b16, BF16), u16_to_f64(x16, BF16)
+    q = np_unpack(wq, N, K, bits)
+    for m in range(M):
+        for k in range(K):
+            want = sum(x[m, n] * (s[n, k // gs] * q[n, k] + b[n, k // gs]) for n in range(N))
+            assert abs(y[m, k] - want) <= 1e-12 * (1 + abs(want)), (m, k)
