@@ -316,6 +316,7 @@ def side_lines(torch, api, inputs, dev, stream, hbm, tf_peak):
     Every weight here is quantized before its timed calls and no timed kernel
     writes one, so the kernels may stream weights before their dependency wait
     (the same setting as the decode step)."""
+    import random
     out, tfl = {}, {}
     api.aq_set_weight_prefetch(True)
     # --- tiny fp16 qmv/qmm (512x512, 4-bit g64), M = 1 and 8: L2-resident, so
@@ -360,6 +361,70 @@ def side_lines(torch, api, inputs, dev, stream, hbm, tf_peak):
             tfl["fp4_%s_M%d" % (kind, M)] = {"tflops": round(2 * M * 4096 * 4096 / (t * 1e-3) / 1e12, 1),
                                             "ms": round(t, 4)}
         del wcs
+    # --- W4A4 (aq_qqmm): x fake-quantized to FP4 E8M0 g32, FP4 weights
+    # 4096 x 4096 (20 copies for the decode rows, 180 MB > L2)
+    copies = [inputs.fp4(4096, 4096, 32, seed=80 + i) for i in range(20)]
+    wcs = [(c.to(dev), sc.to(dev)) for c, sc in copies]
+    del copies
+    for M in (1, 16):
+        xf = inputs.fp4_x(M, 4096).to(dev)
+        yf = [torch.empty((M, 4096), dtype=torch.bfloat16, device=dev) for _ in wcs]
+        byt = 20 * (4096 * 2048 + 4096 * 128 + 2 * M * 4096 * 2)
+
+        def chain_qq():
+            for (c, sc), yy in zip(wcs, yf):
+                api.aq_qqmm(xf, c, sc, 32, out=yy)
+        t = graph_time_ms(torch, stream, chain_qq, 2)
+        out["w4a4_qqmm_M%d" % M] = {"per_call_gbs": round(byt / (t * 1e-3) / 1e9, 1),
+                                    "us_per_call": round(t * 1e3 / 20, 2),
+                                    "launches_per_call": 2}
+    wc, sc = wcs[0]
+    for M in (256, 4096):
+        xf = inputs.fp4_x(M, 4096).to(dev)
+        yf = torch.empty((M, 4096), dtype=torch.bfloat16, device=dev)
+        t = graph_time_ms(torch, stream, lambda: api.aq_qqmm(xf, wc, sc, 32, out=yf), 10)
+        out["w4a4_qqmm_M%d" % M] = {"tflops": round(2 * M * 4096 * 4096 / (t * 1e-3) / 1e12, 1),
+                                    "ms": round(t, 4), "launches_per_call": 2}
+    del wcs
+    # --- gather (aq_gather_qmm): a mixture-of-experts decode step, 8 experts
+    # of 1408 x 2048 (bf16, 4-bit g64), 48 token rows routed to 2 experts each:
+    # 96 pairs, each pair streaming its expert's weights (the pair path)
+    E, NE, KE, TOK = 8, 1408, 2048, 48
+    qs = [api.aq_quantize(inputs.normal((NE, KE), 0.02, 1, inputs.gen(90 + e)).to(dev), 4, 64)
+          for e in range(E)]
+    wq_e, s_e, b_e = (torch.stack([q[j] for q in qs]) for j in range(3))
+    del qs
+    xg = inputs.normal((TOK, 1, KE), 1.0, 1, inputs.gen(98)).to(dev)
+    grng = random.Random(5)
+    lhs = [t for t in range(TOK) for _ in range(2)]
+    rhs = [e for t in range(TOK) for e in grng.sample(range(E), 2)]
+    yg = torch.empty((len(lhs), 1, NE), dtype=torch.bfloat16, device=dev)
+    t = graph_time_ms(torch, stream, lambda: api.aq_gather_qmm(xg, wq_e, s_e, b_e, lhs, rhs, 4, 64,
+                                                               out=yg), 5)
+    pair_bytes = NE * KE // 2 + 4 * NE * (KE // 64) + 2 * KE + 2 * NE
+    out["gather_moe_decode_96pairs"] = {
+        "us_per_call": round(t * 1e3, 2),
+        "gbs_pair_bytes": round(len(lhs) * pair_bytes / (t * 1e-3) / 1e9, 1),
+        "note": "each pair streams its expert (8 experts read 12 times each on average)"}
+    del wq_e, s_e, b_e
+    # --- non-transposed product (aq_qmm_nt, dy . W): the down projection's
+    # weight (2048 x 8192, bf16, 4-bit g64), x [M, 2048] -> y [M, 8192];
+    # 16 weight copies (150 MB > L2)
+    wts = [api.aq_quantize(inputs.normal((2048, 8192), 0.02, 1, inputs.gen(120 + i)).to(dev), 4, 64)
+           for i in range(16)]
+    for M in (1, 16):
+        xn = inputs.normal((M, 2048), 1.0, 1, inputs.gen(130)).to(dev)
+        yn = torch.empty((M, 8192), dtype=torch.bfloat16, device=dev)
+
+        def chain_nt():
+            for q in wts:
+                api.aq_qmm_nt(xn, *q, 4, 64, out=yn)
+        t = graph_time_ms(torch, stream, chain_nt, 2)
+        byt = 16 * (2048 * 4096 + 4 * 2048 * 128 + 2 * M * 2048 + 2 * M * 8192)
+        out["qmm_nt_down_M%d" % M] = {"gbs": round(byt / (t * 1e-3) / 1e9, 1),
+                                      "us_per_call": round(t * 1e3 / 16, 2),
+                                      "frac_of_hbm": round(byt / (t * 1e-3) / 1e9 / hbm, 4)}
+    del wts
     # --- chained fp16 qmm, 20 products per chain, bits 2, 3, 4, 6, 8
     x, w1, w2 = inputs.chained()
     xd = x.to(dev)

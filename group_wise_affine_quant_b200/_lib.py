@@ -15,7 +15,7 @@ STATUS_NAMES = {0: "AQ_OK", 1: "AQ_ERR_INVALID_ARG", 2: "AQ_ERR_UNSUPPORTED",
                 3: "AQ_ERR_MISALIGNED", 4: "AQ_ERR_CUDA", 5: "AQ_ERR_WORKSPACE"}
 AQ_F16, AQ_BF16 = 0, 1
 AQ_MODE_AFFINE, AQ_MODE_FP4 = 0, 1
-AQ_OP_QMV, AQ_OP_QMM, AQ_OP_QCONV2D, AQ_OP_QQMM = 0, 1, 2, 3
+AQ_OP_QMV, AQ_OP_QMM, AQ_OP_QCONV2D, AQ_OP_QQMM, AQ_OP_QMM_NT = 0, 1, 2, 3, 4
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -30,6 +30,7 @@ SIGNATURES = {
     "aq_qqmm": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _P, _SZ, _P]),
     "aq_qmv": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
     "aq_qmm": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
+    "aq_qmm_nt": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _SZ, _P]),
     "aq_qmv_noalloc": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I, _I, _I, _P]),
     "aq_qconv2d_nhwc": (_I, [_P, _P, _P, _P, _P] + [_I] * 15 + [_P, _SZ, _P]),
     "aq_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I, _I, _I, _I]),

@@ -10,9 +10,9 @@ import torch
 
 from . import _lib
 from ._lib import (AQ_BF16, AQ_F16, AQ_MODE_AFFINE, AQ_MODE_FP4, AQ_OP_QCONV2D, AQ_OP_QMM,
-                   AQ_OP_QMV, AQ_OP_QQMM, AqError, check, lib)
+                   AQ_OP_QMM_NT, AQ_OP_QMV, AQ_OP_QQMM, AqError, check, lib)
 
-__all__ = ["aq_quantize", "aq_quantize_fp4", "aq_quantize_dequantize_fp", "aq_qqmm", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_gather_qmm", "aq_qconv2d_nhwc",
+__all__ = ["aq_quantize", "aq_quantize_fp4", "aq_quantize_dequantize_fp", "aq_qqmm", "aq_dequantize", "aq_qmv", "aq_qmv_batched", "aq_qmm", "aq_qmm_nt", "aq_gather_qmm", "aq_qconv2d_nhwc",
            "aq_workspace_size", "aq_qmv_noalloc", "aq_last_error", "aq_set_weight_prefetch",
            "aq_get_weight_prefetch", "aq_set_input_prefetch", "aq_get_input_prefetch", "AqError", "AQ_MODE_AFFINE", "AQ_MODE_FP4", "Workspace"]
 
@@ -243,6 +243,22 @@ def aq_gather_qmm(x, w_q, scales, biases, lhs_indices=None, rhs_indices=None, bi
 def aq_qmm(x, w_q, scales, biases, bits=4, group_size=64, out=None, workspace=None):
     """y = x . dequant(w)^T for any M."""
     return _mm("aq_qmm", AQ_OP_QMM, x, w_q, scales, biases, bits, group_size, out, workspace)
+
+
+def aq_qmm_nt(x, w_q, scales, biases, bits=4, group_size=64, out=None, workspace=None):
+    """y [M, K] = x [M, N] . dequant(w) with the weight stored [N, K] as for
+    aq_qmv / aq_qmm (the transpose = false product)."""
+    M, N = x.shape
+    K = w_q.shape[1] * 8 // bits
+    mode = _mode(scales)
+    if out is None:
+        out = torch.empty((M, K), dtype=x.dtype, device=x.device)
+    ws_bytes = aq_workspace_size(AQ_OP_QMM_NT, M, N, K, bits, group_size, mode)
+    ws = (workspace or _default_ws).get(x.device, ws_bytes)
+    check(lib().aq_qmm_nt(_ptr(x), _ptr(w_q), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, bits,
+                          group_size, mode, _dt(x), _ptr(ws), 0 if ws is None else ws.numel(),
+                          _stream(x.device)), "aq_qmm_nt")
+    return out
 
 
 def conv_out_hw(H, W, kh, kw, stride, pad):

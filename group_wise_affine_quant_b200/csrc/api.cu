@@ -436,6 +436,27 @@ size_t aq_gather_qmm_workspace_size(int64_t n_pairs, int64_t M, int64_t N, int64
                   aq_workspace_size(AQ_OP_QMV, M, N, K, bits, group_size, mode, 1));
 }
 
+aq_status aq_qmm_nt(const void* x, const void* w_q, const void* scales, const void* biases,
+                    void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                    aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
+                    aq_stream_t stream) {
+  g_err[0] = 0;
+  aq_status st = check_weight(w_q, scales, biases, N, K, bits, group_size, mode, dtype);
+  if (st != AQ_OK) return st;
+  if (M < 0 || M > kMaxDim) return fail(AQ_ERR_INVALID_ARG, "M=%lld out of range", (long long)M);
+  if (M == 0 || K == 0) return AQ_OK;
+  if (!y) return fail(AQ_ERR_INVALID_ARG, "y must not be NULL");
+  if (!aligned(y, 16)) return fail(AQ_ERR_MISALIGNED, "y must be 16-byte aligned");
+  if (N == 0) return zero_output(y, M, K, stream);
+  if (!x) return fail(AQ_ERR_INVALID_ARG, "x must not be NULL");
+  if (!aligned(x, 2)) return fail(AQ_ERR_MISALIGNED, "x must be 2-byte aligned");
+  const size_t need = aq::qmm_nt_workspace(M, N, K);
+  if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
+  return cuda_status(aq::launch_qmm_nt(x, w_q, scales, biases, y, M, N, K, bits, group_size, mode,
+                                       dtype, workspace, (cudaStream_t)stream),
+                     "aq_qmm_nt launch");
+}
+
 aq_status aq_quantize_dequantize_fp(const void* x, void* out, int64_t N, int64_t K, int bits,
                                     int group_size, aq_dtype dtype, aq_stream_t stream) {
   g_err[0] = 0;
@@ -569,6 +590,7 @@ size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, in
     return std::max(need, aq::plan_qmv(M, N, K, bits, group_size, mode).ws_bytes);
   }
   if (op == AQ_OP_QQMM) return qqmm_mm_bytes(M, N, K, group_size) + (size_t)(M * K) * 2;
+  if (op == AQ_OP_QMM_NT) return aq::qmm_nt_workspace(M, N, K);
   return 0;
 }
 

@@ -86,6 +86,10 @@ cudaError_t launch_quantize(const void* w, void* w_q, void* scales, void* biases
                             int64_t K, int bits, int gs, int dtype, cudaStream_t st);
 cudaError_t launch_quantize_fp4(const void* w, void* codes, void* scales, int64_t N, int64_t K,
                                 int gs, int dtype, cudaStream_t st);
+size_t qmm_nt_workspace(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_qmm_nt(const void* x, const void* w_q, const void* scales, const void* biases,
+                          void* y, int64_t M, int64_t N, int64_t K, int bits, int gs, int mode,
+                          int dtype, void* workspace, cudaStream_t st);
 cudaError_t launch_quantize_dequantize_fp(const void* w, void* out, int64_t N, int64_t K, int bits,
                                           int gs, int dtype, cudaStream_t st);
 cudaError_t launch_dequantize(const void* w_q, const void* scales, const void* biases,

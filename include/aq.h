@@ -76,7 +76,9 @@ typedef enum {
   AQ_MODE_FP4 = 1           /* bits = 4; group_size 32 (E8M0) or 16 (E4M3); biases NULL */
 } aq_mode;
 
-typedef enum { AQ_OP_QMV = 0, AQ_OP_QMM = 1, AQ_OP_QCONV2D = 2, AQ_OP_QQMM = 3 } aq_op;
+typedef enum {
+  AQ_OP_QMV = 0, AQ_OP_QMM = 1, AQ_OP_QCONV2D = 2, AQ_OP_QQMM = 3, AQ_OP_QMM_NT = 4
+} aq_op;
 
 /*
  * aq_quantize — affine group quantizer ("mlx 1.0.0, .../quantized.cpp",
@@ -188,6 +190,26 @@ typedef struct aq_qmv_problem {
 AQ_API aq_status aq_qmv_batched(const aq_qmv_problem* problems, int count, int64_t M, int bits,
                                 int group_size, aq_mode mode, aq_dtype dtype, void* workspace,
                                 size_t workspace_bytes, aq_stream_t stream);
+
+/*
+ * aq_qmm_nt — the non-transposed product of a quantized weight ("Add the
+ * 3bit packed qmm_t": quantized_matmul with transpose = false, the product
+ * its VJP forms for x):
+ *   y [M, K] = x [M, N] . w_hat [N, K]
+ * with w_q / scales / biases exactly as aq_qmv / aq_qmm take them (N rows of
+ * K codes quantized along K), so one stored weight serves both x . w_hat^T
+ * and x . w_hat.  x [M, N] T (2-byte aligned), y [M, K] T (16-byte aligned).
+ * fp32 arithmetic on the exact w_hat (scale and bias kept as factors of the
+ * codes); each y is rounded to T once.  Runs 16 rows of x per launch (the
+ * weight is streamed once per 16 rows).  Workspace:
+ * aq_workspace_size(AQ_OP_QMM_NT, M, N, K, bits, group_size, mode, 1) bytes
+ * under aq_qmv's rules (partial sums after the first 64 KB, which the call
+ * leaves untouched).
+ */
+AQ_API aq_status aq_qmm_nt(const void* x, const void* w_q, const void* scales, const void* biases,
+                           void* y, int64_t M, int64_t N, int64_t K, int bits, int group_size,
+                           aq_mode mode, aq_dtype dtype, void* workspace, size_t workspace_bytes,
+                           aq_stream_t stream);
 
 /*
  * aq_gather_qmm — batched matmul over index pairs ("Add the 3bit packed

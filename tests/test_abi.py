@@ -230,3 +230,23 @@ def test_gather_qmm_validation():
     assert ws(3, 16, 2048, 8192, 4, 64, 0) > 0
     assert ws(3, 17, 2048, 8192, 4, 64, 0) == 0                   # qmm pairs need none
     assert ws(0, 1, 2048, 8192, 4, 64, 0) == 0
+
+
+def test_qmm_nt_validation_and_workspace():
+    f = L().aq_qmm_nt
+
+    def call(**kw):
+        a = dict(x=A, w=A, s=A, b=A, y=A, M=1, N=640, K=1024, bits=4, gs=64, mode=0, dt=1, ws=A,
+                 wsb=1 << 30)
+        a.update(kw)
+        return f(a["x"], a["w"], a["s"], a["b"], a["y"], a["M"], a["N"], a["K"], a["bits"], a["gs"],
+                 a["mode"], a["dt"], a["ws"], a["wsb"], None)
+    assert call(bits=7) == UNSUPPORTED
+    assert call(K=96, gs=64) == INVALID
+    assert call(y=A + 8) == MISALIGNED
+    assert call(x=A + 1) == MISALIGNED
+    assert call(M=0) == OK
+    need = L().aq_workspace_size(4, 16, 640, 1024, 4, 64, 0, 1)
+    assert need > 65536                                       # partials after the counters
+    assert call(M=16, ws=None, wsb=0) == WORKSPACE
+    assert L().aq_workspace_size(4, 1, 48, 1024, 4, 64, 0, 1) == 0   # one split: no partials
