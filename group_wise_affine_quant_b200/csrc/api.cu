@@ -450,7 +450,7 @@ aq_status aq_qmm_nt(const void* x, const void* w_q, const void* scales, const vo
   if (N == 0) return zero_output(y, M, K, stream);
   if (!x) return fail(AQ_ERR_INVALID_ARG, "x must not be NULL");
   if (!aligned(x, 2)) return fail(AQ_ERR_MISALIGNED, "x must be 2-byte aligned");
-  const size_t need = aq::qmm_nt_workspace(M, N, K);
+  const size_t need = aq::qmm_nt_workspace(M, N, K, bits);
   if ((st = check_workspace(workspace, workspace_bytes, need)) != AQ_OK) return st;
   return cuda_status(aq::launch_qmm_nt(x, w_q, scales, biases, y, M, N, K, bits, group_size, mode,
                                        dtype, workspace, (cudaStream_t)stream),
@@ -590,7 +590,7 @@ size_t aq_workspace_size(aq_op op, int64_t M, int64_t N, int64_t K, int bits, in
     return std::max(need, aq::plan_qmv(M, N, K, bits, group_size, mode).ws_bytes);
   }
   if (op == AQ_OP_QQMM) return qqmm_mm_bytes(M, N, K, group_size) + (size_t)(M * K) * 2;
-  if (op == AQ_OP_QMM_NT) return aq::qmm_nt_workspace(M, N, K);
+  if (op == AQ_OP_QMM_NT) return aq::qmm_nt_workspace(M, N, K, bits);
   return 0;
 }
 

@@ -205,7 +205,8 @@ cudaError_t nt_by_bits(const void* x, const void* w_q, const void* scales, const
 
 }  // namespace
 
-size_t qmm_nt_workspace(int64_t M, int64_t N, int64_t K) {
+size_t qmm_nt_workspace(int64_t M, int64_t N, int64_t K, int bits) {
+  (void)bits;
   const NtPlan p = plan_nt(N, K);
   if (p.splits <= 1) return 0;
   return kNtCounterArea + (size_t)p.splits * (size_t)std::min<int64_t>(M, 16) * (size_t)K * 4;

@@ -246,7 +246,8 @@ def test_qmm_nt_validation_and_workspace():
     assert call(y=A + 8) == MISALIGNED
     assert call(x=A + 1) == MISALIGNED
     assert call(M=0) == OK
-    need = L().aq_workspace_size(4, 16, 640, 1024, 4, 64, 0, 1)
+    need = L().aq_workspace_size(4, 1, 640, 1024, 4, 64, 0, 1)
     assert need > 65536                                       # partials after the counters
-    assert call(M=16, ws=None, wsb=0) == WORKSPACE
-    assert L().aq_workspace_size(4, 1, 48, 1024, 4, 64, 0, 1) == 0   # one split: no partials
+    assert call(M=1, ws=None, wsb=0) == WORKSPACE
+    assert L().aq_workspace_size(4, 16, 640, 1024, 4, 64, 0, 1) > need   # partials grow with M
+    assert L().aq_workspace_size(4, 1, 32, 1024, 4, 64, 0, 1) == 0   # one split: no partials
