@@ -724,6 +724,21 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
           ++j;
         }
       }
+      // On abort, the copies still in flight land before the CTA exits: a
+      // bounded wait on the full barrier of every chunk issued in the last
+      // lap of each ring (these barriers take only the TMA's bytes).
+      if (*abort_flag && lane == 0) {
+        auto drain = [&](int base, int slots, int issued) {
+          for (int q = issued - 1; q >= 0 && q >= issued - slots; --q) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(full_l(base + q % slots), (q / slots) & 1))
+              if (globaltimer_ns() - t0 > 1000000000ull) break;
+          }
+        };
+        drain(0, WS, c);
+        drain(WS, SS, j);
+      }
+      __syncwarp();
     } else {
       // ------------------ packed codes, scales, biases by cp.async
       // Each lane copies 4 rows per stage, one commit group per stage, and
@@ -806,6 +821,14 @@ qmm_tc_kernel(const __grid_constant__ QmmMaps maps, const QmmArgs a) {
     // abort, so nothing is in flight when TMEM is freed).  The elected lane
     // is the issuing lane (the lowest lane of the full warp).
     if (elect_one()) mma_commit(acc_full);
+    __syncwarp();
+    // This warp frees TMEM at the end: every MMA it issued has completed by
+    // then, also on abort, when the epilogue does not wait for them (bounded).
+    {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(acc_full, 0))
+        if (globaltimer_ns() - t0 > 1000000000ull) { *abort_flag = 1; break; }
+    }
     __syncwarp();
   } else {
     // ------------------------------------------- dequantizers (warps 2..5)
