@@ -383,6 +383,98 @@ static aq_status check_gather(const int32_t* lhs, const int32_t* rhs, int64_t n_
   return AQ_OK;
 }
 
+// Expert grouping of a gather: the pairs that share weight matrix e, up to
+// 16 / M of them per problem, become one problem of Mb rows (the largest
+// group's rows; smaller groups are padded with zero rows).  Row maps index x
+// as [x_batch * M, K] and y as [n_pairs * M, N].
+struct GatherGroups {
+  bool use = false;
+  int G = 0, Mb = 0;
+  std::vector<int64_t> expert;          // weight matrix of each group
+  std::vector<int32_t> xmap, ymap;      // G * Mb rows each
+};
+
+static GatherGroups group_pairs(const int32_t* lhs, const int32_t* rhs, int64_t n_pairs,
+                                int64_t M, int64_t N, int64_t K, int64_t x_batch) {
+  GatherGroups gg;
+  const int64_t per = 16 / M;                              // pairs per problem
+  if (per < 2 || (K * 2) % 16 || (N * 2) % 16 || n_pairs > 65536 || x_batch * M > INT32_MAX)
+    return gg;
+  // pairs ordered by weight matrix (stable: pair order within a matrix)
+  std::vector<int64_t> order((size_t)n_pairs);
+  for (int64_t i = 0; i < n_pairs; ++i) order[(size_t)i] = i;
+  auto mat = [&](int64_t i) { return rhs ? (int64_t)rhs[i] : i; };
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int64_t a, int64_t b) { return mat(a) < mat(b); });
+  std::vector<std::vector<int64_t>> groups;
+  for (size_t q = 0; q < order.size();) {
+    const int64_t e = mat(order[q]);
+    std::vector<int64_t> g;
+    while (q < order.size() && mat(order[q]) == e && (int64_t)g.size() < per) g.push_back(order[q++]);
+    gg.expert.push_back(e);
+    groups.push_back(std::move(g));
+  }
+  gg.G = (int)groups.size();
+  if (gg.G >= n_pairs) return gg;                          // nothing shared: no gain
+  for (auto& g : groups) gg.Mb = std::max(gg.Mb, (int)(g.size() * M));
+  gg.xmap.assign((size_t)gg.G * gg.Mb, -1);
+  gg.ymap.assign((size_t)gg.G * gg.Mb, -1);
+  for (int gi = 0; gi < gg.G; ++gi)
+    for (size_t q = 0; q < groups[(size_t)gi].size(); ++q) {
+      const int64_t i = groups[(size_t)gi][q];
+      const int64_t l = lhs ? lhs[i] : i;
+      for (int64_t m = 0; m < M; ++m) {
+        const size_t row = (size_t)gi * gg.Mb + q * M + m;
+        gg.xmap[row] = (int32_t)(l * M + m);
+        gg.ymap[row] = (int32_t)(i * M + m);
+      }
+    }
+  gg.use = true;
+  return gg;
+}
+
+static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Workspace of the grouped path: the batch's own workspace first (counters in
+// the first 64 KB), then the gathered x and the grouped y.
+static aq_status run_grouped(const GatherGroups& gg, const void* x, const void* w_q,
+                             const void* scales, const void* biases, void* y, int64_t M,
+                             int64_t N, int64_t K, int bits, int group_size, aq_mode mode,
+                             aq_dtype dtype, void* workspace, size_t workspace_bytes,
+                             aq_stream_t stream) {
+  const int64_t G = gg.G, Mb = gg.Mb;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  std::vector<aq_qmv_problem> Q((size_t)G);
+  for (int64_t g = 0; g < G; ++g) {
+    Q[(size_t)g] = gather_pair(x, w_q, scales, biases, y, 0, gg.expert[(size_t)g], 0, Mb, N, K,
+                               bits, group_size, mode);
+  }
+  const size_t need_b = aq_qmv_batched_workspace_size(Q.data(), (int)G, Mb, bits, group_size, mode);
+  const size_t off_x = align256(std::max<size_t>(65536, need_b));
+  const size_t off_y = off_x + align256((size_t)(G * Mb * K) * 2);
+  const size_t need = off_y + align256((size_t)(G * Mb * N) * 2);
+  if (!workspace || workspace_bytes < need) return AQ_ERR_WORKSPACE;
+  for (int64_t g = 0; g < G; ++g) {
+    Q[(size_t)g].x = ws + off_x + (size_t)(g * Mb * K) * 2;
+    Q[(size_t)g].y = ws + off_y + (size_t)(g * Mb * N) * 2;
+  }
+  aq_status st = cuda_status(aq::launch_row_copy(x, ws + off_x, gg.xmap.data(), (int)(G * Mb),
+                                                 K * 2, false, (cudaStream_t)stream),
+                             "aq_gather_qmm row gather");
+  if (st != AQ_OK) return st;
+  // The batch reads the gathered x that the launch above writes: no input
+  // prefetch for this thread's inner call.
+  const int input_prefetch = g_input_prefetch;
+  g_input_prefetch = 0;
+  st = aq_qmv_batched(Q.data(), (int)G, Mb, bits, group_size, mode, dtype, workspace, off_x,
+                      stream);
+  g_input_prefetch = input_prefetch;
+  if (st != AQ_OK) return st;
+  return cuda_status(aq::launch_row_copy(ws + off_y, y, gg.ymap.data(), (int)(G * Mb), N * 2,
+                                         true, (cudaStream_t)stream),
+                     "aq_gather_qmm row scatter");
+}
+
 aq_status aq_gather_qmm(const void* x, const void* w_q, const void* scales, const void* biases,
                         const int32_t* lhs_indices, const int32_t* rhs_indices, void* y,
                         int64_t n_pairs, int64_t M, int64_t N, int64_t K, int64_t x_batch,
@@ -403,10 +495,19 @@ aq_status aq_gather_qmm(const void* x, const void* w_q, const void* scales, cons
                                i, M, N, K, bits, group_size, mode);
   // Decode-sized pairs whose matrices the batched decode kernels take run as
   // one batch (the unit scheduler walks every pair's row tiles and K-slices);
-  // the others, and M > 16, run one call per pair.
-  if (M <= 16 && check_batch(P.data(), (int)n_pairs, M, bits, group_size, mode, dtype) == AQ_OK)
+  // pairs that share a weight matrix are grouped into one problem first when
+  // that saves weight reads.  The others, and M > 16, run one call per pair.
+  if (M <= 16 && check_batch(P.data(), (int)n_pairs, M, bits, group_size, mode, dtype) == AQ_OK) {
+    GatherGroups gg = group_pairs(lhs_indices, rhs_indices, n_pairs, M, N, K, x_batch);
+    if (gg.use) {
+      st = run_grouped(gg, x, w_q, scales, biases, y, M, N, K, bits, group_size, mode, dtype,
+                       workspace, workspace_bytes, stream);
+      if (st != AQ_ERR_WORKSPACE) return st;
+      g_err[0] = 0;                                        // too small for grouping: per pair
+    }
     return aq_qmv_batched(P.data(), (int)n_pairs, M, bits, group_size, mode, dtype, workspace,
                           workspace_bytes, stream);
+  }
   g_err[0] = 0;
   for (int64_t i = 0; i < n_pairs; ++i) {
     const aq_qmv_problem& q = P[(size_t)i];
@@ -432,8 +533,16 @@ size_t aq_gather_qmm_workspace_size(int64_t n_pairs, int64_t M, int64_t N, int64
   // depends on the shapes only) and one call per pair.
   const void* a = reinterpret_cast<const void*>((uintptr_t)1 << 20);
   std::vector<aq_qmv_problem> P((size_t)n_pairs, aq_qmv_problem{a, a, a, a, const_cast<void*>(a), N, K});
-  return std::max(aq_qmv_batched_workspace_size(P.data(), (int)n_pairs, M, bits, group_size, mode),
-                  aq_workspace_size(AQ_OP_QMV, M, N, K, bits, group_size, mode, 1));
+  size_t need = std::max(aq_qmv_batched_workspace_size(P.data(), (int)n_pairs, M, bits, group_size, mode),
+                         aq_workspace_size(AQ_OP_QMV, M, N, K, bits, group_size, mode, 1));
+  // the expert-grouped path: at most n_pairs problems of at most 16 rows
+  if (16 / M >= 2) {
+    const size_t b16 = aq_qmv_batched_workspace_size(P.data(), (int)n_pairs, 16, bits, group_size, mode);
+    need = std::max(need, align256(std::max<size_t>(65536, b16)) +
+                              align256((size_t)(n_pairs * 16 * K) * 2) +
+                              align256((size_t)(n_pairs * 16 * N) * 2));
+  }
+  return need;
 }
 
 aq_status aq_qmm_nt(const void* x, const void* w_q, const void* scales, const void* biases,

@@ -14,6 +14,11 @@ size_t qmm_nt_workspace(int64_t M, int64_t N, int64_t K, int bits);
 cudaError_t launch_qmm_nt(const void* x, const void* w_q, const void* scales, const void* biases,
                           void* y, int64_t M, int64_t N, int64_t K, int bits, int gs, int mode,
                           int dtype, void* workspace, cudaStream_t st);
+// Row gather / scatter of aq_gather_qmm's expert grouping (gather.cu): row
+// maps of up to kGatherMapRows rows travel as kernel parameters.
+constexpr int kGatherMapRows = 960;
+cudaError_t launch_row_copy(const void* src, void* dst, const int32_t* map, int rows,
+                            int64_t bytes, bool scatter, cudaStream_t st);
 cudaError_t launch_quantize_dequantize_fp(const void* w, void* out, int64_t N, int64_t K, int bits,
                                           int gs, int dtype, cudaStream_t st);
 cudaError_t launch_dequantize(const void* w_q, const void* scales, const void* biases,

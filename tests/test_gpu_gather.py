@@ -93,3 +93,24 @@ def test_gather_moe_decode_many_pairs():
     torch.cuda.synchronize()
     assert api.lib().aq_device_errors() == 0
     _check(x, wq, s, b, lhs, rhs, y, bits, gs, dt)
+
+
+@pytest.mark.parametrize("M", [1, 2, 5])
+def test_gather_grouped_by_expert(M):
+    """Pairs that share an expert run as one problem (x rows gathered, y rows
+    scattered back): one expert with more pairs than a problem holds (split
+    into several groups, the last padded with zero rows), a permuted x order,
+    and the counter area of the workspace left zero."""
+    dt, bits, gs = 1, 4, 64
+    Bx, E, N, K = 6, 3, 384, 1024
+    wq, s, b = _experts(E, N, K, bits, gs, dt, seed=300 + M)
+    x = to_dev(normal((Bx, M, K), 1.0, dt, gen(400 + M)))
+    rng = np.random.default_rng(M)
+    rhs = [0] * 20 + [2] * 3 + [1]
+    lhs = [int(v) for v in rng.integers(0, Bx, len(rhs))]
+    ws = api.Workspace()
+    y = api.aq_gather_qmm(x, wq, s, b, lhs, rhs, bits, gs, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.lib().aq_device_errors() == 0
+    assert int(ws.get(x.device, 1)[:65536].count_nonzero()) == 0
+    _check(x, wq, s, b, lhs, rhs, y, bits, gs, dt)
