@@ -388,7 +388,7 @@ def side_lines(torch, api, inputs, dev, stream, hbm, tf_peak):
     del wcs
     # --- gather (aq_gather_qmm): a mixture-of-experts decode step, 8 experts
     # of 1408 x 2048 (bf16, 4-bit g64), 48 token rows routed to 2 experts each:
-    # 96 pairs, each pair streaming its expert's weights (the pair path)
+    # 96 pairs, grouped by expert (each expert streamed once per call)
     E, NE, KE, TOK = 8, 1408, 2048, 48
     qs = [api.aq_quantize(inputs.normal((NE, KE), 0.02, 1, inputs.gen(90 + e)).to(dev), 4, 64)
           for e in range(E)]
@@ -402,10 +402,13 @@ def side_lines(torch, api, inputs, dev, stream, hbm, tf_peak):
     t = graph_time_ms(torch, stream, lambda: api.aq_gather_qmm(xg, wq_e, s_e, b_e, lhs, rhs, 4, 64,
                                                                out=yg), 5)
     pair_bytes = NE * KE // 2 + 4 * NE * (KE // 64) + 2 * KE + 2 * NE
+    expert_bytes = E * (NE * KE // 2 + 4 * NE * (KE // 64)) + len(lhs) * 2 * (KE + NE)
     out["gather_moe_decode_96pairs"] = {
         "us_per_call": round(t * 1e3, 2),
-        "gbs_pair_bytes": round(len(lhs) * pair_bytes / (t * 1e-3) / 1e9, 1),
-        "note": "each pair streams its expert (8 experts read 12 times each on average)"}
+        "gbs_expert_bytes": round(expert_bytes / (t * 1e-3) / 1e9, 1),
+        "gbs_pair_equivalent": round(len(lhs) * pair_bytes / (t * 1e-3) / 1e9, 1),
+        "note": "pairs grouped by expert: 8 problems of up to 16 rows, x rows gathered and "
+                "y rows scattered by two copy kernels"}
     del wq_e, s_e, b_e
     # --- non-transposed product (aq_qmm_nt, dy . W): the down projection's
     # weight (2048 x 8192, bf16, 4-bit g64), x [M, 2048] -> y [M, 8192];
