@@ -158,14 +158,23 @@ def dist_setup():
     return world, rank, local
 
 
-def max_over_ranks(v, world):
+def max_over_ranks(v, world, device="cuda"):
+    """The largest of the ranks' values (a step time: the job is as slow as
+    its slowest rank).  `device`: where the collective's tensor lives (the
+    process group's backend: cuda for nccl, cpu for gloo)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_gbs(world, bytes_per_rank_step, ms_per_step):
+    """Whole-job throughput of `world` replicas, each streaming
+    bytes_per_rank_step per step, over the max-over-ranks step time."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
 
 
 def barrier(world):
@@ -549,7 +558,7 @@ def main():
     ms = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms, world)
     step_bytes = n_layers * sum(layer_bytes(M) for M in QMV_M)
-    value = world * step_bytes / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, ms)
 
     # Per-M views of the batched step.
     per_m = {}
@@ -609,7 +618,7 @@ def main():
         c.record(stream)
         torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a.elapsed_time(c) / args.steps, world)
-    e2e = {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+    e2e = {"value": round(whole_job_gbs(world, step_bytes, e2e_ms), 1), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # Dominant kernel: every launch of the step is qmv_mma_kernel (4-bit
