@@ -17,7 +17,7 @@ import numpy as np
 from .build_oracle import build as _build
 
 F16, BF16 = 0, 1
-AFFINE, FP4 = 0, 1
+AFFINE, FP4, MXFP8 = 0, 1, 2
 
 _lib = None
 
@@ -44,6 +44,8 @@ def lib():
             getattr(_lib, name).restype = I
         _lib.orc_quantize_fp4.argtypes = [P, I64, I64, I, I, P, P]
         _lib.orc_quantize_fp4.restype = I
+        _lib.orc_quantize_mxfp8.argtypes = [P, I64, I64, I, P, P]
+        _lib.orc_quantize_mxfp8.restype = I
         _lib.orc_quantize_dequantize_fp.argtypes = [P, I64, I64, I, I, I, P]
         _lib.orc_quantize_dequantize_fp.restype = I
         _lib.orc_quantize.argtypes = [P, I64, I64, I, I, I, P, P, P]
@@ -143,6 +145,17 @@ def quantize_fp4(w16, gs, dt):
     return codes, scales
 
 
+def quantize_mxfp8(w16, dt):
+    """MXFP8 weights: w16 [N, K] uint16 T patterns -> (codes [N, K] E4M3
+    bytes, scales [N, K/32] E8M0 bytes)."""
+    w16 = _c(w16, np.uint16)
+    N, K = w16.shape
+    codes = np.zeros((N, K), np.uint8)
+    scales = np.zeros((N, K // 32), np.uint8)
+    _check(lib().orc_quantize_mxfp8(_p(w16), N, K, dt, _p(codes), _p(scales)), "quantize_mxfp8")
+    return codes, scales
+
+
 def quantize_dequantize_fp(w16, bits, gs, dt):
     """[P4] fp_quantize_dequantize: w16 [N, K] uint16 T patterns -> the fake-
     quantized [N, K] T patterns (E2M1 elements for bits 4, E4M3 for bits 8;
@@ -172,7 +185,7 @@ def unpack(wq, N, K, bits):
 def dequantize(wq, scales, biases, N, K, bits, gs, mode, dt):
     """-> (w_hat fp64 exact [N, K], w_t uint16 T patterns [N, K])."""
     wq = _c(wq, np.uint8)
-    scales = _c(scales, np.uint8 if mode == FP4 else np.uint16)
+    scales = _c(scales, np.uint8 if mode in (FP4, MXFP8) else np.uint16)
     biases = None if biases is None else _c(biases, np.uint16)
     wh = np.zeros((N, K), np.float64)
     wt = np.zeros((N, K), np.uint16)
@@ -187,7 +200,7 @@ def qmm(x16, wq, scales, biases, N, bits, gs, mode, dt, w_in_t=False):
     x16 = _c(x16, np.uint16)
     M, K = x16.shape
     wq = _c(wq, np.uint8)
-    scales = _c(scales, np.uint8 if mode == FP4 else np.uint16)
+    scales = _c(scales, np.uint8 if mode in (FP4, MXFP8) else np.uint16)
     biases = None if biases is None else _c(biases, np.uint16)
     y = np.zeros((M, N), np.float64)
     den = np.zeros((M, N), np.float64)
@@ -227,7 +240,7 @@ def qmm_sampled(x16, wq, scales, biases, N, bits, gs, mode, dt, ms, ns, w_in_t=F
     x16 = _c(x16, np.uint16)
     M, K = x16.shape
     wq = _c(wq, np.uint8)
-    scales = _c(scales, np.uint8 if mode == FP4 else np.uint16)
+    scales = _c(scales, np.uint8 if mode in (FP4, MXFP8) else np.uint16)
     biases = None if biases is None else _c(biases, np.uint16)
     ms = _c(ms, np.int64)
     ns = _c(ns, np.int64)

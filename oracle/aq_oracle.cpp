@@ -22,7 +22,9 @@
 //        extract_bits, FP4_LUT, dequantize_scale (E8M0 / FP8 scales), fp_qmm_t,
 //        and the FP4 quantizer's steps: to_fp8_e8m0, to_fp4_e2m1 and
 //        fp_quantize_dequantize (scale = absmax / 6, or / 448 for 8-bit
-//        elements), which QQMatmul applies to x before the FP4 matmul.
+//        elements), which QQMatmul applies to x before the FP4 matmul; the
+//        8-bit branch of fp_qmm_t / fp_qmm_dispatch_typed (MXFP8 weights:
+//        E4M3 elements, E8M0 scales at group 32).
 //
 // Precision.  The quantizer runs in fp32, in the order the quantize routine of
 // [P4] takes its steps, because its codes, scales and biases are fixed by fp32
@@ -44,7 +46,7 @@
 namespace {
 
 enum { DT_F16 = 0, DT_BF16 = 1 };
-enum { MODE_AFFINE = 0, MODE_FP4 = 1 };
+enum { MODE_AFFINE = 0, MODE_FP4 = 1, MODE_MXFP8 = 2 };
 
 // ---------------------------------------------------------------- T <-> real
 // IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits.
@@ -259,7 +261,7 @@ void dequant_row(const uint8_t* wq, const void* scales, const uint16_t* biases,
         out[k] = sc * (double)read_code(row, k, bits) + bi;
       }
     }
-  } else {
+  } else if (mode == MODE_FP4) {
     const uint8_t* row = wq + n * (K / 2);
     const uint8_t* s = (const uint8_t*)scales + n * G;
     for (int64_t g = 0; g < G; ++g) {
@@ -267,6 +269,18 @@ void dequant_row(const uint8_t* wq, const void* scales, const uint16_t* biases,
       for (int64_t j = 0; j < gs; ++j) {
         int64_t k = g * gs + j;
         out[k] = e2m1_value(read_code(row, k, 4)) * sc;
+      }
+    }
+  } else {
+    // MXFP8 ([P4] fp_qmm_t, bits 8): one E4M3 byte per element (FromFP8) times
+    // the group's E8M0 scale as T.
+    const uint8_t* row = wq + n * K;
+    const uint8_t* s = (const uint8_t*)scales + n * G;
+    for (int64_t g = 0; g < G; ++g) {
+      double sc = fp_scale_in_t(s[g], gs, dt);
+      for (int64_t j = 0; j < gs; ++j) {
+        int64_t k = g * gs + j;
+        out[k] = e4m3_value(row[k]) * sc;
       }
     }
   }
@@ -287,6 +301,8 @@ int check_common(int64_t N, int64_t K, int bits, int gs, int mode, int dt) {
     if (!valid_bits(bits) || !valid_group(gs)) return 1;
   } else if (mode == MODE_FP4) {
     if (bits != 4 || (gs != 16 && gs != 32)) return 1;
+  } else if (mode == MODE_MXFP8) {
+    if (bits != 8 || gs != 32) return 1;               // [P4] fp_qmm_dispatch_typed: bits 8 -> group 32
   } else {
     return 1;
   }
@@ -359,6 +375,37 @@ int orc_quantize_fp4(const uint16_t* w, int64_t N, int64_t K, int gs, int dt, ui
         uint8_t& dst = codes[n * (K / 2) + k / 2];
         if (k % 2 == 0) dst = (uint8_t)((dst & 0xF0) | c);
         else dst = (uint8_t)((dst & 0x0F) | (c << 4));
+      }
+    }
+  }
+  return 0;
+}
+
+// MXFP8 quantizer: the steps of [P4] fp_quantize_dequantize for 8-bit
+// elements up to the codes and the scale byte.  w is [N, K] T; codes is
+// [N, K] E4M3 bytes; scales is [N, K/32] E8M0 bytes.  Per group of 32, fp32:
+//   absmax (NaN ignored), scale = absmax / 448, byte = to_fp8_e8m0(scale),
+//   s = the byte decoded, code_j = ToFP8(s == 0 ? 0 : w_j / s)
+int orc_quantize_mxfp8(const uint16_t* w, int64_t N, int64_t K, int dt, uint8_t* codes,
+                       uint8_t* scales) {
+  if (dt != DT_F16 && dt != DT_BF16) return 1;
+  if (N < 0 || K < 0 || K % 32) return 1;
+  const int64_t G = K / 32;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < G; ++g) {
+      const uint16_t* wg = w + n * K + g * 32;
+      float amax = -std::numeric_limits<float>::infinity();
+      for (int j = 0; j < 32; ++j) {
+        const float a = std::fabs(t_to_float(wg[j], dt));
+        amax = (amax < a) ? a : amax;
+      }
+      const float scale = amax / 448.0f;
+      const unsigned byte = e8m0_encode(scale);
+      const float sdec = (float)e8m0_value(byte);
+      scales[n * G + g] = (uint8_t)byte;
+      for (int j = 0; j < 32; ++j) {
+        const float el = sdec == 0.0f ? 0.0f : t_to_float(wg[j], dt) / sdec;
+        codes[n * K + g * 32 + j] = (uint8_t)e4m3_encode(el);
       }
     }
   }

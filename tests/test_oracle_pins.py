@@ -743,3 +743,57 @@ def test_qmm_nt_is_x_times_w_hat_by_brute_force(bits):
         for k in range(K):
             want = sum(x[m, n] * (s[n, k // gs] * q[n, k] + b[n, k // gs]) for n in range(N))
             assert abs(y[m, k] - want) <= 1e-12 * (1 + abs(want)), (m, k)
+
+
+# ------------------------------------------------------------------- MXFP8
+
+def test_mxfp8_dequantize_is_e4m3_times_e8m0():
+    """Every E4M3 byte under several E8M0 scales: the value torch's
+    float8_e4m3fn decode gives, times 2^(s - 127) (the scale as bf16)."""
+    N, K = 4, 256
+    codes = np.tile(np.arange(256, dtype=np.uint8), (N, 1))
+    sc = np.array([[127, 120, 131, 127, 100, 140, 127, 127]] * N, np.uint8)
+    wh, _ = oracle.dequantize(codes, sc, None, N, K, 8, 32, oracle.MXFP8, BF16)
+    dec = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    want = dec * np.repeat(np.ldexp(1.0, sc.astype(np.int64) - 127), 32, axis=1)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(wh), nan)
+    assert np.array_equal(wh[~nan], want[~nan])
+
+
+def test_mxfp8_quantize_codes_match_torch_float8():
+    """Groups whose absmax is 448 * 2^k: the scale byte is 127 + k and every
+    code is torch's float8_e4m3fn encoding (round to nearest even) of w / 2^k."""
+    rng = np.random.default_rng(8)
+    rows, ks = [], []
+    for k in (-4, 0, 3):
+        v = rng.uniform(-1.0, 1.0, 64) * 448.0
+        v[0], v[40] = 448.0, -448.0
+        rows.append(v * 2.0 ** k)
+        ks.append(k)
+    w16 = f64_to_u16(np.array(rows), BF16)
+    codes, sc = oracle.quantize_mxfp8(w16, BF16)
+    w = u16_to_f64(w16, BF16)
+    for i, k in enumerate(ks):
+        assert list(sc[i]) == [127 + k, 127 + k]
+        want = torch.from_numpy((w[i] / 2.0 ** k).astype(np.float32)).to(
+            torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(codes[i], want), i
+
+
+def test_mxfp8_qmm_is_x_times_w_hat():
+    rng = np.random.default_rng(9)
+    M, N, K = 3, 6, 128
+    codes = rng.integers(0, 0x7E, size=(N, K)).astype(np.uint8)   # finite E4M3 bytes
+    sc = rng.integers(118, 136, size=(N, K // 32)).astype(np.uint8)
+    x16 = f64_to_u16(rng.standard_normal((M, K)), BF16)
+    y, _ = oracle.qmm(x16, codes, sc, None, N, 8, 32, oracle.MXFP8, BF16)
+    dec = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    W = dec * np.repeat(np.ldexp(1.0, sc.astype(np.int64) - 127), 32, axis=1)
+    assert np.allclose(y, u16_to_f64(x16, BF16) @ W.T, rtol=1e-12, atol=1e-12)
+
+
+def test_mxfp8_mode_rules():
+    with pytest.raises(Exception):
+        oracle.dequantize(np.zeros((1, 64), np.uint8), np.zeros((1, 4), np.uint8), None, 1, 64, 8,
+                          16, oracle.MXFP8, BF16)                  # group 32 only
