@@ -63,6 +63,8 @@ _I32P = ctypes.POINTER(ctypes.c_int32)
 SIGNATURES["aq_gather_qmm"] = (_I, [_P, _P, _P, _P, _I32P, _I32P, _P, _I64, _I64, _I64, _I64, _I64,
                                     _I64, _I, _I, _I, _I, _P, _SZ, _P])
 SIGNATURES["aq_gather_qmm_workspace_size"] = (_SZ, [_I64, _I64, _I64, _I64, _I, _I, _I])
+SIGNATURES["aq_testing_gather_groups"] = (_I, [_I32P, _I32P, _I64, _I64, _I64, _I64, _I64, _I32P,
+                                               _I32P, _I64, ctypes.POINTER(_I)])
 
 _lib = None
 

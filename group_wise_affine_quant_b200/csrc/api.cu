@@ -625,6 +625,20 @@ aq_status aq_qqmm(const void* x, const void* w_q, const void* scales, void* y, i
   return st;
 }
 
+int aq_testing_gather_groups(const int32_t* lhs_indices, const int32_t* rhs_indices,
+                             int64_t n_pairs, int64_t M, int64_t N, int64_t K, int64_t x_batch,
+                             int32_t* xmap, int32_t* ymap, int64_t map_rows, int* rows_per_group) {
+  const GatherGroups gg = group_pairs(lhs_indices, rhs_indices, n_pairs, M, N, K, x_batch);
+  if (!gg.use) return 0;
+  if (rows_per_group) *rows_per_group = gg.Mb;
+  const int64_t rows = (int64_t)gg.G * gg.Mb;
+  for (int64_t i = 0; i < rows && i < map_rows; ++i) {
+    if (xmap) xmap[i] = gg.xmap[(size_t)i];
+    if (ymap) ymap[i] = gg.ymap[(size_t)i];
+  }
+  return gg.G;
+}
+
 void aq_testing_set_wait_limit_ns(uint64_t ns) { aq::testing_set_mv_wait_ns(ns); }
 void aq_testing_set_start_delay_ns(uint64_t ns) { aq::testing_set_mv_delay_ns(ns); }
 void aq_testing_set_qmv_kernel(int which) { g_qmv_kernel.store(which, std::memory_order_relaxed); }
