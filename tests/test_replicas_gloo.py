@@ -48,3 +48,13 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.0, 1) == 3.0
     assert bench.whole_job_gbs(1, 1e9, 1.0) == pytest.approx(1000.0)
+
+
+def test_traffic_record_matches_current_decode_sources():
+    """The decode kernel's committed DRAM-traffic ratio applies only while its
+    sources hash to the profiled version; the committed record does."""
+    import bench
+    r = bench.traffic_for("qmv_mma_kernel", "decode-stack-batched")
+    assert r is not None and 0.9 < r < 1.1
+    assert bench.traffic_for("qmv_mma_kernel", "another-workload") is None
+    assert bench.traffic_for("no_such_kernel", "decode-stack-batched") is None
