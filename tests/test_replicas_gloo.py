@@ -50,11 +50,22 @@ def test_single_rank_is_identity():
     assert bench.whole_job_gbs(1, 1e9, 1.0) == pytest.approx(1000.0)
 
 
-def test_traffic_record_matches_current_decode_sources():
-    """The decode kernel's committed DRAM-traffic ratio applies only while its
-    sources hash to the profiled version; the committed record does."""
+def test_traffic_record_applies_only_to_the_profiled_sources(tmp_path, monkeypatch):
+    """A kernel's DRAM-traffic ratio (profiles/traffic.json) is used only while
+    its sources hash to the profiled version and the workload matches."""
+    import hashlib
+    import json
     import bench
-    r = bench.traffic_for("qmv_mma_kernel", "decode-stack-batched")
-    assert r is not None and 0.9 < r < 1.1
-    assert bench.traffic_for("qmv_mma_kernel", "another-workload") is None
-    assert bench.traffic_for("no_such_kernel", "decode-stack-batched") is None
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    (tmp_path / "profiles").mkdir()
+    rec = {"k": {"workload": "w", "sources": ["k.cu"],
+                 "sources_sha256_16": hashlib.sha256(b"kernel v1").hexdigest()[:16],
+                 "dram_bytes_per_algorithmic_byte": 0.99}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_for("k", "w") == 0.99
+    assert bench.traffic_for("k", "other") is None
+    assert bench.traffic_for("missing", "w") is None
+    src.write_text("kernel v2")                         # the kernel changed since the capture
+    assert bench.traffic_for("k", "w") is None
