@@ -224,10 +224,14 @@ AQ_API aq_status aq_qmm_nt(const void* x, const void* w_q, const void* scales, c
  *            AQ_ERR_INVALID_ARG.
  * Each pair's result is the one aq_qmv (M <= 16) or aq_qmm defines.  Pairs of
  * decode size whose matrices meet aq_qmv_batched's conditions run as one
- * batch (one launch per 40 pairs); the others run one call per pair, and
- * every pair's pointers must then meet that call's alignment rules (the
- * error names the pair).  Workspace: aq_gather_qmm_workspace_size bytes,
- * under aq_qmv's rules.
+ * batch (one launch per 40 problems); when pairs share a weight matrix and
+ * M <= 8 (and K, N are multiples of 8), up to 16 / M of them form one
+ * problem first: their x rows are copied together into the workspace and
+ * the problem's y rows copied back (two extra launches), so each matrix is
+ * streamed once per call.  The other pairs run one call per pair, and every
+ * pair's pointers must then meet that call's alignment rules (the error
+ * names the pair).  Workspace: aq_gather_qmm_workspace_size bytes, under
+ * aq_qmv's rules.
  */
 AQ_API aq_status aq_gather_qmm(const void* x, const void* w_q, const void* scales,
                                const void* biases, const int32_t* lhs_indices,
